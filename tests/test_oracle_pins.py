@@ -1,0 +1,313 @@
+"""Pins for the float64 oracle: what the pages and the mathematics fix.
+
+None of these tests retypes the oracle's formulas.  Each checks the oracle
+against something independent of it:
+* hand-worked closed forms (tests/golden/hand_worked.json);
+* library routines for special cases (torch float64 scaled_dot_product_attention,
+  rms_norm, bfloat16 widening);
+* invariants the pages state: RoPE scores depend only on m - n, rotation keeps
+  the norm, softmax rows are a probability vector, GQA with Hkv = Hq is MHA and
+  equals MHA on repeat_interleave'd K/V, cached decode equals full recomputation;
+* the complex-number form of RoPE (each pair is a complex number multiplied by
+  exp(i p theta)), a derivation different from the oracle's pairwise rotation.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "hand_worked.json")
+MATH_NS = {"cos": math.cos, "sin": math.sin, "exp": math.exp, "sqrt": math.sqrt}
+
+
+def _bits(x):
+    """Float values (exact in bf16) -> uint16 bf16 bit patterns."""
+    t = torch.tensor(np.asarray(x, dtype=np.float32)).to(torch.bfloat16)
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
+def _eval(e):
+    return np.vectorize(lambda s: float(eval(s, {"__builtins__": {}}, MATH_NS)))(np.asarray(e))
+
+
+def _rand_bits(rng, *shape):
+    return _bits(rng.standard_normal(shape).astype(np.float32))
+
+
+# ---------------------------------------------------------------------------
+# hand-worked closed forms
+# ---------------------------------------------------------------------------
+def _golden_cases():
+    with open(GOLDEN) as f:
+        return json.load(f)["cases"]
+
+
+@pytest.mark.parametrize("case", _golden_cases(), ids=lambda c: c["name"])
+def test_hand_worked(case):
+    want = _eval(case["expect"])
+    op = case["op"]
+    if op == "rope":
+        x = np.asarray(case["x"], dtype=np.float64)
+        got = oracle.rope(x, np.asarray(case["pos"]))
+    elif op == "rmsnorm":
+        got = oracle.rmsnorm(np.asarray(case["x"], dtype=np.float64), case["eps"])
+    elif op == "prefill":
+        got, _, _ = oracle.prefill(_bits(case["q"]), _bits(case["k"]), _bits(case["v"]),
+                                   case["qk_norm"])
+    elif op == "decode":
+        got, _ = oracle.decode_step(_bits(case["q"]), _bits(case["k"]), _bits(case["v"]),
+                                    _bits(case["k_cache"]), _bits(case["v_cache"]),
+                                    case["lens"], case["qk_norm"])
+    else:
+        raise AssertionError(op)
+    np.testing.assert_allclose(got, want, rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# bf16 widening and RMSNorm against library routines
+# ---------------------------------------------------------------------------
+def test_bf16_widening_matches_torch():
+    rng = np.random.default_rng(1)
+    raw = rng.integers(0, 1 << 16, size=4096, dtype=np.uint16)
+    raw = raw[~np.isnan(torch.tensor(raw.view(np.int16)).view(torch.bfloat16).float().numpy())]
+    want = torch.tensor(raw.view(np.int16)).view(torch.bfloat16).to(torch.float64).numpy()
+    np.testing.assert_array_equal(oracle.bf16_to_f64(raw), want)
+
+
+@pytest.mark.parametrize("D", [4, 64, 96, 128])
+def test_rmsnorm_matches_library(D):
+    rng = np.random.default_rng(D)
+    x = rng.standard_normal((37, D)) * rng.uniform(0.01, 10, size=(37, 1))
+    want = F.rms_norm(torch.tensor(x), (D,), eps=1e-6).numpy()
+    np.testing.assert_allclose(oracle.rmsnorm(x, 1e-6), want, rtol=1e-13, atol=1e-14)
+
+
+def test_rmsnorm_output_mean_square():
+    # mean(y^2) = ms / (ms + eps) exactly, ms = mean(x^2)
+    rng = np.random.default_rng(2)
+    x = rng.standard_normal((16, 128)) * 1e-3
+    eps = 1e-6
+    y = oracle.rmsnorm(x, eps)
+    ms = (x ** 2).mean(-1)
+    np.testing.assert_allclose((y ** 2).mean(-1), ms / (ms + eps), rtol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# RoPE
+# ---------------------------------------------------------------------------
+def _rope_complex(x, pos, base=10000.0, interleaved=False):
+    """RoPE as complex multiplication: pair i is z_i = x_a + i x_b, z_i *= e^{i p th_i}."""
+    D = x.shape[-1]
+    half = D // 2
+    if interleaved:
+        z = x[..., 0::2] + 1j * x[..., 1::2]
+    else:
+        z = x[..., :half] + 1j * x[..., half:]
+    th = base ** (-np.arange(0, D, 2, dtype=np.float64) / D)
+    z = z * np.exp(1j * np.asarray(pos, dtype=np.float64)[..., None, None] * th)
+    out = np.empty_like(x)
+    if interleaved:
+        out[..., 0::2], out[..., 1::2] = z.real, z.imag
+    else:
+        out[..., :half], out[..., half:] = z.real, z.imag
+    return out
+
+
+@pytest.mark.parametrize("interleaved", [False, True])
+@pytest.mark.parametrize("D", [2, 8, 64, 96, 128])
+def test_rope_equals_complex_rotation(D, interleaved):
+    rng = np.random.default_rng(D)
+    x = rng.standard_normal((50, 3, D))
+    pos = rng.integers(0, 5000, size=50)
+    got = oracle.rope(x, pos, interleaved=interleaved)
+    np.testing.assert_allclose(got, _rope_complex(x, pos, interleaved=interleaved),
+                               rtol=0, atol=1e-11)
+
+
+def test_rope_position_zero_is_identity_and_keeps_norm():
+    rng = np.random.default_rng(3)
+    x = rng.standard_normal((20, 4, 128))
+    np.testing.assert_array_equal(oracle.rope(x, np.zeros(20, dtype=np.int64)), x)
+    y = oracle.rope(x, rng.integers(0, 4096, size=20))
+    np.testing.assert_allclose(np.linalg.norm(y, axis=-1), np.linalg.norm(x, axis=-1),
+                               rtol=1e-13)
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_rope_scores_depend_on_distance_only(D):
+    # q_m . k_n is unchanged when both positions shift by the same s.
+    rng = np.random.default_rng(4)
+    q = rng.standard_normal((1, 1, D))
+    k = rng.standard_normal((1, 1, D))
+    for m, n, s in [(5, 3, 100), (0, 0, 777), (2047, 1, 9), (10, 400, 1234)]:
+        a = (oracle.rope(q, [m]) * oracle.rope(k, [n])).sum()
+        b = (oracle.rope(q, [m + s]) * oracle.rope(k, [n + s])).sum()
+        assert abs(a - b) < 1e-10 * max(1.0, abs(a))
+    # ... and it does depend on the distance
+    a = (oracle.rope(q, [5]) * oracle.rope(k, [3])).sum()
+    c = (oracle.rope(q, [6]) * oracle.rope(k, [3])).sum()
+    assert abs(a - c) > 1e-6
+
+
+def test_norm_and_rope_commute():
+    # Unit-gain RMSNorm scales the whole vector; rotation keeps its norm.
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((30, 2, 128))
+    pos = rng.integers(0, 3000, size=30)
+    a = oracle.rope(oracle.rmsnorm(x, 1e-6), pos)
+    b = oracle.rmsnorm(oracle.rope(x, pos), 1e-6)
+    np.testing.assert_allclose(a, b, rtol=0, atol=1e-13)
+
+
+# ---------------------------------------------------------------------------
+# attention core: library special case, softmax, GQA reductions
+# ---------------------------------------------------------------------------
+def _sdpa(q, k, v, causal=True, scale=None):
+    """torch float64 SDPA on [B, T, H, D] arrays (K/V heads repeated per group)."""
+    qt = torch.tensor(q).transpose(1, 2)
+    kt = torch.tensor(k).transpose(1, 2)
+    vt = torch.tensor(v).transpose(1, 2)
+    g = qt.shape[1] // kt.shape[1]
+    kt = kt.repeat_interleave(g, dim=1)
+    vt = vt.repeat_interleave(g, dim=1)
+    o = F.scaled_dot_product_attention(qt, kt, vt, is_causal=causal, scale=scale)
+    return o.transpose(1, 2).numpy()
+
+
+@pytest.mark.parametrize("B,T,Hq,Hkv,D", [(2, 37, 4, 2, 64), (1, 130, 8, 8, 96),
+                                          (2, 19, 6, 1, 32), (1, 64, 24, 8, 128)])
+def test_attention_core_matches_library_sdpa(B, T, Hq, Hkv, D):
+    rng = np.random.default_rng(B * T + Hq)
+    q = rng.standard_normal((B, T, Hq, D))
+    k = rng.standard_normal((B, T, Hkv, D))
+    v = rng.standard_normal((B, T, Hkv, D))
+    pos = oracle.positions(0, B, T)
+    got = oracle.attention(q, k, v, pos)
+    np.testing.assert_allclose(got, _sdpa(q, k, v), rtol=0, atol=1e-12)
+
+
+def test_attention_probabilities_form_a_distribution():
+    # With v_u = e_u (one-hot), output row t is the probability vector itself.
+    rng = np.random.default_rng(6)
+    T, D = 24, 32
+    q = rng.standard_normal((1, T, 1, D)) * 3
+    k = rng.standard_normal((1, T, 1, D)) * 3
+    v = np.eye(D)[:T].reshape(1, T, 1, D)
+    p = oracle.attention(q, k, v, oracle.positions(0, 1, T))[0, :, 0, :]
+    np.testing.assert_allclose(p.sum(-1), 1.0, rtol=0, atol=1e-12)
+    assert (p >= 0).all()
+    # causal: row t puts no weight on keys after t
+    for t in range(T):
+        assert np.all(p[t, t + 1:] == 0)
+
+
+def test_first_row_returns_first_value_and_equal_keys_average():
+    rng = np.random.default_rng(7)
+    B, T, H, D = 2, 9, 3, 16
+    q = rng.standard_normal((B, T, H, D))
+    k = np.broadcast_to(rng.standard_normal((B, 1, H, D)), (B, T, H, D)).copy()
+    v = rng.standard_normal((B, T, H, D))
+    o = oracle.attention(q, k, v, oracle.positions(0, B, T))
+    np.testing.assert_array_equal(o[:, 0], v[:, 0])
+    for t in range(T):
+        np.testing.assert_allclose(o[:, t], v[:, :t + 1].mean(1), rtol=0, atol=1e-13)
+
+
+def test_gqa_reductions():
+    rng = np.random.default_rng(8)
+    B, T, D = 2, 33, 64
+    pos = oracle.positions(0, B, T)
+    # GQA equals MHA on K/V repeated per group (query head h -> K/V head h // g)
+    q = rng.standard_normal((B, T, 6, D))
+    k = rng.standard_normal((B, T, 2, D))
+    v = rng.standard_normal((B, T, 2, D))
+    got = oracle.attention(q, k, v, pos)
+    mha = oracle.attention(q, np.repeat(k, 3, axis=2), np.repeat(v, 3, axis=2), pos)
+    np.testing.assert_allclose(got, mha, rtol=0, atol=1e-14)
+    # Hkv = Hq is MHA: each head alone equals single-head attention
+    k6 = rng.standard_normal((B, T, 6, D))
+    v6 = rng.standard_normal((B, T, 6, D))
+    full = oracle.attention(q, k6, v6, pos)
+    for h in range(6):
+        one = oracle.attention(q[:, :, h:h + 1], k6[:, :, h:h + 1], v6[:, :, h:h + 1], pos)
+        np.testing.assert_array_equal(full[:, :, h:h + 1], one)
+    # Hkv = 1 is MQA: every query head reads the same K/V
+    k1, v1 = k6[:, :, :1], v6[:, :, :1]
+    mqa = oracle.attention(q, k1, v1, pos)
+    for h in range(6):
+        one = oracle.attention(q[:, :, h:h + 1], k1, v1, pos)
+        np.testing.assert_array_equal(mqa[:, :, h:h + 1], one)
+
+
+def test_row_subset_matches_full():
+    rng = np.random.default_rng(9)
+    B, T, Hq, Hkv, D = 2, 50, 4, 2, 64
+    q = rng.standard_normal((B, T, Hq, D))
+    k = rng.standard_normal((B, T, Hkv, D))
+    v = rng.standard_normal((B, T, Hkv, D))
+    pos = oracle.positions(0, B, T)
+    full = oracle.attention(q, k, v, pos)
+    rows = np.array([0, 7, 199, 399])
+    part = oracle.attention(q, k, v, pos, rows=rows)
+    flat_f = full.reshape(-1, D)
+    flat_p = part.reshape(-1, D)
+    np.testing.assert_array_equal(flat_p[rows], flat_f[rows])
+    assert np.isnan(flat_p[1]).all()
+
+
+def test_hq_not_multiple_of_hkv_is_rejected():
+    q = np.zeros((1, 2, 3, 8))
+    k = np.zeros((1, 2, 2, 8))
+    with pytest.raises(ValueError):
+        oracle.attention(q, k, k, oracle.positions(0, 1, 2))
+
+
+# ---------------------------------------------------------------------------
+# the pages' own check: decode with the cache == full recomputation
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("qk_norm", [False, True])
+def test_cached_decode_equals_full_recompute(qk_norm):
+    rng = np.random.default_rng(10)
+    B, T0, steps, Hq, Hkv, D = 2, 20, 6, 4, 2, 64
+    T = T0 + steps
+    q = _rand_bits(rng, B, T, Hq, D)
+    k = _rand_bits(rng, B, T, Hkv, D)
+    v = _rand_bits(rng, B, T, Hkv, D)
+    o_full, k_rot, v_all = oracle.prefill(q, k, v, qk_norm)
+    # prompt, then token-by-token with a float64 cache
+    Lmax = 32
+    kc = np.zeros((B, Hkv, Lmax, D))
+    vc = np.zeros((B, Hkv, Lmax, D))
+    _, k0, v0 = oracle.prefill(q[:, :T0], k[:, :T0], v[:, :T0], qk_norm)
+    kc[:, :, :T0] = k0.transpose(0, 2, 1, 3)
+    vc[:, :, :T0] = v0.transpose(0, 2, 1, 3)
+    lens = np.full(B, T0)
+    for s in range(steps):
+        t = T0 + s
+        o, knew = oracle.decode_step(q[:, t], k[:, t], v[:, t], kc, vc, lens, qk_norm)
+        np.testing.assert_allclose(o, o_full[:, t], rtol=0, atol=1e-13)
+        np.testing.assert_allclose(knew, k_rot[:, t], rtol=0, atol=1e-15)
+        kc[:, :, t] = knew
+        vc[:, :, t] = v_all[:, t]
+        lens = lens + 1
+
+
+def test_decode_ignores_slots_beyond_length():
+    rng = np.random.default_rng(11)
+    B, Hq, Hkv, D, L = 3, 4, 2, 64, 40
+    lens = np.array([5, 17, 39])
+    kc = rng.standard_normal((B, Hkv, L, D))
+    vc = rng.standard_normal((B, Hkv, L, D))
+    q, k, v = (_rand_bits(rng, B, Hq, D), _rand_bits(rng, B, Hkv, D), _rand_bits(rng, B, Hkv, D))
+    o1, _ = oracle.decode_step(q, k, v, kc, vc, lens, True)
+    for b in range(B):
+        kc[b, :, lens[b]:] = np.nan
+        vc[b, :, lens[b]:] = np.nan
+    o2, _ = oracle.decode_step(q, k, v, kc, vc, lens, True)
+    np.testing.assert_array_equal(o1, o2)
