@@ -1,0 +1,493 @@
+"""Benchmark: one attention layer of the 3.8B-style model, prefill + batched decode.
+
+One step = one pass of the whole hot path over one batch of synthetic input:
+  prefill phase  (B=8, T=2048, Hq=24, Hkv=8, D=128, QK-RMSNorm, RoPE base 1e4)
+      gqa_rope_append (q in place; rotated k and v into the cache) + gqa_prefill
+  decode step    (B=64, Hq=24, Hkv=8, D=128, cached lengths U[256, 2048], QK-norm)
+      gqa_rope_append (new token at position lens[b]) + gqa_decode over lens[b] + 1
+value = tokens processed per second (8*2048 prompt + 64 generated tokens per step,
+times the number of GPUs), timed on the device with CUDA events; the inputs of a
+step (about 0.9 GB) exceed the 126 MB L2, so no flush is needed between steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+For N > 1 launch under torch.distributed.run: every rank runs its own replica of
+the workload (the path has no exchange step), the timed region is bracketed by
+a barrier and a device synchronise, and the slowest rank's time is used.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from rope_gqa_kv_b200 import inputs  # noqa: E402
+
+METRIC = "GQA prefill TFLOP/s & KV-cache decode GB/s, tokens/s (frac of B200 peak)"
+PREFILL = inputs.BY_NAME["prefill_3p8b"]
+DECODE = inputs.BY_NAME["batched_decode"]
+WORKLOAD = ("3.8B-style attention layer: prefill B=8 T=2048 Hq=24 Hkv=8 D=128 QK-norm, "
+            "then one decode step B=64 Hq=24 Hkv=8 D=128 with cached lengths U[256,2048]")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ---------------------------------------------------------------------------
+# work accounting (algorithmic, not what the kernels happen to move)
+# ---------------------------------------------------------------------------
+def prefill_flops(w=PREFILL) -> float:
+    """4*D flops per (query, visible key, query head): QK^T and PV, causal pairs only."""
+    return 4.0 * w.D * (w.T * (w.T + 1) / 2) * w.B * w.Hq
+
+
+def decode_bytes(lens_new, w=DECODE) -> float:
+    """K and V of every visible slot, once per KV head, plus q in and o out."""
+    kv = float(np.sum(lens_new)) * w.Hkv * w.D * 2 * 2
+    return kv + 2 * w.B * w.Hq * w.D * 2
+
+
+def tokens_per_step() -> int:
+    return PREFILL.B * PREFILL.T + DECODE.B
+
+
+# ---------------------------------------------------------------------------
+# peaks, clocks, profile summary
+# ---------------------------------------------------------------------------
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed loops run."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,utilization.gpu,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.idx = device_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=5)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        sm, smax, util, reasons = [], [], [], set()
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                s, m, u = float(parts[1]), float(parts[2]), float(parts[4])
+            except ValueError:
+                continue
+            sm.append(s)
+            smax.append(m)
+            util.append(u)
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        loaded = [s for s, u in zip(sm, util) if u > 0] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in ("prefill.cu", "ptx.cuh", "common.cuh"):
+        with open(os.path.join(ROOT, "rope_gqa_kv_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic():
+    """DRAM bytes per prefill launch from the committed ncu summary, if it still
+    describes the current kernel source (else None)."""
+    p = os.path.join(ROOT, "profiles", "prefill_3p8b_ncu.txt")
+    if not os.path.exists(p):
+        return None
+    vals = {}
+    with open(p) as f:
+        for ln in f:
+            if ":" in ln:
+                k, v = ln.split(":", 1)
+                vals[k.strip()] = v.strip()
+    if vals.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+class Layer:
+    """Device-resident buffers of one replica of the workload."""
+
+    def __init__(self, dev):
+        import rope_gqa_kv_b200 as gqa
+        self.gqa = gqa
+        gqa.load()
+        self.dev = dev
+        xp = inputs.make_inputs(PREFILL)
+        xd = inputs.make_inputs(DECODE)
+        self.host_p = {k: xp[k] for k in ("q", "k", "v")}
+        q1, k1, v1 = xd["steps"][0]
+        self.host_d = {"q": q1, "k": k1, "v": v1, "lens": xd["lens"]}
+        d = lambda t: t.to(dev)  # noqa: E731
+        self.pq, self.pk, self.pv = d(xp["q"]), d(xp["k"]), d(xp["v"])
+        self.pkc, self.pvc = d(xp["k_cache"]), d(xp["v_cache"])
+        self.pout = torch.empty_like(self.pq)
+        self.dq, self.dk, self.dv = d(q1), d(k1), d(v1)
+        self.dkc, self.dvc = d(xd["k_cache"]), d(xd["v_cache"])
+        self.pos = d(xd["lens"])
+        self.lens_new = torch.empty_like(self.pos)
+        self.max_len = int(xd["lens"].max()) + 1
+        self.dout = torch.empty_like(self.dq)
+        nbytes = gqa.gqa_decode_workspace_bytes(DECODE.B, DECODE.Hq, DECODE.D, self.max_len)
+        self.ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.lens_new_host = (xd["lens"] + 1).numpy()
+        # pinned host copies for the end-to-end leg
+        self.pin = {k: v.pin_memory() for k, v in
+                    (("pq", xp["q"]), ("pk", xp["k"]), ("pv", xp["v"]), ("dq", q1), ("dk", k1),
+                     ("dv", v1), ("pos", xd["lens"]))}
+        self.pin_out_p = torch.empty(self.pout.shape, dtype=torch.bfloat16).pin_memory()
+        self.pin_out_d = torch.empty(self.dout.shape, dtype=torch.bfloat16).pin_memory()
+
+    def step(self, ev=None):
+        """The device-resident step.  ev: optional list of 4 event pairs to record."""
+        g = self.gqa
+        g.gqa_rope_append(self.pq, self.pk, self.pv, self.pkc, self.pvc, qk_norm=True,
+                          max_pos0=0, status=self.status)
+        if ev is not None:
+            ev[0].record()
+        g.gqa_prefill(self.pq, self.pkc, self.pvc, out=self.pout, status=self.status)
+        if ev is not None:
+            ev[1].record()
+        g.gqa_rope_append(self.dq, self.dk, self.dv, self.dkc, self.dvc, pos0=self.pos,
+                          max_pos0=self.max_len - 1, new_len=self.lens_new, qk_norm=True,
+                          status=self.status)
+        if ev is not None:
+            ev[2].record()
+        g.gqa_decode(self.dq, self.dkc, self.dvc, self.lens_new, self.max_len, out=self.dout,
+                     workspace=self.ws, status=self.status)
+        if ev is not None:
+            ev[3].record()
+
+    def step_e2e(self):
+        """Same step from pinned host buffers: H2D inputs, compute, D2H outputs."""
+        self.pq.copy_(self.pin["pq"], non_blocking=True)
+        self.pk.copy_(self.pin["pk"], non_blocking=True)
+        self.pv.copy_(self.pin["pv"], non_blocking=True)
+        self.dq.copy_(self.pin["dq"], non_blocking=True)
+        self.dk.copy_(self.pin["dk"], non_blocking=True)
+        self.dv.copy_(self.pin["dv"], non_blocking=True)
+        self.pos.copy_(self.pin["pos"], non_blocking=True)
+        self.step()
+        self.pin_out_p.copy_(self.pout, non_blocking=True)
+        self.pin_out_d.copy_(self.dout, non_blocking=True)
+
+    def e2e_bytes(self):
+        h2d = sum(t.numel() * t.element_size() for t in self.pin.values())
+        d2h = self.pin_out_p.numel() * 2 + self.pin_out_d.numel() * 2
+        return h2d, d2h
+
+
+def _barrier_sync(dist_on):
+    if dist_on:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+
+
+def _max_over_ranks(x: float, dist_on: bool, dev) -> float:
+    if not dist_on:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def run_ours(args, rank, world, dev, dist_on):
+    layer = Layer(dev)
+    peaks, peak_src = load_peaks()
+    for _ in range(args.warmup):
+        layer.step()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+
+    # -- device-resident timed region (per-kernel events on the launching stream) --
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    start = torch.cuda.Event(enable_timing=True)
+    stop = torch.cuda.Event(enable_timing=True)
+    _barrier_sync(dist_on)
+    start.record()
+    for i in range(args.steps):
+        layer.step(evs[i])
+    stop.record()
+    _barrier_sync(dist_on)
+    ms_total = start.elapsed_time(stop)
+    t_prefill = t_append_d = t_decode = 0.0
+    for i in range(args.steps):
+        e = evs[i]
+        t_prefill += e[0].elapsed_time(e[1])
+        t_append_d += e[1].elapsed_time(e[2])
+        t_decode += e[2].elapsed_time(e[3])
+    ms_total = _max_over_ranks(ms_total, dist_on, dev)
+
+    # -- end-to-end region: host buffers in, results out, every step --
+    for _ in range(min(args.warmup, 3)):
+        layer.step_e2e()
+    _barrier_sync(dist_on)
+    s2 = torch.cuda.Event(enable_timing=True)
+    e2 = torch.cuda.Event(enable_timing=True)
+    s2.record()
+    for _ in range(args.steps):
+        layer.step_e2e()
+    e2.record()
+    _barrier_sync(dist_on)
+    ms_e2e = _max_over_ranks(s2.elapsed_time(e2), dist_on, dev)
+    clocks = sampler.stop() if sampler else None
+    status = int(layer.status.item())
+    if rank != 0:
+        return None
+
+    K = args.steps
+    ms_step = ms_total / K
+    tok = tokens_per_step() * world
+    pf_ms = t_prefill / K
+    dec_ms = t_decode / K
+    pf_tflops = prefill_flops() / (pf_ms * 1e-3) / 1e12
+    dec_gbs = decode_bytes(layer.lens_new_host) / (dec_ms * 1e-3) / 1e9
+    long_run = ms_total > 1000.0
+    tpeak = peaks["bf16_tflops_sustained"] if long_run else peaks["bf16_tflops"]
+    hpeak = peaks["hbm_gbs"]
+    tag = "of " + peak_src
+    traffic = profiled_traffic()
+    h2d, d2h = layer.e2e_bytes()
+    line = {
+        "metric": METRIC,
+        "value": round(tok / (ms_step * 1e-3), 1),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) bf16 tensors shaped like the pages' 3.8B model)",
+        "config": {"workload": WORKLOAD, "prefill_batch": PREFILL.B, "seq_len": PREFILL.T,
+                   "decode_batch": DECODE.B, "heads": "24q/8kv", "head_dim": 128,
+                   "l2": "inputs exceed L2 (~0.9 GB touched per step); no flush",
+                   "parallelism": "replicas" if world > 1 else "single"},
+        "roofline": {"bound": "tensor", "kernel": "gqa_prefill",
+                     "achieved": round(pf_tflops, 1), "peak": tpeak, "unit": "TFLOP/s",
+                     "frac": round(pf_tflops / tpeak, 4),
+                     "peak_kind": ("bf16 sustained " if long_run else "bf16 burst ") + tag,
+                     "traffic": traffic,
+                     "algorithmic_per_launch": prefill_flops()},
+        "decode_roofline": {"bound": "hbm", "kernel": "gqa_decode",
+                            "achieved": round(dec_gbs, 1), "peak": hpeak, "unit": "GB/s",
+                            "frac": round(dec_gbs / hpeak, 4), "peak_kind": "hbm copy " + tag,
+                            "algorithmic_per_launch": decode_bytes(layer.lens_new_host),
+                            "us_per_launch": round(dec_ms * 1e3, 2)},
+        "phases_ms": {"prefill_kernel": round(pf_ms, 4), "decode_kernels": round(dec_ms, 4),
+                      "decode_append": round(t_append_d / K, 4),
+                      "prefill_append": round(ms_step - pf_ms - dec_ms - t_append_d / K, 4)},
+        "e2e": {"value": round(tok / (ms_e2e / K * 1e-3), 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": round(ms_e2e / K, 4)},
+        "gpu_launches": 5 * K,
+        "clocks": clocks,
+        "device_status": status,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
+    return line
+
+
+# ---------------------------------------------------------------------------
+# the oracle on the host cores (reported baseline / reference arm)
+# ---------------------------------------------------------------------------
+def cpu_baseline(budget_s: float = 15.0):
+    """Time the float64 oracle, as it stands, on a bounded sample of one step.
+
+    Sample: RoPE/QK-norm of all prompt tokens of one sequence, the attention rows
+    of a random subset of (b, t, h) prompt rows, and the decode rows of a subset
+    of sequences; the full-step time is extrapolated by the key visits (the
+    oracle's cost is proportional to query rows x visible keys)."""
+    import oracle
+    oracle.build()
+    cores = os.cpu_count() or 1
+    xp = inputs.make_inputs(PREFILL)
+    xd = inputs.make_inputs(DECODE)
+    rng = np.random.default_rng(0)
+    B, T, Hq = PREFILL.B, PREFILL.T, PREFILL.Hq
+    # 1. prep (norm + rope) of sequence 0's prompt, scaled by B
+    t0 = time.perf_counter()
+    qb = inputs.bits(xp["q"][:1])
+    kb = inputs.bits(xp["k"][:1])
+    pos = oracle.positions(0, 1, T)
+    q1 = oracle.prep(qb, pos, True)
+    k1 = oracle.prep(kb, pos, True)
+    v1 = oracle.bf16_to_f64(inputs.bits(xp["v"][:1]))
+    t_prep = (time.perf_counter() - t0) * B
+    # 2. prefill attention rows (sequence 0), sized to about budget/2
+    per_row_keys = T / 2.0
+    n_rows = 256
+    t_rows = 0.0
+    visits_done = 0.0
+    rows_done = 0
+    while True:
+        rows = rng.integers(0, T * Hq, size=n_rows)
+        t0 = time.perf_counter()
+        oracle.attention(q1, k1, v1, pos, rows=rows, nthreads=cores)
+        t_rows += time.perf_counter() - t0
+        visits_done += float(np.sum(rows // Hq + 1))
+        rows_done += n_rows
+        if t_rows > budget_s / 2 or n_rows > 1 << 20:
+            break
+        n_rows *= 2
+    visits_total = B * Hq * T * (T + 1) / 2.0
+    t_prefill = t_rows * visits_total / visits_done
+    # 3. decode: a subset of sequences, scaled by visible keys
+    lens = xd["lens"].numpy()
+    q, k, v = xd["steps"][0]
+    sel = np.arange(0, DECODE.B, 8)
+    t0 = time.perf_counter()
+    oracle.decode_step(inputs.bits(q[sel]), inputs.bits(k[sel]), inputs.bits(v[sel]),
+                       inputs.bits(xd["k_cache"][sel]), inputs.bits(xd["v_cache"][sel]),
+                       lens[sel], True, nthreads=cores)
+    t_dec = (time.perf_counter() - t0) * float(np.sum(lens + 1)) / float(np.sum(lens[sel] + 1))
+    step_s = t_prep + t_prefill + t_dec
+    return {"value": round(tokens_per_step() / step_s, 2), "unit": "tokens/s", "cores": cores,
+            "kind": "oracle",
+            "sample": ("float64 oracle on one step's sample: QK-norm+RoPE of 1 of 8 prompt "
+                       "sequences, %d random prefill attention rows of sequence 0, decode of "
+                       "8 of 64 sequences; full-step time extrapolated by key visits "
+                       "(%.1f s measured, %.1f s estimated per step)")
+            % (rows_done, t_prep / B + t_rows + t_dec * len(sel) / DECODE.B,
+               step_s),
+            "seconds_per_step_estimated": round(step_s, 2)}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    budget = max(2.0, min(20.0, 120.0 / max(1, args.steps + args.warmup)))
+    vals = []
+    for i in range(args.warmup + args.steps):
+        cb = cpu_baseline(budget)
+        if i >= args.warmup:
+            vals.append(cb)
+    value = statistics.median(v["value"] for v in vals)
+    cb = dict(vals[-1])
+    cb["value"] = value
+    step_s = tokens_per_step() / value
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(step_s * 1e3, 1), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "prefill_batch": PREFILL.B, "seq_len": PREFILL.T,
+                       "decode_batch": DECODE.B, "parallelism": "single"},
+            "cpu_baseline": cb,
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="budget of the CPU-baseline sample (oracle)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        sys.stderr.write("note: --gpus %d but WORLD_SIZE=%d; using WORLD_SIZE\n"
+                         % (args.gpus, world))
+
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py: no CUDA device (the library has no CPU path)")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist_on = world > 1
+    if dist_on:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=dev)
+    try:
+        line = run_ours(args, rank, world, dev, dist_on)
+    finally:
+        if dist_on:
+            torch.distributed.destroy_process_group()
+    if line is not None:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

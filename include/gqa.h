@@ -1,0 +1,160 @@
+/*
+ * gqa.h -- C ABI of the B200 (sm_100a) library for causal grouped-query attention
+ * with rotary position embedding, optional QK-RMSNorm, prompt prefill and
+ * single-token decode against a contiguous per-sequence KV cache.
+ *
+ * The operations follow these passages:
+ *   RoPE: page "750美元从零训练3个LLM：一位开发者的实战复盘", section "V1：现代架构基线"
+ *     (q and k turn by a position-dependent angle so that q_m . k_n depends on
+ *     m - n only); page "从零手训LLaMa：125M模型11小时训练全记录", section
+ *     "核心架构：手动实现LLaMa的四个关键组件".
+ *   GQA: same first page, section "V2：引入前沿技术" (query heads form groups that
+ *     share one K/V head; query head h reads K/V head h / (Hq / Hkv)).
+ *   QK-RMSNorm: page "训练3.8B LLM至0.384 CORE，成本998美元 – Hugo Vergnes",
+ *     sections "设置" (QK-norm) and "无效的方法" (F.rms_norm: eps inside the root).
+ *   Causal attention: same page, section "无效的方法" (causal
+ *     scaled_dot_product_attention, default scale 1/sqrt(D)); page "Build a Large
+ *     Language Model from Scratch" (nxbn.cn), section 3.1.
+ *   KV cache: page "750美元从零训练3个LLM", section "V3：扩容与推理优化" (the new
+ *     token computes its own q, k, v, appends k and v to the cache and attends
+ *     over the whole cache); page "从零手训LLaMa", section on batched KV-cache
+ *     inference.
+ *
+ * Conventions shared by every entry point
+ *   - bf16 tensors are passed as void* and are row-major and contiguous:
+ *       q              [B, T, Hq, D]      (prefill / rope)   [B, Hq, D] (decode)
+ *       k, v (new)     [B, T, Hkv, D]                        [B, Hkv, D] (decode)
+ *       k_cache/v_cache[B, Hkv, Lmax, D]  (one contiguous [Lmax, D] slab per head)
+ *       out            [B, T, Hq, D]      (prefill)          [B, Hq, D] (decode)
+ *   - D is 64, 96 or 128; Hq % Hkv == 0 (a GQA group is g = Hq / Hkv heads);
+ *     Lmax is a multiple of 128.  Every data pointer is 16-byte aligned.
+ *   - All pointers except the stream are DEVICE pointers to caller-owned memory.
+ *     The library allocates no memory and keeps no per-call state; it caches
+ *     one function pointer (the driver's tensor-map encoder) per process.
+ *   - stream is a cudaStream_t (NULL = legacy default stream).  All work is
+ *     queued asynchronously on it; the host return code covers argument
+ *     validation and launch errors only.
+ *   - status_dev, where taken, is an optional device int32 that kernels OR
+ *     GQA_DEV_* bits into (NULL: device-side errors are not reported).  The
+ *     caller zeroes it and reads it after synchronising.
+ *   - RoPE pairs coordinate i with i + D/2 and turns pair i at position p by
+ *     p * base^(-2i/D) radians; QK-RMSNorm (unit gain) runs before RoPE.
+ *   - scale <= 0 selects 1/sqrt(D).
+ *   - Every element written is a bf16 rounded to nearest even from fp32 math.
+ */
+#ifndef GQA_H_
+#define GQA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GQA_OK = 0,
+    GQA_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misalignment, Hq % Hkv != 0 */
+    GQA_ERR_UNSUPPORTED = 2,   /* D not in {64, 96, 128}, or a device below sm_100 */
+    GQA_ERR_CAPACITY = 3,      /* host-known positions or lengths exceed Lmax */
+    GQA_ERR_TIMEOUT = 4,       /* reserved for host-side waits */
+    GQA_ERR_CUDA = 5,          /* a CUDA runtime / driver call failed */
+    GQA_ERR_WORKSPACE = 6      /* workspace missing or smaller than required */
+} gqa_status;
+
+/* Bits OR-ed into *status_dev by kernels. */
+#define GQA_DEV_CAPACITY 0x1   /* a sequence's writes or reads would pass Lmax: skipped */
+#define GQA_DEV_TIMEOUT 0x2    /* a bounded wait inside a kernel gave up: output invalid */
+#define GQA_DEV_BAD_LEN 0x4    /* a length or position < 0 (or 0 where >= 1 is needed) */
+
+typedef struct {
+    int qk_norm;       /* nonzero: unit-gain RMSNorm over D before RoPE */
+    float eps;         /* RMSNorm epsilon inside the root (1e-6 in the pages' model) */
+    float rope_base;   /* RoPE base (10000) */
+} gqa_rope_params;
+
+/*
+ * gqa_rope_apply -- in place on q [B, T, H, D]: q <- RoPE(RMSNorm?(q)) with token
+ * t of sequence b at position pos0[b] + t.
+ *   pos0: device int32 [B], or NULL for position 0.
+ * Errors: GQA_ERR_INVALID_ARG (q null, B/T/H < 1, misaligned), GQA_ERR_UNSUPPORTED.
+ */
+gqa_status gqa_rope_apply(void *q, const int32_t *pos0, int B, int T, int H, int D,
+                          gqa_rope_params p, void *stream);
+
+/*
+ * kv_cache_append -- for every new token t of sequence b and KV head h:
+ *     k_cache[b, h, pos0[b] + t, :] = RoPE(RMSNorm?(k[b, t, h, :]))   (bf16)
+ *     v_cache[b, h, pos0[b] + t, :] = v[b, t, h, :]                  (bit copy)
+ * No other cache slot is touched.
+ *   pos0: device int32 [B] (current cache lengths), or NULL for 0.
+ *   max_pos0_host: a host-known upper bound of pos0, checked against
+ *     max_pos0_host + T <= Lmax (pass -1 to skip the host check).  A sequence
+ *     whose pos0[b] + T exceeds Lmax on the device is skipped and
+ *     GQA_DEV_CAPACITY is raised.
+ *   new_len: optional device int32 [B] output, new_len[b] = pos0[b] + T (the
+ *     lengths a following gqa_decode reads).  NULL to skip.
+ */
+gqa_status kv_cache_append(const void *k, const void *v, void *k_cache, void *v_cache,
+                           const int32_t *pos0, int max_pos0_host, int32_t *new_len,
+                           int B, int T, int Hkv, int D, int Lmax, gqa_rope_params p,
+                           int32_t *status_dev, void *stream);
+
+/*
+ * gqa_rope_append -- gqa_rope_apply on q [B, T, Hq, D] and kv_cache_append of
+ * k, v in ONE launch (the same positions pos0[b] + t for q and k).  Arguments
+ * as in the two calls above.
+ */
+gqa_status gqa_rope_append(void *q, const void *k, const void *v, void *k_cache,
+                           void *v_cache, const int32_t *pos0, int max_pos0_host,
+                           int32_t *new_len, int B, int T, int Hq, int Hkv, int D,
+                           int Lmax, gqa_rope_params p, int32_t *status_dev, void *stream);
+
+/*
+ * gqa_prefill -- causal attention of a prompt that starts at position 0:
+ *     out[b, t, h, :] = sum_{s <= t} softmax_s(q[b,t,h,:] . K[b, h/g, s, :] * scale)
+ *                                   * V[b, h/g, s, :]
+ * q must already be rotated (gqa_rope_apply / gqa_rope_append) and the caches
+ * must hold the prompt's rotated K and raw V in slots 0 .. T-1 (slots >= T are
+ * never read).  Tensor-core kernel (tcgen05 / TMEM, TMA-fed), fp32 softmax.
+ *   T <= Lmax.  Alignment: 16 bytes for every pointer.
+ * Device errors: GQA_DEV_TIMEOUT (a bounded pipeline wait expired).
+ */
+gqa_status gqa_prefill(const void *q, const void *k_cache, const void *v_cache, void *out,
+                       int B, int T, int Hq, int Hkv, int D, int Lmax, float scale,
+                       int32_t *status_dev, void *stream);
+
+/*
+ * gqa_decode -- one query token per sequence against the cache:
+ *     out[b, h, :] = sum_{s < lens[b]} softmax_s(q[b,h,:] . K[b, h/g, s, :] * scale)
+ *                                      * V[b, h/g, s, :]
+ * lens[b] counts the cached tokens INCLUDING the token just appended (the query
+ * sits at position lens[b] - 1 and attends to itself).  Split-K over the cache
+ * length; each KV head's bytes are read once per group of g query heads.
+ *   lens: device int32 [B], 1 <= lens[b] <= Lmax (others: GQA_DEV_BAD_LEN /
+ *     GQA_DEV_CAPACITY and that sequence's output is zero).
+ *   max_len_host: host-known upper bound of lens (<= Lmax); it sizes the grid
+ *     and the workspace.  Lengths above it raise GQA_DEV_CAPACITY.
+ *   ws, ws_bytes: device scratch of at least
+ *     gqa_decode_workspace_bytes(B, Hq, D, max_len_host) bytes; contents on
+ *     entry do not matter.  Two calls in flight must not share one workspace.
+ */
+gqa_status gqa_decode(const void *q, const void *k_cache, const void *v_cache,
+                      const int32_t *lens, int max_len_host, void *out, int B, int Hq,
+                      int Hkv, int D, int Lmax, float scale, void *ws, size_t ws_bytes,
+                      int32_t *status_dev, void *stream);
+
+/* Bytes of workspace gqa_decode needs for these sizes (0 on invalid sizes). */
+size_t gqa_decode_workspace_bytes(int B, int Hq, int D, int max_len);
+
+/* Static, human-readable text for a status code. */
+const char *gqa_status_string(gqa_status s);
+
+/* Library version as MAJOR * 10000 + MINOR * 100 + PATCH. */
+int gqa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GQA_H_ */

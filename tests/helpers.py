@@ -1,0 +1,69 @@
+"""Shared helpers for the GPU parity tests (no attention arithmetic here)."""
+import numpy as np
+import torch
+
+import oracle
+from rope_gqa_kv_b200 import inputs
+
+# Tolerance for floating-point outputs against the float64 oracle, on O(1)
+# outputs (bf16 inputs, fp32 accumulation, bf16 outputs): max |d| <= 1e-2 for the
+# kernel's arithmetic, plus half an ulp of the exact value in bf16 for the
+# rounding of the answer to the output format (up to 0.0078 for |o| in [2, 4),
+# which no bf16 output can avoid), and mean |d| <= 1e-3.
+MAX_ABS = 1e-2
+MEAN_ABS = 1e-3
+# Absolute floor of the one-ulp check: fp32 rotation of O(1) inputs can lose a
+# few fp32 ulps (~1e-6) when the result cancels to nearly zero.
+ULP_ABS_FLOOR = 2.0 ** -18
+
+
+def bf16_ulp(x):
+    mag = np.maximum(np.abs(np.asarray(x, dtype=np.float64)), 2.0 ** -126)
+    return 2.0 ** (np.floor(np.log2(mag)) - 7)
+
+
+def bits(t: torch.Tensor) -> np.ndarray:
+    return inputs.bits(t.detach().cpu())
+
+
+def f64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().cpu().to(torch.float64).numpy()
+
+
+def assert_close(got: torch.Tensor, want: np.ndarray, what: str, max_abs=MAX_ABS,
+                 mean_abs=MEAN_ABS):
+    g = f64(got)
+    assert g.shape == want.shape, (what, g.shape, want.shape)
+    assert np.isfinite(g).all(), "%s: non-finite output" % what
+    d = np.abs(g - want)
+    allow = max_abs + 0.5 * bf16_ulp(want)
+    if not ((d <= allow).all() and d.mean() <= mean_abs):
+        i = np.unravel_index(np.argmax(d), d.shape)
+        w = want[i]
+        rne = float(torch.tensor(w, dtype=torch.float64).to(torch.bfloat16).double())
+        raise AssertionError(
+            "%s: max|d| %.4g (<= %.3g + half ulp) mean|d| %.3g (<= %.3g); worst at %s: got %.6g "
+            "want %.6g (bf16 rounding of want alone: %.3g); elements over: %d of %d"
+            % (what, d.max(), max_abs, d.mean(), mean_abs, i, g[i], w, abs(rne - w),
+               int((d > allow).sum()), d.size))
+    return d.max(), d.mean()
+
+
+def assert_within_one_ulp(got: torch.Tensor, want: np.ndarray, what: str):
+    """Every bf16 element within one bf16 ulp (plus ULP_ABS_FLOOR) of the exact value."""
+    g = f64(got)
+    w = np.asarray(want, dtype=np.float64)
+    ulp = bf16_ulp(w)
+    bad = np.abs(g - w) > ulp + ULP_ABS_FLOOR
+    assert not bad.any(), "%s: %d elements off by more than one bf16 ulp (worst %.3g ulp)" % (
+        what, bad.sum(), (np.abs(g - w) / ulp).max())
+
+
+def oracle_cache_after(k_rot_f64, v_f64, B, Hkv, Lmax, D):
+    """Float64 caches [B, Hkv, Lmax, D] holding prompt slots 0..T-1 (rest zero)."""
+    T = k_rot_f64.shape[1]
+    kc = np.zeros((B, Hkv, Lmax, D))
+    vc = np.zeros((B, Hkv, Lmax, D))
+    kc[:, :, :T] = k_rot_f64.transpose(0, 2, 1, 3)
+    vc[:, :, :T] = v_f64.transpose(0, 2, 1, 3)
+    return kc, vc

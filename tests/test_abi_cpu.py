@@ -1,0 +1,114 @@
+"""C-ABI checks that need no GPU: exported symbols and host-side validation.
+
+The argument checks below all fail before the library touches the CUDA
+runtime, so they run on a machine without a GPU.
+"""
+import ctypes
+import re
+import os
+
+import pytest
+
+import rope_gqa_kv_b200 as gqa
+from rope_gqa_kv_b200 import _lib
+from rope_gqa_kv_b200 import build as gqa_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gqa.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    gqa_build.build()
+    return gqa.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:gqa_status|size_t|const char \*|int)\s*\**\s*(\w+)\s*\(",
+                                 text, flags=re.M)))
+
+
+def test_header_declares_the_four_entry_points():
+    names = declared_functions()
+    for n in ("gqa_rope_apply", "kv_cache_append", "gqa_prefill", "gqa_decode"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert names, "no declarations parsed from gqa.h"
+    raw = ctypes.CDLL(_lib.LIB_PATH)
+    for n in names:
+        assert hasattr(raw, n), "libgqa.so does not export %s" % n
+    # the binding covers exactly the declared surface
+    assert sorted(_lib.SIGNATURES) == names
+
+
+def test_status_strings_and_version(lib):
+    for s in range(7):
+        assert lib.gqa_status_string(s)
+    assert lib.gqa_status_string(99) == b"unknown status"
+    assert lib.gqa_version() >= 100
+
+
+def test_workspace_size(lib):
+    # B * Hq * ceil(max_len / 64) rows of (D + 2) floats, plus slack
+    assert lib.gqa_decode_workspace_bytes(64, 24, 128, 2049) == 64 * 24 * 33 * (128 + 2) * 4 + 256
+    assert lib.gqa_decode_workspace_bytes(0, 24, 128, 100) == 0
+    assert lib.gqa_decode_workspace_bytes(1, 24, 80, 100) == 0
+
+
+P = _lib.RopeParams(0, 1e-6, 10000.0)
+FAKE = ctypes.c_void_p(0x10000)          # 16-byte aligned, never dereferenced
+ODD = ctypes.c_void_p(0x10008)           # misaligned
+
+
+def test_rope_apply_validation(lib):
+    assert lib.gqa_rope_apply(None, None, 1, 1, 1, 64, P, None) == 1
+    assert lib.gqa_rope_apply(FAKE, None, 1, 1, 1, 80, P, None) == 2
+    assert lib.gqa_rope_apply(ODD, None, 1, 1, 1, 64, P, None) == 1
+    assert lib.gqa_rope_apply(FAKE, None, 0, 1, 1, 64, P, None) == 1
+    bad = _lib.RopeParams(0, 1e-6, 0.5)
+    assert lib.gqa_rope_apply(FAKE, None, 1, 1, 1, 64, bad, None) == 1
+
+
+def test_append_validation(lib):
+    f = FAKE
+    # capacity known on the host: max_pos0 + T > Lmax
+    assert lib.kv_cache_append(f, f, f, f, None, 120, None, 1, 16, 2, 64, 128, P, None, None) == 3
+    # Lmax not a multiple of 128
+    assert lib.kv_cache_append(f, f, f, f, None, 0, None, 1, 16, 2, 64, 100, P, None, None) == 1
+    assert lib.kv_cache_append(f, f, f, f, None, 0, None, 1, 16, 2, 72, 128, P, None, None) == 2
+    # fused call: Hq not a multiple of Hkv
+    assert lib.gqa_rope_append(f, f, f, f, f, None, 0, None, 1, 1, 6, 4, 64, 128, P, None,
+                               None) == 1
+
+
+def test_prefill_validation(lib):
+    f = FAKE
+    assert lib.gqa_prefill(f, f, f, f, 1, 10, 6, 4, 64, 128, 0.0, None, None) == 1
+    assert lib.gqa_prefill(f, f, f, f, 1, 10, 4, 2, 48, 128, 0.0, None, None) == 2
+    assert lib.gqa_prefill(f, f, f, f, 1, 300, 4, 2, 64, 256, 0.0, None, None) == 3
+    assert lib.gqa_prefill(f, f, f, ODD, 1, 10, 4, 2, 64, 128, 0.0, None, None) == 1
+    assert lib.gqa_prefill(f, f, f, f, 1, 0, 4, 2, 64, 128, 0.0, None, None) == 1
+
+
+def test_decode_validation(lib):
+    f = FAKE
+    ws = ctypes.c_size_t(1 << 20)
+    assert lib.gqa_decode(f, f, f, f, 100, f, 1, 4, 2, 64, 128, 0.0, None, 0, None, None) == 6
+    assert lib.gqa_decode(f, f, f, f, 100, f, 1, 4, 2, 64, 128, 0.0, f, 16, None, None) == 6
+    assert lib.gqa_decode(f, f, f, f, 200, f, 1, 4, 2, 64, 128, 0.0, f, ws, None, None) == 3
+    assert lib.gqa_decode(f, f, f, f, 0, f, 1, 4, 2, 64, 128, 0.0, f, ws, None, None) == 1
+    assert lib.gqa_decode(f, f, f, f, 100, f, 1, 5, 2, 64, 128, 0.0, f, ws, None, None) == 1
+    assert lib.gqa_decode(f, f, f, f, 100, f, 1, 4, 2, 32, 128, 0.0, f, ws, None, None) == 2
+    assert lib.gqa_decode(None, f, f, f, 100, f, 1, 4, 2, 64, 128, 0.0, f, ws, None, None) == 1
+
+
+def test_binding_refuses_cpu_tensors(lib):
+    import torch
+    q = torch.zeros(1, 4, 2, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        gqa.gqa_rope_apply(q)

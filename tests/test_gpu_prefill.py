@@ -1,0 +1,102 @@
+"""GPU parity: the prefill phase (QK-norm + RoPE + append, then the tcgen05 kernel).
+
+Each case runs the whole phase on the GPU through the C ABI -- gqa_rope_append
+on the prompt's q, k, v, then gqa_prefill -- and compares the output with the
+float64 oracle's prefill on the same bf16 inputs, element by element: fully at
+the sizes the oracle finishes in seconds (which still span several tiles and a
+ragged tail), and on sampled rows at the 3.8B-style full size.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import rope_gqa_kv_b200 as gqa
+from rope_gqa_kv_b200 import inputs
+
+from helpers import assert_close, bits
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _run_phase(x, w, out=None):
+    dq, dk, dv = x["q"].to(DEV), x["k"].to(DEV), x["v"].to(DEV)
+    dkc, dvc = x["k_cache"].to(DEV), x["v_cache"].to(DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    gqa.gqa_rope_append(dq, dk, dv, dkc, dvc, qk_norm=w.qk_norm, max_pos0=0, status=status)
+    o = gqa.gqa_prefill(dq, dkc, dvc, out=out, status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0, "device status %#x" % status.item()
+    return o
+
+
+@pytest.mark.parametrize("name", ["tiny_gqa", "mha_prefill", "generation"])
+def test_named_workload_full_output(cuda_lib, name):
+    w = inputs.BY_NAME[name]
+    x = inputs.make_inputs(w, decode_steps=0)
+    o = _run_phase(x, w)
+    want, _, _ = oracle.prefill(bits(x["q"]), bits(x["k"]), bits(x["v"]), w.qk_norm)
+    assert_close(o, want, name)
+
+
+@pytest.mark.parametrize("B,T,Hq,Hkv,D,qk", [
+    (2, 1, 4, 2, 64, False),          # a single token
+    (1, 200, 6, 2, 128, True),        # ragged second tile
+    (2, 300, 3, 3, 96, False),        # MHA, ragged pair
+    (1, 385, 8, 1, 64, True),         # MQA, three pairs, ragged
+    (1, 256, 4, 2, 128, False),       # T == Lmax exactly
+    (3, 129, 6, 3, 96, True),         # one row into the second tile
+])
+def test_shapes_and_tails(cuda_lib, B, T, Hq, Hkv, D, qk):
+    w = inputs.custom("pf", B=B, Hq=Hq, Hkv=Hkv, D=D, T=T, qk_norm=qk, seed_index=T + D)
+    x = inputs.make_inputs(w)
+    o = _run_phase(x, w)
+    want, _, _ = oracle.prefill(bits(x["q"]), bits(x["k"]), bits(x["v"]), qk)
+    assert_close(o, want, "B%d T%d Hq%d Hkv%d D%d" % (B, T, Hq, Hkv, D))
+
+
+def test_output_rows_beyond_t_untouched(cuda_lib):
+    w = inputs.custom("pf", B=1, Hq=2, Hkv=1, D=64, T=70)
+    x = inputs.make_inputs(w)
+    big = torch.full((1, 128, 2, 64), 3.0, dtype=torch.bfloat16, device=DEV)
+    out = big[:, :70]     # a view: rows 70.. of `big` must keep their value
+    o = _run_phase(x, w, out=out.contiguous())
+    assert o.shape == (1, 70, 2, 64)
+    assert (big[:, 70:] == 3.0).all()
+
+
+def _sample_rows(B, T, Hq, rng, n_random=400):
+    ts = [0, 1, 127, 128, 129, 255, 256, 511, 1000, 1023, 1024, T - 129, T - 2, T - 1]
+    rows = set()
+    for b in {0, B - 1}:
+        for h in {0, Hq // 2, Hq - 1}:
+            for t in ts:
+                if 0 <= t < T:
+                    rows.add((b * T + t) * Hq + h)
+    rows.update(rng.integers(0, B * T * Hq, size=n_random).tolist())
+    return np.array(sorted(rows), dtype=np.int64)
+
+
+def test_prefill_3p8b_full_size_sampled(cuda_lib):
+    """B=8, T=2048, Hq=24, Hkv=8, D=128, QK-norm: the launch the benchmark times."""
+    w = inputs.BY_NAME["prefill_3p8b"]
+    x = inputs.make_inputs(w)
+    o = _run_phase(x, w)
+    rows = _sample_rows(w.B, w.T, w.Hq, np.random.default_rng(0))
+    want, _, _ = oracle.prefill(bits(x["q"]), bits(x["k"]), bits(x["v"]), True, rows=rows)
+    got = o.reshape(-1, w.D)[torch.as_tensor(rows, device=DEV)]
+    assert_close(got, want.reshape(-1, w.D)[rows], "3.8B prefill (%d sampled rows)" % len(rows))
+    # properties that hold for every row: finite and bounded by the values' range
+    of = o.float()
+    assert torch.isfinite(of).all()
+    vmax = x["v"].float().abs().max().item()
+    assert of.abs().max().item() <= vmax + 1e-2
+
+
+def test_prefill_deterministic(cuda_lib):
+    w = inputs.custom("pf", B=2, Hq=6, Hkv=2, D=128, T=700, qk_norm=True)
+    x = inputs.make_inputs(w)
+    a = _run_phase(x, w)
+    b = _run_phase(x, w)
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
