@@ -18,9 +18,9 @@
 //   2. chunk softmax in base 2: m = max, p = 2^(s - m), l = sum p.
 //   3. p.V: lane (key group, 16-byte column chunk) accumulates G x 8 outputs
 //      over its keys, then the key groups are summed through shared memory.
-// The partial (m, l, o) of each split goes to the workspace; a second kernel
-// merges the splits of each (b, query head): M = max m_i,
-// o = sum_i 2^(m_i - M) o_i / sum_i 2^(m_i - M) l_i.
+// The partial (m, l, o) of each split goes to the workspace; a second kernel,
+// launched as a programmatic dependent of the first, merges the splits of each
+// (b, query head): M = max m_i, o = sum_i 2^(m_i - M) o_i / sum_i 2^(m_i - M) l_i.
 #include "common.cuh"
 #include "ptx.cuh"
 
@@ -67,6 +67,9 @@ decode_split_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ __align__(8) uint64_t bars[2];
 
+    // The merge kernel may be scheduled now; it waits for this grid to finish
+    // before it reads anything.
+    asm volatile("griddepcontrol.launch_dependents;");
     const int split = blockIdx.x;
     const int kvh = blockIdx.y / n_sub;
     const int sub = blockIdx.y - kvh * n_sub;
@@ -254,33 +257,53 @@ decode_split_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__
     }
 }
 
-// Merge the splits of one (b, query head): one thread per output coordinate.
-template <int CH>
-__global__ void decode_combine_kernel(const float *__restrict__ ws_o,
-                                      const float *__restrict__ ws_ml,
-                                      const int32_t *__restrict__ lens, int max_len, int Hq,
-                                      int D, int Lmax, int n_splits, uint16_t *__restrict__ out) {
-    const int h = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
+// Merge the splits of one (b, query head): one warp per row.  Lanes read the
+// splits' (m, l) in parallel and reduce them with shuffles; each lane then owns
+// D/32 output coordinates and walks the splits with independent loads.
+constexpr int kCombWarps = 8;
+
+template <int D>
+__global__ void __launch_bounds__(kCombWarps * 32)
+decode_combine_kernel(const float *__restrict__ ws_o, const float *__restrict__ ws_ml,
+                      const int32_t *__restrict__ lens, int max_len, int B, int Hq, int Lmax,
+                      int n_splits, int CH, uint16_t *__restrict__ out) {
+    // Programmatic dependent launch: everything above this line may overlap the
+    // split kernel; the partials are read only after it has completed.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    const int lane = threadIdx.x & 31;
+    const int row = blockIdx.x * kCombWarps + (threadIdx.x >> 5);   // b * Hq + h
+    if (row >= B * Hq) return;
+    const int b = row / Hq;
     const int len = lens[b];
-    uint16_t *o = out + ((size_t)b * Hq + h) * D;
+    constexpr int kPer = D / 32;
+    uint16_t *o = out + (size_t)row * D;
     if (len < 1 || len > max_len || len > Lmax) {
-        if (d < D) o[d] = 0;
+#pragma unroll
+        for (int k = 0; k < kPer; ++k) o[lane + 32 * k] = 0;
         return;
     }
     const int ns = (len + CH - 1) / CH;
-    const size_t row0 = ((size_t)b * Hq + h) * n_splits;
+    const float *ml = ws_ml + (size_t)row * n_splits * 2;
+    const float *po = ws_o + (size_t)row * n_splits * D;
     float M = -INFINITY;
-    for (int i = 0; i < ns; ++i) M = fmaxf(M, ws_ml[(row0 + i) * 2]);
-    float L = 0.f, acc = 0.f;
+    for (int i = lane; i < ns; i += 32) M = fmaxf(M, ml[2 * i]);
+    M = warp_max(M);
+    float L = 0.f;
+    for (int i = lane; i < ns; i += 32) L = fmaf(ex2(ml[2 * i] - M), ml[2 * i + 1], L);
+    L = warp_sum(L);
+    float acc[kPer];
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) acc[k] = 0.f;
+#pragma unroll 4
     for (int i = 0; i < ns; ++i) {
-        const float w = ex2(ws_ml[(row0 + i) * 2] - M);
-        L = fmaf(w, ws_ml[(row0 + i) * 2 + 1], L);
-        if (d < D) acc = fmaf(w, ws_o[(row0 + i) * D + d], acc);
+        const float w = ex2(ml[2 * i] - M);
+#pragma unroll
+        for (int k = 0; k < kPer; ++k) acc[k] = fmaf(w, po[(size_t)i * D + lane + 32 * k], acc[k]);
     }
-    if (d < D) {
-        const float r = acc / L;
-        o[d] = (uint16_t)(pack_bf16x2(r, 0.f) & 0xffffu);
-    }
+    const float inv = 1.f / L;
+#pragma unroll
+    for (int k = 0; k < kPer; ++k)
+        o[lane + 32 * k] = (uint16_t)(pack_bf16x2(acc[k] * inv, 0.f) & 0xffffu);
 }
 
 template <int D, int G, int CH>
@@ -301,10 +324,21 @@ cudaError_t launch_decode(const void *q, const void *kc, const void *vc, const i
         n_sub, ws_o, ws_ml, status);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    decode_combine_kernel<CH><<<dim3(Hq, B), D, 0, s>>>(ws_o, ws_ml, lens, max_len, Hq, D, Lmax,
-                                                        n_splits,
-                                                        static_cast<uint16_t *>(out));
-    return cudaGetLastError();
+    // The merge is launched as a programmatic dependent of the split kernel, so
+    // its launch and scheduling overlap the split kernel's last wave.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((B * Hq + kCombWarps - 1) / kCombWarps));
+    cfg.blockDim = dim3(kCombWarps * 32);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, decode_combine_kernel<D>, (const float *)ws_o,
+                              (const float *)ws_ml, lens, max_len, B, Hq, Lmax, n_splits, CH,
+                              static_cast<uint16_t *>(out));
 }
 
 // Query heads per CTA: the largest of {3, 2, 1} (D = 128) or {4, 3, 2, 1}

@@ -9,11 +9,12 @@
 //
 // One CTA owns two 128-row query tiles of one (b, h) -- rows [256i, 256i+128)
 // and [256i+128, 256i+256) -- and streams the key/value tiles they need.
-// Warp roles (320 threads):
-//   warps 0-3  softmax of tile 0 (thread = query row = TMEM lane)
-//   warps 4-7  softmax of tile 1
-//   warp 8     TMA producer: Q tiles once, then a K ring and a V ring
-//   warp 9     MMA issuer (one thread): S_t = Q_t K^T and O_t += P_t V
+// Warp roles (384 threads, three warpgroups):
+//   warps 0-3  softmax of tile 0 (thread = query row = TMEM lane), 232 registers
+//   warps 4-7  softmax of tile 1, 232 registers
+//   warp 8     TMA producer: Q tiles once, then a K ring and a V ring  } 40
+//   warp 9     MMA issuer (one thread): S_t = Q_t K^T and O_t += P_t V } registers
+//   warps 10-11 idle (they complete the third warpgroup)              }
 // Tensor memory (512 columns): S0 [0,128) S1 [128,256) fp32 scores, with the
 // bf16 probabilities P_t written over the first 64 columns of S_t; O0 [256, 256+D)
 // O1 [384, 384+D) fp32 accumulators.
@@ -37,9 +38,16 @@
 namespace gqa {
 namespace {
 
-constexpr int kPfThreads = 320;
+constexpr int kPfThreads = 384;   // three warpgroups
 constexpr int kTmaWarp = 8;
 constexpr int kMmaWarp = 9;
+// Registers: launched at 168 per thread (65536 / 384, rounded down to 8); the two
+// softmax warpgroups take 224 each and the producer/MMA warpgroup keeps 56:
+// 2 * 224 + 56 = 3 * 168, so the increases are exactly covered by the decrease.
+constexpr int kLaunchRegs = 168;
+constexpr uint32_t kSoftmaxRegs = 224;
+constexpr uint32_t kControlRegs = 56;
+static_assert(2 * kSoftmaxRegs + kControlRegs == 3 * kLaunchRegs, "register split must balance");
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale O only past 2^8 growth
 
 template <int D>
@@ -214,6 +222,7 @@ __device__ void softmax_tile(PfSync &sy, uint32_t tmem, int t, int q_first, int 
 #pragma unroll
         for (int c = 0; c < 4; ++c) ptx::tmem_ld32(lane_addr + s_col + 32 * c, sv[c]);
         ptx::tmem_wait_ld();
+#define SV(c) __uint_as_float(sv[(c) >> 5][(c) & 31])
 
         const int key0 = j * 128;
         if (j == diag || key0 + 128 > T) {
@@ -223,9 +232,16 @@ __device__ void softmax_tile(PfSync &sy, uint32_t tmem, int t, int q_first, int 
                 if (key > qrow || key >= T) sv[c >> 5][c & 31] = __float_as_uint(-INFINITY);
             }
         }
-        float smax = -INFINITY;
+        // Row maximum: four independent chains of three-input max.
+        float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < 128; ++c) smax = fmaxf(smax, __uint_as_float(sv[c >> 5][c & 31]));
+        for (int c = 0; c < 128; c += 8) {
+            mx0 = ptx::fmax3(mx0, SV(c), SV(c + 1));
+            mx1 = ptx::fmax3(mx1, SV(c + 2), SV(c + 3));
+            mx2 = ptx::fmax3(mx2, SV(c + 4), SV(c + 5));
+            mx3 = ptx::fmax3(mx3, SV(c + 6), SV(c + 7));
+        }
+        const float smax = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
         const float m_new = fmaxf(m, smax * scale_log2);
         const bool resc = m_new > m + kRescaleThreshold;
         const float alpha = resc ? ex2(m - m_new) : 1.f;
@@ -244,23 +260,33 @@ __device__ void softmax_tile(PfSync &sy, uint32_t tmem, int t, int q_first, int 
                 ptx::tmem_st32(lane_addr + o_col + 32 * c, o);
             }
         }
+        // p = 2^(s * scale_log2 - m): packed FMA for the exponent argument, the
+        // special-function unit for 2^x, four independent partial row sums.
         const float neg_m = -m;
+        float la0 = 0.f, la1 = 0.f, lb0 = 0.f, lb1 = 0.f;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
             uint32_t p[16];
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
-                const float p0 = ex2(fmaf(__uint_as_float(sv[c][2 * e]), scale_log2, neg_m));
-                const float p1 = ex2(fmaf(__uint_as_float(sv[c][2 * e + 1]), scale_log2, neg_m));
+                float x0, x1;
+                ptx::ffma2(x0, x1, SV(32 * c + 2 * e), SV(32 * c + 2 * e + 1), scale_log2,
+                           scale_log2, neg_m, neg_m);
+                const float p0 = ex2(x0), p1 = ex2(x1);
                 p[e] = pack_bf16x2(p0, p1);
-                // normalise by the weights the MMA really uses (the rounded ones)
-                l += bf16lo(p[e]) + bf16hi(p[e]);
+                if (e & 1)
+                    ptx::fadd2(la0, la1, la0, la1, p0, p1);
+                else
+                    ptx::fadd2(lb0, lb1, lb0, lb1, p0, p1);
             }
             ptx::tmem_st16(lane_addr + s_col + 16 * c, p);
         }
+#undef SV
+        l += (la0 + la1) + (lb0 + lb1);
         ptx::tmem_wait_st();
         ptx::tc_fence_before();
-        ptx::mbar_arrive(A(sy.p_full[t]));
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(A(sy.p_full[t]));
     }
     if (ok) ok = __all_sync(0xffffffffu, ptx::mbar_wait(A(sy.o_final[t]), 0));
     if (!ok) {
@@ -322,7 +348,7 @@ prefill_kernel(const __grid_constant__ PfMaps maps, uint16_t *__restrict__ out, 
         }
         for (int t = 0; t < 2; ++t) {
             ptx::mbar_init(A(sy.s_full[t]), 1);
-            ptx::mbar_init(A(sy.p_full[t]), 128);
+            ptx::mbar_init(A(sy.p_full[t]), 4);   // one elected lane per softmax warp
             ptx::mbar_init(A(sy.o_final[t]), 1);
         }
         ptx::mbar_init(A(sy.mma_done), 1);
@@ -342,13 +368,17 @@ prefill_kernel(const __grid_constant__ PfMaps maps, uint16_t *__restrict__ out, 
     ptx::tc_fence_after();
     const uint32_t tmem = sy.tmem_base;
 
-    if (warp == kTmaWarp) {
-        if (lane == 0) producer<D>(maps, sy, smem, b, h, kvh, Hkv, q0, has1, n_kv, status);
-        __syncwarp();
-    } else if (warp == kMmaWarp) {
-        if (lane == 0) mma_issuer<D>(sy, smem, tmem, has1, n0, n1, n_kv, status);
-        __syncwarp();
+    if (warp >= 8) {
+        ptx::regs_dec<kControlRegs>();
+        if (warp == kTmaWarp) {
+            if (lane == 0) producer<D>(maps, sy, smem, b, h, kvh, Hkv, q0, has1, n_kv, status);
+            __syncwarp();
+        } else if (warp == kMmaWarp) {
+            if (lane == 0) mma_issuer<D>(sy, smem, tmem, has1, n0, n1, n_kv, status);
+            __syncwarp();
+        }
     } else {
+        ptx::regs_inc<kSoftmaxRegs>();
         const int t = warp >> 2;
         if (t == 0 || has1) {
             uint16_t *base = out + ((size_t)b * T * Hq + h) * D;
@@ -422,6 +452,11 @@ gqa_status launch_prefill(const void *q, const void *kc, const void *vc, void *o
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kSmem) !=
         cudaSuccess)
         return GQA_ERR_CUDA;
+    // The warpgroup register split assumes the launch allocation of kLaunchRegs per
+    // thread; with any other count the increases could not be satisfied, so refuse.
+    cudaFuncAttributes attr;
+    if (cudaFuncGetAttributes(&attr, kern) != cudaSuccess) return GQA_ERR_CUDA;
+    if (attr.numRegs != kLaunchRegs) return GQA_ERR_UNSUPPORTED;
     const int n_pairs = (T + 255) / 256;
     const long long grid = (long long)n_pairs * Hq * B;
     kern<<<(unsigned)grid, kPfThreads, S::kSmem, s>>>(maps, static_cast<uint16_t *>(out), B, T,

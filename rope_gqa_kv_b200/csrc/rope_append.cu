@@ -5,9 +5,10 @@
 // QK-norm: page "训练3.8B LLM至0.384 CORE，成本998美元 – Hugo Vergnes", section "设置";
 // KV-cache append: first page, section "V3：扩容与推理优化".
 //
-// One CTA per token (b, t).  The CTA first turns the token's position into the
-// D/2 rotation angles (float64 angle p * base^(-2i/D), then cos/sin rounded to
-// fp32) in shared memory, shared by all of the token's heads.  Each head vector
+// One CTA per token (b, t).  The CTA issues the loads of its first head vectors,
+// then turns the token's position into the D/2 rotation angles (float64 angle
+// p * base^(-2i/D) reduced to [-pi, pi] in float64, cos/sin in fp32) in shared
+// memory, shared by all of the token's heads.  Each head vector
 // is then owned by TPV threads: thread j holds the 16-byte chunk j of the first
 // half (coordinates 8j..8j+7) and the matching chunk of the second half
 // (coordinates D/2+8j..), i.e. exactly the 8 rotation pairs it needs, so every
@@ -118,15 +119,6 @@ rope_append_kernel(uint16_t *__restrict__ q, const uint16_t *__restrict__ k,
     if (p0 < 0) return;
     if (write_cache && p0 + T > Lmax) write_cache = false;
 
-    for (int i = threadIdx.x; i < S::kHalf; i += kThreads) {
-        const double theta = pow((double)base, -2.0 * (double)i / (double)D);
-        double sd, cd;
-        sincos((double)p * theta, &sd, &cd);
-        cs[i] = (float)cd;
-        sn[i] = (float)sd;
-    }
-    __syncthreads();
-
     const int nq = q ? Hq : 0;
     const int nk = write_cache ? Hkv : 0;
     const int nvec = nq + 2 * nk;
@@ -140,14 +132,8 @@ rope_append_kernel(uint16_t *__restrict__ q, const uint16_t *__restrict__ k,
     const size_t tok_q = (size_t)token * Hq * D;
     const size_t tok_kv = (size_t)token * Hkv * D;
 
-    // Every lane of a group runs the loop the same number of times (the shuffle
-    // in the norm needs the whole group), inactive lanes just skip memory.
-    for (int base_vec = 0; base_vec < nvec; base_vec += kSlots) {
-        const int vi = base_vec + warp * S::kVecPerWarp + slot;
-        const bool live = vi < nvec;
-        const uint16_t *src;
-        uint16_t *dst;
-        bool rotate;
+    // Where vector vi comes from and goes to; `rotate` is false for value heads.
+    auto locate = [&](int vi, const uint16_t *&src, uint16_t *&dst, bool &rotate) {
         if (vi < nq) {
             src = q + tok_q + (size_t)vi * D;
             dst = q + tok_q + (size_t)vi * D;
@@ -158,14 +144,65 @@ rope_append_kernel(uint16_t *__restrict__ q, const uint16_t *__restrict__ k,
             dst = kc + (((size_t)b * Hkv + h) * Lmax + p) * D;
             rotate = true;
         } else {
-            const int h = vi - nq - nk;
-            src = v + tok_kv + (size_t)(live ? h : 0) * D;
-            dst = vc + (((size_t)b * Hkv + (live ? h : 0)) * Lmax + p) * D;
+            const int h = min(vi - nq - nk, Hkv - 1);
+            src = v + tok_kv + (size_t)h * D;
+            dst = vc + (((size_t)b * Hkv + h) * Lmax + p) * D;
             rotate = false;
         }
+    };
+
+    // The first kPre passes of loads are issued before the angles are computed,
+    // so their memory latency overlaps the trigonometry and the barrier.
+    constexpr int kPre = 2;
+    uint4 ra[kPre], rb[kPre];
+#pragma unroll
+    for (int u = 0; u < kPre; ++u) {
+        const int vi = u * kSlots + warp * S::kVecPerWarp + slot;
+        ra[u] = make_uint4(0, 0, 0, 0);
+        rb[u] = make_uint4(0, 0, 0, 0);
+        if (vi < nvec && active) {
+            const uint16_t *src;
+            uint16_t *dst;
+            bool rot;
+            locate(vi, src, dst, rot);
+            ra[u] = *reinterpret_cast<const uint4 *>(src + 8 * j);
+            rb[u] = *reinterpret_cast<const uint4 *>(src + S::kHalf + 8 * j);
+        }
+    }
+
+    // Angle p * base^(-2i/D) in float64, reduced to [-pi, pi] in float64
+    // (subtracting the nearest multiple of 2*pi), then sin/cos in fp32.
+    for (int i = threadIdx.x; i < S::kHalf; i += kThreads) {
+        const double theta = pow((double)base, -2.0 * (double)i / (double)D);
+        const double a = (double)p * theta;
+        const double two_pi = 6.283185307179586476925286766559;
+        const double r = a - rint(a * (1.0 / two_pi)) * two_pi;
+        float sf, cf;
+        sincosf((float)r, &sf, &cf);
+        cs[i] = cf;
+        sn[i] = sf;
+    }
+    __syncthreads();
+
+    // Every lane of a group runs the loop the same number of times (the shuffle
+    // in the norm needs the whole warp); inactive lanes just skip memory.
+    for (int pass = 0; pass * kSlots < nvec; ++pass) {
+        const int vi = pass * kSlots + warp * S::kVecPerWarp + slot;
+        const bool live = vi < nvec;
+        const uint16_t *src;
+        uint16_t *dst;
+        bool rotate;
+        locate(live ? vi : 0, src, dst, rotate);
         const bool mem = live && active;
         uint4 a = make_uint4(0, 0, 0, 0), bb = make_uint4(0, 0, 0, 0);
-        if (mem) {
+        if (pass < kPre) {
+#pragma unroll
+            for (int u = 0; u < kPre; ++u)
+                if (u == pass) {
+                    a = ra[u];
+                    bb = rb[u];
+                }
+        } else if (mem) {
             a = *reinterpret_cast<const uint4 *>(src + 8 * j);
             bb = *reinterpret_cast<const uint4 *>(src + S::kHalf + 8 * j);
         }
