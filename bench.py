@@ -58,6 +58,12 @@ def decode_bytes(lens_new, w=DECODE) -> float:
     return kv + 2 * w.B * w.Hq * w.D * 2
 
 
+def append_bytes(w=PREFILL) -> float:
+    """Prefill-sized rope+append: q read and written in place, k and v read and
+    written into the cache, all bf16."""
+    return 2.0 * w.B * w.T * (w.Hq + 2 * w.Hkv) * w.D * 2
+
+
 def tokens_per_step() -> int:
     return PREFILL.B * PREFILL.T + DECODE.B
 
@@ -189,8 +195,7 @@ class Layer:
         self.lens_new = torch.empty_like(self.pos)
         self.max_len = int(xd["lens"].max()) + 1
         self.dout = torch.empty_like(self.dq)
-        nbytes = gqa.gqa_decode_workspace_bytes(DECODE.B, DECODE.Hq, DECODE.D, self.max_len)
-        self.ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+        self.ws = gqa.decode_workspace(DECODE.B, DECODE.Hq, DECODE.D, self.max_len, dev)
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
         self.lens_new_host = (xd["lens"] + 1).numpy()
         # pinned host copies for the end-to-end leg
@@ -201,24 +206,27 @@ class Layer:
         self.pin_out_d = torch.empty(self.dout.shape, dtype=torch.bfloat16).pin_memory()
 
     def step(self, ev=None):
-        """The device-resident step.  ev: optional list of 4 event pairs to record."""
+        """The device-resident step.  ev: optional list of 5 events recorded
+        around the four phases (prefill append, prefill, decode append, decode)."""
         g = self.gqa
+        if ev is not None:
+            ev[0].record()
         g.gqa_rope_append(self.pq, self.pk, self.pv, self.pkc, self.pvc, qk_norm=True,
                           max_pos0=0, status=self.status)
         if ev is not None:
-            ev[0].record()
+            ev[1].record()
         g.gqa_prefill(self.pq, self.pkc, self.pvc, out=self.pout, status=self.status)
         if ev is not None:
-            ev[1].record()
+            ev[2].record()
         g.gqa_rope_append(self.dq, self.dk, self.dv, self.dkc, self.dvc, pos0=self.pos,
                           max_pos0=self.max_len - 1, new_len=self.lens_new, qk_norm=True,
                           status=self.status)
         if ev is not None:
-            ev[2].record()
+            ev[3].record()
         g.gqa_decode(self.dq, self.dkc, self.dvc, self.lens_new, self.max_len, out=self.dout,
                      workspace=self.ws, status=self.status)
         if ev is not None:
-            ev[3].record()
+            ev[4].record()
 
     def step_e2e(self):
         """Same step from pinned host buffers: H2D inputs, compute, D2H outputs."""
@@ -265,7 +273,7 @@ def run_ours(args, rank, world, dev, dist_on):
         time.sleep(0.3)
 
     # -- device-resident timed region (per-kernel events on the launching stream) --
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     start = torch.cuda.Event(enable_timing=True)
     stop = torch.cuda.Event(enable_timing=True)
     _barrier_sync(dist_on)
@@ -275,12 +283,13 @@ def run_ours(args, rank, world, dev, dist_on):
     stop.record()
     _barrier_sync(dist_on)
     ms_total = start.elapsed_time(stop)
-    t_prefill = t_append_d = t_decode = 0.0
+    t_append_p = t_prefill = t_append_d = t_decode = 0.0
     for i in range(args.steps):
         e = evs[i]
-        t_prefill += e[0].elapsed_time(e[1])
-        t_append_d += e[1].elapsed_time(e[2])
-        t_decode += e[2].elapsed_time(e[3])
+        t_append_p += e[0].elapsed_time(e[1])
+        t_prefill += e[1].elapsed_time(e[2])
+        t_append_d += e[2].elapsed_time(e[3])
+        t_decode += e[3].elapsed_time(e[4])
     ms_total = _max_over_ranks(ms_total, dist_on, dev)
 
     # -- end-to-end region: host buffers in, results out, every step --
@@ -341,13 +350,19 @@ def run_ours(args, rank, world, dev, dist_on):
                             "frac": round(dec_gbs / hpeak, 4), "peak_kind": "hbm copy " + tag,
                             "algorithmic_per_launch": decode_bytes(layer.lens_new_host),
                             "us_per_launch": round(dec_ms * 1e3, 2)},
-        "phases_ms": {"prefill_kernel": round(pf_ms, 4), "decode_kernels": round(dec_ms, 4),
+        "phases_ms": {"prefill_append": round(t_append_p / K, 4),
+                      "prefill_kernel": round(pf_ms, 4),
                       "decode_append": round(t_append_d / K, 4),
-                      "prefill_append": round(ms_step - pf_ms - dec_ms - t_append_d / K, 4)},
+                      "decode_kernels": round(dec_ms, 4)},
+        "append_roofline": {"bound": "hbm", "kernel": "gqa_rope_append (prefill-sized)",
+                            "achieved": round(append_bytes() / (t_append_p / K * 1e-3) / 1e9, 1),
+                            "peak": hpeak, "unit": "GB/s",
+                            "frac": round(append_bytes() / (t_append_p / K * 1e-3) / 1e9 / hpeak, 4),
+                            "algorithmic_per_launch": append_bytes()},
         "e2e": {"value": round(tok / (ms_e2e / K * 1e-3), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": round(ms_e2e / K, 4)},
-        "gpu_launches": 5 * K,
+        "gpu_launches": 4 * K,
         "clocks": clocks,
         "device_status": status,
     }

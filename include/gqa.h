@@ -130,14 +130,18 @@ gqa_status gqa_prefill(const void *q, const void *k_cache, const void *v_cache, 
  *                                      * V[b, h/g, s, :]
  * lens[b] counts the cached tokens INCLUDING the token just appended (the query
  * sits at position lens[b] - 1 and attends to itself).  Split-K over the cache
- * length; each KV head's bytes are read once per group of g query heads.
+ * length in 64-slot chunks; each KV head's bytes are read once per group of g
+ * query heads; a second kernel merges the chunks.
  *   lens: device int32 [B], 1 <= lens[b] <= Lmax (others: GQA_DEV_BAD_LEN /
  *     GQA_DEV_CAPACITY and that sequence's output is zero).
  *   max_len_host: host-known upper bound of lens (<= Lmax); it sizes the grid
  *     and the workspace.  Lengths above it raise GQA_DEV_CAPACITY.
  *   ws, ws_bytes: device scratch of at least
- *     gqa_decode_workspace_bytes(B, Hq, D, max_len_host) bytes; contents on
- *     entry do not matter.  Two calls in flight must not share one workspace.
+ *     gqa_decode_workspace_bytes(B, Hq, D, max_len_host) bytes, 16-byte aligned;
+ *     contents on entry do not matter.  Calls that may run at the same time on
+ *     the GPU must not share one workspace.
+ * Both launches are programmatic dependents of the kernel before them on the
+ * stream (each waits for its predecessor to complete before reading its data).
  */
 gqa_status gqa_decode(const void *q, const void *k_cache, const void *v_cache,
                       const int32_t *lens, int max_len_host, void *out, int B, int Hq,

@@ -189,6 +189,13 @@ def gqa_decode_workspace_bytes(B, Hq, D, max_len):
     return int(load().gqa_decode_workspace_bytes(B, Hq, D, max_len))
 
 
+def decode_workspace(B, Hq, D, max_len, device):
+    """Scratch for gqa_decode; one workspace serves any number of calls that do
+    not run at the same time."""
+    need = gqa_decode_workspace_bytes(B, Hq, D, max_len)
+    return torch.empty(max(need, 16), dtype=torch.uint8, device=device)
+
+
 def gqa_decode(q, k_cache, v_cache, lens, max_len, out=None, workspace=None, scale=0.0,
                status=None, stream=None):
     """One query token per sequence: q [B, Hq, D] against lens[b] cached keys."""
@@ -205,7 +212,7 @@ def gqa_decode(q, k_cache, v_cache, lens, max_len, out=None, workspace=None, sca
     _need(out, "out", torch.bfloat16, 3)
     need = gqa_decode_workspace_bytes(B, Hq, D, max_len)
     if workspace is None:
-        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+        workspace = decode_workspace(B, Hq, D, max_len, q.device)
     _need(workspace, "workspace", torch.uint8)
     if status is not None:
         _need(status, "status", torch.int32)

@@ -6,120 +6,143 @@
 // "从零手训LLaMa：125M模型11小时训练全记录"; the cache is read once per GQA group,
 // never once per query head (first page, section "V2：引入前沿技术").
 //
-// Work split: CTA (split, kv-head [x head subgroup], b) owns CH consecutive cache
-// slots of one KV head and G of its query heads.  One thread issues two bulk
-// copies (the K chunk and the V chunk, each one contiguous [n, D] block of the
-// per-head slab) into shared memory; the four warps then
-//   1. score: 4 lanes per key, each lane D/4 coordinates held against G query
-//      vectors kept in registers; two xor-shuffles finish each dot product.
-//      Lanes visit their 16-byte chunks in a rotated order (and the query
-//      registers were loaded in that same order) so the 8 lanes of each
-//      shared-memory phase hit 8 different bank groups.
-//   2. chunk softmax in base 2: m = max, p = 2^(s - m), l = sum p.
-//   3. p.V: lane (key group, 16-byte column chunk) accumulates G x 8 outputs
-//      over its keys, then the key groups are summed through shared memory.
-// The partial (m, l, o) of each split goes to the workspace; a second kernel,
-// launched as a programmatic dependent of the first, merges the splits of each
-// (b, query head): M = max m_i, o = sum_i 2^(m_i - M) o_i / sum_i 2^(m_i - M) l_i.
+// Work: CTA (chunk, kv-head x head subgroup, b) covers 64 consecutive cache
+// slots of one KV head and G of its query heads (CTAs past a sequence's length
+// exit at once).  One thread issues three bulk copies -- the K chunk and the G
+// query vectors on one barrier, the V chunk on another (each chunk is one
+// contiguous block of the per-head slab) -- and about 33 KB of shared memory
+// lets six CTAs share an SM, so the loads of some overlap the arithmetic of
+// others.  Each of the four warps takes 16 of the chunk's keys through the
+// whole step on its own:
+//   1. score: 8 lanes per key, lane j holding 16-byte chunks j and j+8 of the row
+//      against the G query vectors in registers (packed fma.f32x2); the 8 lanes
+//      of a key read one contiguous 128-byte span (no bank conflicts) and three
+//      xor-shuffles finish each dot product.  The V chunk keeps streaming in.
+//   2. the warp's softmax statistics in base 2 by xor-shuffles: m_w, p, l_w.
+//   3. p.V: each key's p is broadcast by a shuffle, lanes span D.
+//   4. the four warp partials are merged (rescaled to their common maximum) and
+//      the chunk's (m, l, o) go to the workspace.
+// A second kernel, launched as a programmatic dependent of the first, merges
+// the chunks of each (b, query head): M = max m_i,
+// o = sum_i 2^(m_i - M) o_i / sum_i 2^(m_i - M) l_i.  (Merging inside the
+// first kernel -- the last chunk to finish, found with an atomic ticket, merging
+// the rest -- measured slower: every CTA then has to fence its partial writes.)
+#include <algorithm>
+
 #include "common.cuh"
 #include "ptx.cuh"
 
 namespace gqa {
 namespace {
 
-constexpr int kDecThreads = 128;
+constexpr int kDecWarps = 4;
+constexpr int kDecThreads = kDecWarps * 32;
+constexpr int kDecCH = 64;            // cache slots per CTA
+constexpr int kMaxG = 4;              // query heads per CTA, at most
 
-template <int D, int G, int CH>
+template <int D, int G>
 struct DecShape {
-    static constexpr int kLaneChunks = D / 32;                  // 16-byte chunks per lane (score)
-    static constexpr int kPasses = CH / 32;                     // 32 keys per pass
-    static constexpr int kColChunks = D / 8;                    // 16-byte chunks per row (p.V)
-    static constexpr int kKeyGroups = kDecThreads / kColChunks; // p.V key groups
-    static constexpr int kKBytes = CH * D * 2;
-    static constexpr int kPartialBytes = kKeyGroups * G * D * 4;
-    static constexpr bool kAliasPartial = kPartialBytes <= kKBytes;
-    // layout: [K chunk][V chunk][p: G x CH f32][red: 2 x 4 x G f32][partial (if not aliased)]
-    static constexpr int kOffV = kKBytes;
-    static constexpr int kOffP = 2 * kKBytes;
-    static constexpr int kOffRed = kOffP + G * CH * 4;
-    static constexpr int kOffPartial = kAliasPartial ? 0 : kOffRed + 2 * 4 * G * 4;
-    static constexpr int kSmem = (kAliasPartial ? kOffRed + 2 * 4 * G * 4
-                                                : kOffPartial + kPartialBytes) + 16;
+    static constexpr int CH = kDecCH;
+    static constexpr int kKeysPerWarp = CH / kDecWarps;       // 16: four passes of 4 keys
+    static constexpr int kPasses = kKeysPerWarp / 4;
+    static constexpr int kRowChunks = D / 8;                  // 16-byte chunks per cache row
+    static constexpr int kLaneChunks = (kRowChunks + 7) / 8;  // chunks per lane (8 lanes per key)
+    static constexpr int kEPL = D == 64 ? 2 : 4;              // p.V elements per lane
+    static constexpr int kPVLanes = D / kEPL;                 // 32, 24 or 32 active lanes
+    static constexpr int kKVBytes = CH * D * 2;
+    static constexpr int kQBytes = (G * D * 2 + 127) / 128 * 128;
+    // [K | V | q][(m, l): warps x G x 2 f32]; the warps' partial outputs
+    // (warps x G x D f32) are written over the K chunk once every warp has
+    // finished its scores.
+    static constexpr int kOffV = kKVBytes;
+    static constexpr int kOffQ = 2 * kKVBytes;
+    static constexpr int kOffML = kOffQ + kQBytes;
+    static constexpr int kOffPartial = 0;
+    static constexpr int kSmem = kOffML + kDecWarps * G * 2 * 4;
+    static_assert(kDecWarps * G * D * 4 <= kKVBytes, "partials must fit over the K chunk");
 };
 
-// Rotation of a lane's chunk order that keeps each 8-lane phase conflict free.
-template <int D>
-__device__ __forceinline__ int chunk_rot(int lane) {
-    const int j = lane & 3, kl = (lane >> 2) & 1;
-    if (D == 128) return (j >> 1) + 2 * kl;
-    if (D == 64) return kl;
-    return 0;
-}
+// Workspace: [(m, l): rows x 2 f32][o: rows x D f32] with rows = B x Hq x n_splits,
+// row (b, h, c) = (b * Hq + h) * n_splits + c.
 
-template <int D, int G, int CH>
+template <int D, int G>
 __global__ void __launch_bounds__(kDecThreads)
-decode_split_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ kc,
-                    const uint16_t *__restrict__ vc, const int32_t *__restrict__ lens,
-                    int max_len, int Hq, int Hkv, int Lmax, float scale_log2, int n_splits,
-                    int n_sub, float *__restrict__ ws_o, float *__restrict__ ws_ml,
-                    int32_t *status) {
-    using S = DecShape<D, G, CH>;
+decode_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ kc,
+              const uint16_t *__restrict__ vc, const int32_t *__restrict__ lens, int max_len,
+              int Hq, int Hkv, int Lmax, float scale_log2, int n_splits, int n_sub,
+              float *__restrict__ ws_ml, float *__restrict__ ws_o, int32_t *status) {
+    using S = DecShape<D, G>;
+    constexpr int CH = S::CH;
     extern __shared__ __align__(128) uint8_t smem[];
-    __shared__ __align__(8) uint64_t bars[2];
+    __shared__ __align__(8) uint64_t bars[2];     // [0]: K chunk + q, [1]: V chunk
+    __shared__ float sw[kDecWarps * kMaxG];       // warp merge weights [warp][head]
 
-    // The merge kernel may be scheduled now; it waits for this grid to finish
-    // before it reads anything.
+    // Launched as a programmatic dependent of whatever precedes it on the stream
+    // (normally the append that wrote lens and the new K/V slot): wait for it to
+    // complete before reading anything it produced.  The merge kernel may then
+    // be scheduled; it waits for this grid before it reads the partials.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;");
-    const int split = blockIdx.x;
-    const int kvh = blockIdx.y / n_sub;
-    const int sub = blockIdx.y - kvh * n_sub;
+    const int c = blockIdx.x;                     // chunk of the sequence
+    const int kvh = blockIdx.y / n_sub, sub = blockIdx.y - kvh * n_sub;
     const int b = blockIdx.z;
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int g = Hq / Hkv;
+    const int h0 = kvh * g + sub * G;             // first query head of this CTA
     const int len = lens[b];
     if (len < 1 || len > max_len || len > Lmax) {
-        if (split == 0 && blockIdx.y == 0 && tid == 0)
+        if (c == 0 && blockIdx.y == 0 && tid == 0)
             report(status, len < 1 ? GQA_DEV_BAD_LEN : GQA_DEV_CAPACITY);
         return;
     }
-    const int key0 = split * CH;
+    const int key0 = c * CH;
     if (key0 >= len) return;
-    const int n = min(CH, len - key0);
-    const int g = Hq / Hkv;
-    const int h0 = kvh * g + sub * G;        // first query head of this CTA
-
+    const int nk = min(CH, len - key0);
     const uint32_t bar_k = ptx::smem_addr(&bars[0]);
     const uint32_t bar_v = ptx::smem_addr(&bars[1]);
-    const uint16_t *ks = reinterpret_cast<const uint16_t *>(smem);
-    const uint16_t *vs = reinterpret_cast<const uint16_t *>(smem + S::kOffV);
-    float *ps = reinterpret_cast<float *>(smem + S::kOffP);
-    float *red = reinterpret_cast<float *>(smem + S::kOffRed);
-    float *partial = reinterpret_cast<float *>(smem + S::kOffPartial);
-
     if (tid == 0) {
         ptx::mbar_init(bar_k, 1);
         ptx::mbar_init(bar_v, 1);
         ptx::fence_barrier_init();
-        const size_t slab = ((size_t)b * Hkv + kvh) * Lmax + key0;
-        const uint32_t bytes = (uint32_t)n * D * 2;
+        const uint32_t bytes = (uint32_t)nk * D * 2;
+        const size_t slab = (((size_t)b * Hkv + kvh) * Lmax + key0) * D;
         const uint64_t pol = ptx::policy_evict_first();
-        ptx::mbar_arrive_expect_tx(bar_k, bytes);
-        ptx::bulk_g2s_hint(ptx::smem_addr(smem), kc + slab * D, bytes, bar_k, pol);
+        ptx::mbar_arrive_expect_tx(bar_k, bytes + G * D * 2);
+        ptx::bulk_g2s_hint(ptx::smem_addr(smem), kc + slab, bytes, bar_k, pol);
+        ptx::bulk_g2s(ptx::smem_addr(smem + S::kOffQ), q + ((size_t)b * Hq + h0) * D, G * D * 2,
+                      bar_k);
         ptx::mbar_arrive_expect_tx(bar_v, bytes);
-        ptx::bulk_g2s_hint(ptx::smem_addr(smem + S::kOffV), vc + slab * D, bytes, bar_v, pol);
+        ptx::bulk_g2s_hint(ptx::smem_addr(smem + S::kOffV), vc + slab, bytes, bar_v, pol);
+    }
+    __syncthreads();   // barriers initialised before anyone waits on them
+    const uint16_t *ks = reinterpret_cast<const uint16_t *>(smem);
+    const uint16_t *vs = reinterpret_cast<const uint16_t *>(smem + S::kOffV);
+    const uint16_t *qs = reinterpret_cast<const uint16_t *>(smem + S::kOffQ);
+    float *wml = reinterpret_cast<float *>(smem + S::kOffML);           // [warp][G][2]
+    float *partial = reinterpret_cast<float *>(smem + S::kOffPartial);  // [warp][G][D]
+    if (!__syncthreads_and(ptx::mbar_wait(bar_k, 0))) {
+        // A copy that missed its deadline may still land in this CTA's shared
+        // memory: give both one more bounded wait before the CTA retires.
+        ptx::mbar_wait(bar_k, 0);
+        ptx::mbar_wait(bar_v, 0);
+        if (tid == 0) report(status, GQA_DEV_TIMEOUT);
+        return;
     }
 
-    // Query registers, in this lane's rotated chunk order (overlaps the copies).
-    const int lane = tid & 31, warp = tid >> 5;
-    const int j = lane & 3;
-    const int rot = chunk_rot<D>(lane);
+    const int j = lane & 7;          // lane within its key's group of 8
+    const int kq = lane >> 3;        // key slot within a pass
+    const int kw0 = warp * S::kKeysPerWarp;                  // this warp's first key
+    const int kwn = max(0, min(S::kKeysPerWarp, nk - kw0));  // its live keys
+
+    // ---- 1. scores: 8 lanes per key; lane j holds 16-byte chunks j, j+8 ----
     float qr[G][S::kLaneChunks][8];
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
-        const uint16_t *qh = q + ((size_t)b * Hq + h0 + h) * D + j * (D / 4);
+    for (int h = 0; h < G; ++h)
 #pragma unroll
         for (int i = 0; i < S::kLaneChunks; ++i) {
-            const int c = (i + rot) % S::kLaneChunks;
-            const uint4 w = *reinterpret_cast<const uint4 *>(qh + c * 8);
+            const int cc = j + 8 * i;
+            uint4 w = make_uint4(0, 0, 0, 0);
+            if (cc < S::kRowChunks) w = *reinterpret_cast<const uint4 *>(qs + h * D + cc * 8);
             const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -127,218 +150,240 @@ decode_split_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__
                 qr[h][i][2 * e + 1] = bf16hi(ww[e]);
             }
         }
-    }
-    __syncthreads();   // barrier init visible to all threads
-
-    bool ok = ptx::mbar_wait(bar_k, 0);
-    // ---- 1. scores ------------------------------------------------------------
+    float sc[S::kPasses][G];
 #pragma unroll
     for (int pass = 0; pass < S::kPasses; ++pass) {
-        const int key = pass * 32 + warp * 8 + (lane >> 2);
-        const uint16_t *krow = ks + key * D + j * (D / 4);
-        float acc[G];
+        const int kl = pass * 4 + kq;                     // key within the warp's 16
+        const uint16_t *krow = ks + (kw0 + kl) * D;
+        float acc0[G], acc1[G];
 #pragma unroll
-        for (int h = 0; h < G; ++h) acc[h] = 0.f;
+        for (int h = 0; h < G; ++h) acc0[h] = acc1[h] = 0.f;
 #pragma unroll
         for (int i = 0; i < S::kLaneChunks; ++i) {
-            const int c = (i + rot) % S::kLaneChunks;
-            const uint4 w = *reinterpret_cast<const uint4 *>(krow + c * 8);
-            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+            const int cc = j + 8 * i;
+            if (cc < S::kRowChunks) {
+                const uint4 w = *reinterpret_cast<const uint4 *>(krow + cc * 8);
+                const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float k0 = bf16lo(ww[e]), k1 = bf16hi(ww[e]);
+                for (int e = 0; e < 4; ++e) {
+                    const float k0 = bf16lo(ww[e]), k1 = bf16hi(ww[e]);
 #pragma unroll
-                for (int h = 0; h < G; ++h) {
-                    acc[h] = fmaf(qr[h][i][2 * e], k0, acc[h]);
-                    acc[h] = fmaf(qr[h][i][2 * e + 1], k1, acc[h]);
+                    for (int h = 0; h < G; ++h)
+                        ptx::ffma2(acc0[h], acc1[h], qr[h][i][2 * e], qr[h][i][2 * e + 1], k0, k1,
+                                   acc0[h], acc1[h]);
                 }
             }
         }
 #pragma unroll
         for (int h = 0; h < G; ++h) {
-            acc[h] += __shfl_xor_sync(0xffffffffu, acc[h], 1);
-            acc[h] += __shfl_xor_sync(0xffffffffu, acc[h], 2);
+            float a = acc0[h] + acc1[h];
+            a += __shfl_xor_sync(0xffffffffu, a, 1);
+            a += __shfl_xor_sync(0xffffffffu, a, 2);
+            a += __shfl_xor_sync(0xffffffffu, a, 4);
+            sc[pass][h] = kl < kwn ? a * scale_log2 : -INFINITY;
         }
-        if (j == 0) {
+    }
+
+    // ---- 2. the warp's own softmax statistics (base 2) ----
+    float mw[G], lw[G], pw[S::kPasses][G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+        float m = sc[0][h];
+#pragma unroll
+        for (int pass = 1; pass < S::kPasses; ++pass) m = fmaxf(m, sc[pass][h]);
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
+        const float mref = m == -INFINITY ? 0.f : m;      // a warp with no live key
+        float l = 0.f;
+#pragma unroll
+        for (int pass = 0; pass < S::kPasses; ++pass) {
+            pw[pass][h] = ex2(sc[pass][h] - mref);
+            l += pw[pass][h];                             // 8 lanes = one key
+        }
+        l += __shfl_xor_sync(0xffffffffu, l, 8);
+        l += __shfl_xor_sync(0xffffffffu, l, 16);
+        mw[h] = m;
+        lw[h] = l;
+    }
+
+    // ---- 3. p . V over the warp's live keys: lanes span D ----
+    if (!__syncthreads_and(ptx::mbar_wait(bar_v, 0))) {
+        ptx::mbar_wait(bar_v, 0);
+        if (tid == 0) report(status, GQA_DEV_TIMEOUT);
+        return;
+    }
+    float o[G][S::kEPL];
+#pragma unroll
+    for (int h = 0; h < G; ++h)
+#pragma unroll
+        for (int e = 0; e < S::kEPL; ++e) o[h][e] = 0.f;
+#pragma unroll
+    for (int kl = 0; kl < S::kKeysPerWarp; ++kl) {
+        if (kl >= kwn) break;                             // warp-uniform
+        float pk[G];
+#pragma unroll
+        for (int h = 0; h < G; ++h) pk[h] = __shfl_sync(0xffffffffu, pw[kl >> 2][h], (kl & 3) * 8);
+        if (lane < S::kPVLanes) {
+            const uint16_t *vrow = vs + (kw0 + kl) * D;
+            float v[S::kEPL];
+            if constexpr (S::kEPL == 4) {
+                const uint2 w = *reinterpret_cast<const uint2 *>(vrow + lane * 4);
+                v[0] = bf16lo(w.x);
+                v[1] = bf16hi(w.x);
+                v[2] = bf16lo(w.y);
+                v[3] = bf16hi(w.y);
+            } else {
+                const uint32_t w = *reinterpret_cast<const uint32_t *>(vrow + lane * 2);
+                v[0] = bf16lo(w);
+                v[1] = bf16hi(w);
+            }
 #pragma unroll
             for (int h = 0; h < G; ++h)
-                ps[h * CH + key] = key < n ? acc[h] * scale_log2 : -INFINITY;
+#pragma unroll
+                for (int e = 0; e < S::kEPL; e += 2)
+                    ptx::ffma2(o[h][e], o[h][e + 1], pk[h], pk[h], v[e], v[e + 1], o[h][e],
+                               o[h][e + 1]);
         }
     }
-    __syncthreads();
-
-    // ---- 2. chunk softmax (base 2) --------------------------------------------
-    float m[G], l[G];
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-        float s = -INFINITY;
-        for (int key = tid; key < CH; key += kDecThreads) s = fmaxf(s, ps[h * CH + key]);
-        s = warp_max(s);
-        if (lane == 0) red[warp * G + h] = s;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-        m[h] = fmaxf(fmaxf(red[0 * G + h], red[1 * G + h]), fmaxf(red[2 * G + h], red[3 * G + h]));
-        float sum = 0.f;
-        for (int key = tid; key < CH; key += kDecThreads) {
-            const float p = ex2(ps[h * CH + key] - m[h]);
-            ps[h * CH + key] = p;
-            sum += p;
-        }
-        sum = warp_sum(sum);
-        if (lane == 0) red[4 * G + warp * G + h] = sum;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int h = 0; h < G; ++h)
-        l[h] = (red[4 * G + 0 * G + h] + red[4 * G + 1 * G + h]) +
-               (red[4 * G + 2 * G + h] + red[4 * G + 3 * G + h]);
-
-    // ---- 3. p . V ---------------------------------------------------------------
-    ok = ptx::mbar_wait(bar_v, 0) && ok;
-    const int col = tid % S::kColChunks;
-    const int kg = tid / S::kColChunks;
-    float o[G][8];
-#pragma unroll
-    for (int h = 0; h < G; ++h)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) o[h][e] = 0.f;
-    if (kg < S::kKeyGroups) {
-        for (int key = kg; key < n; key += S::kKeyGroups) {
-            const uint4 w = *reinterpret_cast<const uint4 *>(vs + key * D + col * 8);
-            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-            float pv[G];
-#pragma unroll
-            for (int h = 0; h < G; ++h) pv[h] = ps[h * CH + key];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float v0 = bf16lo(ww[e]), v1 = bf16hi(ww[e]);
-#pragma unroll
-                for (int h = 0; h < G; ++h) {
-                    o[h][2 * e] = fmaf(pv[h], v0, o[h][2 * e]);
-                    o[h][2 * e + 1] = fmaf(pv[h], v1, o[h][2 * e + 1]);
-                }
-            }
-        }
-    }
-    if (S::kAliasPartial) __syncthreads();   // every lane is done reading K
-    if (kg < S::kKeyGroups) {
+    if (lane < S::kPVLanes) {
 #pragma unroll
         for (int h = 0; h < G; ++h) {
-            float4 *dst = reinterpret_cast<float4 *>(partial + (kg * G + h) * D + col * 8);
-            dst[0] = make_float4(o[h][0], o[h][1], o[h][2], o[h][3]);
-            dst[1] = make_float4(o[h][4], o[h][5], o[h][6], o[h][7]);
+            float *dst = partial + (warp * G + h) * D + lane * S::kEPL;
+            if constexpr (S::kEPL == 4)
+                *reinterpret_cast<float4 *>(dst) = make_float4(o[h][0], o[h][1], o[h][2], o[h][3]);
+            else
+                *reinterpret_cast<float2 *>(dst) = make_float2(o[h][0], o[h][1]);
+        }
+    }
+    if (lane == 0) {
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            wml[(warp * G + h) * 2] = mw[h];
+            wml[(warp * G + h) * 2 + 1] = lw[h];
         }
     }
     __syncthreads();
-    const size_t row0 = ((size_t)b * Hq + h0) * n_splits + split;   // (b, h0, split)
+
+    // ---- 4. merge the warps; the chunk's (m, l, o) to the workspace ----
+    const size_t row0 = ((size_t)b * Hq + h0) * n_splits + c;
+    if (tid < G) {
+        const int h = tid;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, wml[(w * G + h) * 2]);
+        float L = 0.f;
+#pragma unroll
+        for (int w = 0; w < kDecWarps; ++w) {
+            const float mwv = wml[(w * G + h) * 2];
+            const float f = mwv == -INFINITY ? 0.f : ex2(mwv - M);
+            sw[w * kMaxG + h] = f;
+            L = fmaf(f, wml[(w * G + h) * 2 + 1], L);
+        }
+        ws_ml[(row0 + (size_t)h * n_splits) * 2 + 0] = M;
+        ws_ml[(row0 + (size_t)h * n_splits) * 2 + 1] = L;
+    }
+    __syncthreads();
     for (int idx = tid; idx < G * D; idx += kDecThreads) {
         const int h = idx / D, d = idx - h * D;
         float acc = 0.f;
-#pragma unroll 4
-        for (int gi = 0; gi < S::kKeyGroups; ++gi) acc += partial[(gi * G + h) * D + d];
+#pragma unroll
+        for (int w = 0; w < kDecWarps; ++w)
+            acc = fmaf(sw[w * kMaxG + h], partial[(w * G + h) * D + d], acc);
         ws_o[(row0 + (size_t)h * n_splits) * D + d] = acc;
     }
-    if (tid < G) {
-        float mm = 0.f, ll = 0.f;
-#pragma unroll
-        for (int h = 0; h < G; ++h)
-            if (h == tid) { mm = m[h]; ll = l[h]; }
-        ws_ml[(row0 + (size_t)tid * n_splits) * 2 + 0] = mm;
-        ws_ml[(row0 + (size_t)tid * n_splits) * 2 + 1] = ll;
-    }
-    if (!ok) {
-        // A copy that missed its deadline may still land in this CTA's shared
-        // memory: give both one more bounded wait before the CTA retires.
-        ptx::mbar_wait(bar_k, 0);
-        ptx::mbar_wait(bar_v, 0);
-        if (tid == 0) report(status, GQA_DEV_TIMEOUT);
-    }
+
 }
 
-// Merge the splits of one (b, query head): one warp per row.  Lanes read the
-// splits' (m, l) in parallel and reduce them with shuffles; each lane then owns
-// D/32 output coordinates and walks the splits with independent loads.
-constexpr int kCombWarps = 8;
+// Merge the chunks of one (b, query head): one CTA per row, one thread per output
+// coordinate.  Warp 0 turns the chunks' maxima into weights 2^(m_i - M) in shared
+// memory; then every thread walks the chunks with independent coalesced loads.
+constexpr int kCombMaxStored = 1024;      // chunk weights kept in shared memory
 
-template <int D>
-__global__ void __launch_bounds__(kCombWarps * 32)
-decode_combine_kernel(const float *__restrict__ ws_o, const float *__restrict__ ws_ml,
-                      const int32_t *__restrict__ lens, int max_len, int B, int Hq, int Lmax,
-                      int n_splits, int CH, uint16_t *__restrict__ out) {
-    // Programmatic dependent launch: everything above this line may overlap the
-    // split kernel; the partials are read only after it has completed.
+__global__ void __launch_bounds__(128)
+decode_merge_kernel(const float *__restrict__ ws_ml, const float *__restrict__ ws_o,
+                    const int32_t *__restrict__ lens, int max_len, int Hq, int D, int Lmax,
+                    int n_splits, uint16_t *__restrict__ out) {
+    __shared__ float wsplit[kCombMaxStored];
+    __shared__ float stats[2];
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    const int lane = threadIdx.x & 31;
-    const int row = blockIdx.x * kCombWarps + (threadIdx.x >> 5);   // b * Hq + h
-    if (row >= B * Hq) return;
+    const int row = blockIdx.x;                   // b * Hq + h
     const int b = row / Hq;
+    const int tid = threadIdx.x, lane = tid & 31;
     const int len = lens[b];
-    constexpr int kPer = D / 32;
     uint16_t *o = out + (size_t)row * D;
     if (len < 1 || len > max_len || len > Lmax) {
-#pragma unroll
-        for (int k = 0; k < kPer; ++k) o[lane + 32 * k] = 0;
+        for (int d = tid; d < D; d += blockDim.x) o[d] = 0;
         return;
     }
-    const int ns = (len + CH - 1) / CH;
+    const int ns = (len + kDecCH - 1) / kDecCH;
     const float *ml = ws_ml + (size_t)row * n_splits * 2;
     const float *po = ws_o + (size_t)row * n_splits * D;
-    float M = -INFINITY;
-    for (int i = lane; i < ns; i += 32) M = fmaxf(M, ml[2 * i]);
-    M = warp_max(M);
-    float L = 0.f;
-    for (int i = lane; i < ns; i += 32) L = fmaf(ex2(ml[2 * i] - M), ml[2 * i + 1], L);
-    L = warp_sum(L);
-    float acc[kPer];
-#pragma unroll
-    for (int k = 0; k < kPer; ++k) acc[k] = 0.f;
-#pragma unroll 4
-    for (int i = 0; i < ns; ++i) {
-        const float w = ex2(ml[2 * i] - M);
-#pragma unroll
-        for (int k = 0; k < kPer; ++k) acc[k] = fmaf(w, po[(size_t)i * D + lane + 32 * k], acc[k]);
+    const bool stored = ns <= kCombMaxStored;
+    if (tid < 32) {
+        float M = -INFINITY;
+        for (int i = lane; i < ns; i += 32) M = fmaxf(M, ml[2 * i]);
+        M = warp_max(M);
+        float L = 0.f;
+        for (int i = lane; i < ns; i += 32) {
+            const float w = ex2(ml[2 * i] - M);
+            if (stored) wsplit[i] = w;
+            L = fmaf(w, ml[2 * i + 1], L);
+        }
+        L = warp_sum(L);
+        if (lane == 0) {
+            stats[0] = M;
+            stats[1] = L;
+        }
     }
-    const float inv = 1.f / L;
-#pragma unroll
-    for (int k = 0; k < kPer; ++k)
-        o[lane + 32 * k] = (uint16_t)(pack_bf16x2(acc[k] * inv, 0.f) & 0xffffu);
+    __syncthreads();
+    const float M = stats[0], inv = 1.f / stats[1];
+    for (int d = tid; d < D; d += blockDim.x) {
+        float acc = 0.f;
+        if (stored) {
+#pragma unroll 8
+            for (int i = 0; i < ns; ++i) acc = fmaf(wsplit[i], po[(size_t)i * D + d], acc);
+        } else {
+            for (int i = 0; i < ns; ++i) acc = fmaf(ex2(ml[2 * i] - M), po[(size_t)i * D + d], acc);
+        }
+        o[d] = (uint16_t)(pack_bf16x2(acc * inv, 0.f) & 0xffffu);
+    }
 }
 
-template <int D, int G, int CH>
+template <int D, int G>
 cudaError_t launch_decode(const void *q, const void *kc, const void *vc, const int32_t *lens,
                           int max_len, void *out, int B, int Hq, int Hkv, int Lmax,
-                          float scale_log2, float *ws_o, float *ws_ml, int n_splits,
-                          int32_t *status, cudaStream_t s) {
-    using S = DecShape<D, G, CH>;
-    auto kern = decode_split_kernel<D, G, CH>;
+                          float scale_log2, void *ws, int n_splits, int32_t *status,
+                          cudaStream_t s) {
+    using S = DecShape<D, G>;
+    auto kern = decode_kernel<D, G>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          S::kSmem);
     if (e != cudaSuccess) return e;
     const int n_sub = (Hq / Hkv) / G;
-    dim3 grid(n_splits, Hkv * n_sub, B);
-    kern<<<grid, kDecThreads, S::kSmem, s>>>(
-        static_cast<const uint16_t *>(q), static_cast<const uint16_t *>(kc),
-        static_cast<const uint16_t *>(vc), lens, max_len, Hq, Hkv, Lmax, scale_log2, n_splits,
-        n_sub, ws_o, ws_ml, status);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    // The merge is launched as a programmatic dependent of the split kernel, so
-    // its launch and scheduling overlap the split kernel's last wave.
+    const size_t rows = (size_t)B * Hq * n_splits;
+    float *ws_ml = static_cast<float *>(ws);
+    float *ws_o = ws_ml + rows * 2;
+    // Both launches are programmatic dependents of the kernel before them.
+    cudaLaunchAttribute pdl[1];
+    pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl[0].val.programmaticStreamSerializationAllowed = 1;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)((B * Hq + kCombWarps - 1) / kCombWarps));
-    cfg.blockDim = dim3(kCombWarps * 32);
-    cfg.dynamicSmemBytes = 0;
+    cfg.gridDim = dim3(n_splits, Hkv * n_sub, B);
+    cfg.blockDim = dim3(kDecThreads);
+    cfg.dynamicSmemBytes = S::kSmem;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
+    cfg.attrs = pdl;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, decode_combine_kernel<D>, (const float *)ws_o,
-                              (const float *)ws_ml, lens, max_len, B, Hq, Lmax, n_splits, CH,
-                              static_cast<uint16_t *>(out));
+    e = cudaLaunchKernelEx(&cfg, kern, static_cast<const uint16_t *>(q),
+                           static_cast<const uint16_t *>(kc), static_cast<const uint16_t *>(vc),
+                           lens, max_len, Hq, Hkv, Lmax, scale_log2, n_splits, n_sub, ws_ml, ws_o,
+                           status);
+    if (e != cudaSuccess) return e;
+    cfg.gridDim = dim3((unsigned)(B * Hq));
+    cfg.blockDim = dim3(128);
+    cfg.dynamicSmemBytes = 0;
+    return cudaLaunchKernelEx(&cfg, decode_merge_kernel, (const float *)ws_ml, (const float *)ws_o,
+                              lens, max_len, Hq, D, Lmax, n_splits, static_cast<uint16_t *>(out));
 }
 
 // Query heads per CTA: the largest of {3, 2, 1} (D = 128) or {4, 3, 2, 1}
@@ -350,28 +395,19 @@ int heads_per_cta(int g, int D) {
     return 1;
 }
 
-template <int D, int CH>
+template <int D>
 cudaError_t launch_g(int G, const void *q, const void *kc, const void *vc, const int32_t *lens,
                      int max_len, void *out, int B, int Hq, int Hkv, int Lmax, float sl2,
-                     float *wo, float *wml, int ns, int32_t *st, cudaStream_t s) {
+                     void *ws, int ns, int32_t *st, cudaStream_t s) {
     switch (G) {
-        case 1: return launch_decode<D, 1, CH>(q, kc, vc, lens, max_len, out, B, Hq, Hkv, Lmax, sl2, wo, wml, ns, st, s);
-        case 2: return launch_decode<D, 2, CH>(q, kc, vc, lens, max_len, out, B, Hq, Hkv, Lmax, sl2, wo, wml, ns, st, s);
-        case 3: return launch_decode<D, 3, CH>(q, kc, vc, lens, max_len, out, B, Hq, Hkv, Lmax, sl2, wo, wml, ns, st, s);
+        case 1: return launch_decode<D, 1>(q, kc, vc, lens, max_len, out, B, Hq, Hkv, Lmax, sl2, ws, ns, st, s);
+        case 2: return launch_decode<D, 2>(q, kc, vc, lens, max_len, out, B, Hq, Hkv, Lmax, sl2, ws, ns, st, s);
+        case 3: return launch_decode<D, 3>(q, kc, vc, lens, max_len, out, B, Hq, Hkv, Lmax, sl2, ws, ns, st, s);
         default:
             if constexpr (D != 128)
-                return launch_decode<D, 4, CH>(q, kc, vc, lens, max_len, out, B, Hq, Hkv, Lmax, sl2, wo, wml, ns, st, s);
+                return launch_decode<D, 4>(q, kc, vc, lens, max_len, out, B, Hq, Hkv, Lmax, sl2, ws, ns, st, s);
             return cudaErrorInvalidValue;
     }
-}
-
-constexpr int kMinSplitChunk = 64;
-
-// Chunk length: 128 slots when that still yields about two CTAs per SM,
-// otherwise 64 (short caches / small batches are latency-bound).
-int pick_chunk(int B, int Hkv, int n_sub, int max_len) {
-    const long long ctas128 = (long long)B * Hkv * n_sub * ((max_len + 127) / 128);
-    return ctas128 >= 2 * 148 ? 128 : 64;
 }
 
 }  // namespace
@@ -379,9 +415,9 @@ int pick_chunk(int B, int Hkv, int n_sub, int max_len) {
 
 extern "C" size_t gqa_decode_workspace_bytes(int B, int Hq, int D, int max_len) {
     if (B < 1 || Hq < 1 || max_len < 1 || !gqa_host::head_dim_ok(D)) return 0;
-    const size_t ns = (size_t)(max_len + gqa::kMinSplitChunk - 1) / gqa::kMinSplitChunk;
+    const size_t ns = (size_t)(max_len + gqa::kDecCH - 1) / gqa::kDecCH;
     const size_t rows = (size_t)B * Hq * ns;
-    return rows * (size_t)D * 4 + rows * 2 * 4 + 256;
+    return rows * 2 * 4 + rows * (size_t)D * 4;
 }
 
 extern "C" gqa_status gqa_decode(const void *q, const void *k_cache, const void *v_cache,
@@ -404,27 +440,15 @@ extern "C" gqa_status gqa_decode(const void *q, const void *k_cache, const void 
 
     const int g = Hq / Hkv;
     const int G = gqa::heads_per_cta(g, D);
-    const int CH = gqa::pick_chunk(B, Hkv, g / G, max_len_host);
-    const int ns = (max_len_host + CH - 1) / CH;
-    const size_t rows = (size_t)B * Hq * ns;
-    float *ws_o = static_cast<float *>(ws);
-    float *ws_ml = ws_o + rows * D;
+    const int ns = (max_len_host + gqa::kDecCH - 1) / gqa::kDecCH;
     const float sc = scale > 0.f ? scale : 1.0f / sqrtf((float)D);
     const float sl2 = sc * 1.4426950408889634f;   // scores in base-2 units
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e;
-    if (CH == 128) {
-        switch (D) {
-            case 64: e = gqa::launch_g<64, 128>(G, q, k_cache, v_cache, lens, max_len_host, out, B, Hq, Hkv, Lmax, sl2, ws_o, ws_ml, ns, status_dev, s); break;
-            case 96: e = gqa::launch_g<96, 128>(G, q, k_cache, v_cache, lens, max_len_host, out, B, Hq, Hkv, Lmax, sl2, ws_o, ws_ml, ns, status_dev, s); break;
-            default: e = gqa::launch_g<128, 128>(G, q, k_cache, v_cache, lens, max_len_host, out, B, Hq, Hkv, Lmax, sl2, ws_o, ws_ml, ns, status_dev, s); break;
-        }
-    } else {
-        switch (D) {
-            case 64: e = gqa::launch_g<64, 64>(G, q, k_cache, v_cache, lens, max_len_host, out, B, Hq, Hkv, Lmax, sl2, ws_o, ws_ml, ns, status_dev, s); break;
-            case 96: e = gqa::launch_g<96, 64>(G, q, k_cache, v_cache, lens, max_len_host, out, B, Hq, Hkv, Lmax, sl2, ws_o, ws_ml, ns, status_dev, s); break;
-            default: e = gqa::launch_g<128, 64>(G, q, k_cache, v_cache, lens, max_len_host, out, B, Hq, Hkv, Lmax, sl2, ws_o, ws_ml, ns, status_dev, s); break;
-        }
+    switch (D) {
+        case 64: e = gqa::launch_g<64>(G, q, k_cache, v_cache, lens, max_len_host, out, B, Hq, Hkv, Lmax, sl2, ws, ns, status_dev, s); break;
+        case 96: e = gqa::launch_g<96>(G, q, k_cache, v_cache, lens, max_len_host, out, B, Hq, Hkv, Lmax, sl2, ws, ns, status_dev, s); break;
+        default: e = gqa::launch_g<128>(G, q, k_cache, v_cache, lens, max_len_host, out, B, Hq, Hkv, Lmax, sl2, ws, ns, status_dev, s); break;
     }
     return e == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
 }

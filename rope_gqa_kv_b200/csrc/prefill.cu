@@ -81,6 +81,9 @@ template <int D>
 __device__ void producer(const PfMaps &maps, PfSync &sy, uint8_t *smem, int b, int h, int kvh,
                          int Hkv, int q0, bool has1, int n_kv, int32_t *status) {
     using S = PfShape<D>;
+    // The kernel is a programmatic dependent of the preceding one (normally the
+    // append that rotated q and filled the cache): wait for it before loading.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const uint32_t qbytes = S::kTileBytes * (has1 ? 2 : 1);
     ptx::mbar_arrive_expect_tx(A(sy.q_full), qbytes);
     for (int t = 0; t < (has1 ? 2 : 1); ++t)
@@ -459,8 +462,22 @@ gqa_status launch_prefill(const void *q, const void *kc, const void *vc, void *o
     if (attr.numRegs != kLaunchRegs) return GQA_ERR_UNSUPPORTED;
     const int n_pairs = (T + 255) / 256;
     const long long grid = (long long)n_pairs * Hq * B;
-    kern<<<(unsigned)grid, kPfThreads, S::kSmem, s>>>(maps, static_cast<uint16_t *>(out), B, T,
-                                                      Hq, Hkv, scale_log2, n_pairs, status);
+    // Programmatic dependent launch: the prologue (barriers, tensor memory,
+    // descriptor prefetch) overlaps the tail of the preceding kernel; the TMA
+    // producer waits for that kernel before its first load.
+    cudaLaunchAttribute pdl[1];
+    pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kPfThreads);
+    cfg.dynamicSmemBytes = S::kSmem;
+    cfg.stream = s;
+    cfg.attrs = pdl;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, maps, static_cast<uint16_t *>(out), B, T, Hq, Hkv,
+                           scale_log2, n_pairs, status) != cudaSuccess)
+        return GQA_ERR_CUDA;
     return gqa_host::launch_status();
 }
 

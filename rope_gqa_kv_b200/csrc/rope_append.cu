@@ -100,6 +100,10 @@ rope_append_kernel(uint16_t *__restrict__ q, const uint16_t *__restrict__ k,
     using S = RopeShape<D>;
     __shared__ float cs[S::kHalf];
     __shared__ float sn[S::kHalf];
+    // A kernel launched after this one as a programmatic dependent (the prefill
+    // or the decode) may start its prologue now; it waits for this grid to
+    // complete before it reads anything written here.
+    asm volatile("griddepcontrol.launch_dependents;");
 
     const int token = blockIdx.x;              // b * T + t
     const int b = token / T;

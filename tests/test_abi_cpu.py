@@ -54,8 +54,9 @@ def test_status_strings_and_version(lib):
 
 
 def test_workspace_size(lib):
-    # B * Hq * ceil(max_len / 64) rows of (D + 2) floats, plus slack
-    assert lib.gqa_decode_workspace_bytes(64, 24, 128, 2049) == 64 * 24 * 33 * (128 + 2) * 4 + 256
+    # B * Hq * ceil(max_len / 64) rows of (D + 2) floats
+    assert lib.gqa_decode_workspace_bytes(64, 24, 128, 2049) == 64 * 24 * 33 * (128 + 2) * 4
+    assert lib.gqa_decode_workspace_bytes(1, 3, 64, 64) == 3 * (64 + 2) * 4
     assert lib.gqa_decode_workspace_bytes(0, 24, 128, 100) == 0
     assert lib.gqa_decode_workspace_bytes(1, 24, 80, 100) == 0
 

@@ -161,3 +161,28 @@ def test_cached_decode_matches_longer_prefill_on_gpu(cuda_lib):
         pos = pos + 1
     torch.cuda.synchronize()
     assert torch.equal(kc.view(torch.int16), kc2.view(torch.int16))
+
+
+def test_workspace_reuse_and_garbage_contents(cuda_lib):
+    """One workspace serves consecutive calls (same bits each time), whatever it
+    held before (it is filled with garbage first)."""
+    w = inputs.custom("dec", B=7, Hq=12, Hkv=4, D=128, decode_steps=1, qk_norm=False,
+                      cached_len_range=(1, 900), seed_index=33)
+    x = inputs.make_inputs(w)
+    q = x["steps"][0][0].to(DEV)
+    kc, vc = x["k_cache"].to(DEV), x["v_cache"].to(DEV)
+    lens = x["lens"].to(DEV)
+    max_len = int(x["lens"].max())
+    ws = gqa.decode_workspace(w.B, w.Hq, w.D, max_len, DEV)
+    ws.random_(0, 256)
+    outs = []
+    for _ in range(3):
+        outs.append(gqa.gqa_decode(q, kc, vc, lens, max_len, workspace=ws))
+        torch.cuda.synchronize()
+    assert torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16))
+    assert torch.equal(outs[0].view(torch.int16), outs[2].view(torch.int16))
+    want = oracle.attention(oracle.bf16_to_f64(bits(x["steps"][0][0]))[:, None],
+                            oracle.bf16_to_f64(bits(x["k_cache"])).transpose(0, 2, 1, 3),
+                            oracle.bf16_to_f64(bits(x["v_cache"])).transpose(0, 2, 1, 3),
+                            (x["lens"].numpy() - 1)[:, None].astype(np.int64))[:, 0]
+    assert_close(outs[0], want, "decode with a reused workspace")
