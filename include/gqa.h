@@ -151,6 +151,33 @@ gqa_status gqa_decode(const void *q, const void *k_cache, const void *v_cache,
 /* Bytes of workspace gqa_decode needs for these sizes (0 on invalid sizes). */
 size_t gqa_decode_workspace_bytes(int B, int Hq, int D, int max_len);
 
+/* Size of the fixed device array gqa_decode_noalloc keeps its scratch in. */
+#define GQA_DECODE_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+/*
+ * gqa_decode_noalloc -- gqa_decode for callers that cannot provide device
+ * scratch memory (no allocator is available to them, or they must not allocate
+ * once running).  The paper has no counterpart of this call; it is a property
+ * of this library.  Same arguments and results as gqa_decode minus the
+ * workspace: the scratch is a GQA_DECODE_NOALLOC_SCRATCH_BYTES (32 MiB) array
+ * inside the library, present on every GPU that loads the library until the
+ * process exits; nothing is allocated per call.
+ *   - Sizes whose gqa_decode_workspace_bytes(B, Hq, D, max_len_host) exceeds
+ *     32 MiB return GQA_ERR_WORKSPACE (the 64 x 24-head x 2049-slot batched
+ *     decode needs 26.4 MB).
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current) and keeps it; make that first call before any stream
+ *     capture.
+ *   - Every call on a device uses the same array: calls that may overlap on the
+ *     GPU (different streams without ordering) race and corrupt each other.
+ *     Calls ordered on one stream are fine; no part of the array has to start
+ *     at zero.
+ */
+gqa_status gqa_decode_noalloc(const void *q, const void *k_cache, const void *v_cache,
+                              const int32_t *lens, int max_len_host, void *out, int B, int Hq,
+                              int Hkv, int D, int Lmax, float scale, int32_t *status_dev,
+                              void *stream);
+
 /* Static, human-readable text for a status code. */
 const char *gqa_status_string(gqa_status s);
 

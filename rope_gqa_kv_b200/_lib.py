@@ -41,6 +41,7 @@ SIGNATURES = {
     "gqa_decode": (_i, [_vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _f, _vp, _sz,
                         _vp, _vp]),
     "gqa_decode_workspace_bytes": (_sz, [_i, _i, _i, _i]),
+    "gqa_decode_noalloc": (_i, [_vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _f, _vp, _vp]),
     "gqa_status_string": (ctypes.c_char_p, [_i]),
     "gqa_version": (_i, []),
 }
@@ -220,4 +221,27 @@ def gqa_decode(q, k_cache, v_cache, lens, max_len, out=None, workspace=None, sca
         _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(lens), int(max_len), _ptr(out), B, Hq, Hkv,
         D, Lmax, float(scale), _ptr(workspace), workspace.numel(), _ptr(status),
         _stream(stream)))
+    return out
+
+
+def gqa_decode_noalloc(q, k_cache, v_cache, lens, max_len, out=None, scale=0.0, status=None,
+                       stream=None):
+    """gqa_decode with its scratch in the library's fixed device array (no
+    workspace argument); for callers that cannot allocate device memory."""
+    _need(q, "q", torch.bfloat16, 3)
+    _need(k_cache, "k_cache", torch.bfloat16, 4)
+    _need(v_cache, "v_cache", torch.bfloat16, 4)
+    _need(lens, "lens", torch.int32, 1)
+    B, Hq, D = q.shape
+    Hkv, Lmax = k_cache.shape[1], k_cache.shape[2]
+    if k_cache.shape != (B, Hkv, Lmax, D) or v_cache.shape != k_cache.shape:
+        raise ValueError("cache shape disagrees with q")
+    if out is None:
+        out = torch.empty_like(q)
+    _need(out, "out", torch.bfloat16, 3)
+    if status is not None:
+        _need(status, "status", torch.int32)
+    _check("gqa_decode_noalloc", load().gqa_decode_noalloc(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(lens), int(max_len), _ptr(out), B, Hq, Hkv,
+        D, Lmax, float(scale), _ptr(status), _stream(stream)))
     return out

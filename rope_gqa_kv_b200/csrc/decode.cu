@@ -28,6 +28,7 @@
 // first kernel -- the last chunk to finish, found with an atomic ticket, merging
 // the rest -- measured slower: every CTA then has to fence its partial writes.)
 #include <algorithm>
+#include <mutex>
 
 #include "common.cuh"
 #include "ptx.cuh"
@@ -451,4 +452,59 @@ extern "C" gqa_status gqa_decode(const void *q, const void *k_cache, const void 
         default: e = gqa::launch_g<128>(G, q, k_cache, v_cache, lens, max_len_host, out, B, Hq, Hkv, Lmax, sl2, ws, ns, status_dev, s); break;
     }
     return e == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
+// gqa_decode_noalloc: the same decode with its scratch in a fixed device array
+// ---------------------------------------------------------------------------
+// Some callers cannot hand this library any device scratch: a host framework
+// that owns every byte of device memory and gives its plugins no allocator, or
+// a serving loop that must not call cudaMalloc once it is running (the call
+// synchronises the device and can fail when memory is tight).  For them the
+// decode can keep its partial results in this file-scope array instead of a
+// caller workspace.  The array is created with the module on every GPU that
+// loads the library and lives until the process exits; the decode needs no
+// part of it to start at zero.  Host code cannot use `g_noalloc_scratch` as an
+// address (it names a host-side stand-in), so the device address is looked up
+// once per device with cudaGetSymbolAddress.
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = GQA_DECODE_NOALLOC_SCRATCH_BYTES;
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void *g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device (looked up once).
+gqa_status noalloc_scratch(void **ptr) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return GQA_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return GQA_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (!g_noalloc_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p)
+            return GQA_ERR_CUDA;
+        g_noalloc_ptr[dev] = p;
+    }
+    *ptr = g_noalloc_ptr[dev];
+    return GQA_OK;
+}
+
+}  // namespace
+
+extern "C" gqa_status gqa_decode_noalloc(const void *q, const void *k_cache, const void *v_cache,
+                                         const int32_t *lens, int max_len_host, void *out, int B,
+                                         int Hq, int Hkv, int D, int Lmax, float scale,
+                                         int32_t *status_dev, void *stream) {
+    if (B < 1 || Hq < 1 || max_len_host < 1 || !gqa_host::head_dim_ok(D))
+        return gqa_host::head_dim_ok(D) ? GQA_ERR_INVALID_ARG : GQA_ERR_UNSUPPORTED;
+    const size_t need = gqa_decode_workspace_bytes(B, Hq, D, max_len_host);
+    if (need == 0 || need > kNoAllocScratchBytes) return GQA_ERR_WORKSPACE;
+    void *scratch = nullptr;
+    const gqa_status st = noalloc_scratch(&scratch);
+    if (st != GQA_OK) return st;
+    return gqa_decode(q, k_cache, v_cache, lens, max_len_host, out, B, Hq, Hkv, D, Lmax, scale,
+                      scratch, kNoAllocScratchBytes, status_dev, stream);
 }
