@@ -4,7 +4,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include "../../include/gqa.h"
+#include "gqa.h"
 
 namespace gqa {
 

@@ -42,11 +42,11 @@ constexpr int kPfThreads = 384;   // three warpgroups
 constexpr int kTmaWarp = 8;
 constexpr int kMmaWarp = 9;
 // Registers: launched at 168 per thread (65536 / 384, rounded down to 8); the two
-// softmax warpgroups take 224 each and the producer/MMA warpgroup keeps 56:
-// 2 * 224 + 56 = 3 * 168, so the increases are exactly covered by the decrease.
+// softmax warpgroups take 208 each and the producer/MMA warpgroup keeps 88:
+// 2 * 208 + 88 = 3 * 168, so the increases are exactly covered by the decrease.
 constexpr int kLaunchRegs = 168;
-constexpr uint32_t kSoftmaxRegs = 224;
-constexpr uint32_t kControlRegs = 56;
+constexpr uint32_t kSoftmaxRegs = 208;
+constexpr uint32_t kControlRegs = 88;
 static_assert(2 * kSoftmaxRegs + kControlRegs == 3 * kLaunchRegs, "register split must balance");
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale O only past 2^8 growth
 
@@ -55,11 +55,15 @@ struct PfShape {
     static constexpr int kBlocks = (D + 63) / 64;           // 128-byte column blocks
     static constexpr int kBlockBytes = 128 * 128;           // 128 rows x 128 bytes
     static constexpr int kTileBytes = kBlocks * kBlockBytes;
-    static constexpr int kStages = D == 64 ? 4 : 2;
+    // K and V rings: as deep as the 227 KB of shared memory allows next to the
+    // two Q tiles (D = 128: K 3 + V 2 stages of 32 KB; D = 64: 4 + 4 of 16 KB).
+    static constexpr int kStagesK = D == 64 ? 4 : 3;
+    static constexpr int kStagesV = D == 64 ? 4 : 2;
     static constexpr int kOffQ = 0;
     static constexpr int kOffK = 2 * kTileBytes;
-    static constexpr int kOffV = kOffK + kStages * kTileBytes;
-    static constexpr int kSmem = kOffV + kStages * kTileBytes + 1024;   // + 1 KB alignment slack
+    static constexpr int kOffV = kOffK + kStagesK * kTileBytes;
+    static constexpr int kSmem = kOffV + kStagesV * kTileBytes + 1024;   // + 1 KB alignment slack
+    static_assert(kSmem <= 227 * 1024, "shared memory per CTA");
     static constexpr int kKSteps = D / 16;
 };
 
@@ -68,7 +72,7 @@ struct PfMaps {
 };
 
 struct PfSync {
-    uint64_t q_full;
+    uint64_t q_full, q_empty;
     uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
     uint64_t s_full[2], p_full[2], o_final[2];
     uint64_t mma_done;
@@ -77,53 +81,96 @@ struct PfSync {
 
 __device__ __forceinline__ uint32_t A(const uint64_t &b) { return ptx::smem_addr(&b); }
 
+// Work item w of the grid's items: the query-tile pair, head and sequence it
+// covers.  Items are numbered longest first (pairs nearer the end of the
+// prompt see more keys), with the heads of one KV group side by side.
+struct PfItem {
+    int b, h, kvh, q0, n0, n1, n_kv;
+    bool has1;
+};
+
+__device__ __forceinline__ PfItem pf_item(int w, int n_pairs, int B, int T, int Hq, int Hkv) {
+    const int per_pair = Hq * B;
+    const int pi = w / per_pair;
+    const int rest = w - pi * per_pair;
+    PfItem it;
+    it.h = rest % Hq;
+    it.b = rest / Hq;
+    it.kvh = it.h / (Hq / Hkv);
+    it.q0 = (n_pairs - 1 - pi) * 256;
+    it.has1 = it.q0 + 128 < T;
+    it.n0 = (min(T, it.q0 + 128) + 127) / 128;
+    it.n1 = it.has1 ? (min(T, it.q0 + 256) + 127) / 128 : 0;
+    it.n_kv = it.has1 ? it.n1 : it.n0;
+    return it;
+}
+
+struct PfGrid {
+    int n_items, n_pairs, B, T, Hq, Hkv;
+};
+
 template <int D>
-__device__ void producer(const PfMaps &maps, PfSync &sy, uint8_t *smem, int b, int h, int kvh,
-                         int Hkv, int q0, bool has1, int n_kv, int32_t *status) {
+__device__ void producer(const PfMaps &maps, PfSync &sy, uint8_t *smem, const PfGrid &g,
+                         int32_t *status) {
     using S = PfShape<D>;
     // The kernel is a programmatic dependent of the preceding one (normally the
     // append that rotated q and filled the cache): wait for it before loading.
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    const uint32_t qbytes = S::kTileBytes * (has1 ? 2 : 1);
-    ptx::mbar_arrive_expect_tx(A(sy.q_full), qbytes);
-    for (int t = 0; t < (has1 ? 2 : 1); ++t)
-        for (int kb = 0; kb < S::kBlocks; ++kb)
-            ptx::tma_load_4d(ptx::smem_addr(smem + S::kOffQ + t * S::kTileBytes + kb * S::kBlockBytes),
-                             &maps.q, A(sy.q_full), kb * 64, h, q0 + 128 * t, b);
-    int issued_k = 0, issued_v = 0;
+    int kc = 0, vc = 0, qc = 0;     // K, V tiles and Q pairs this CTA has loaded
     bool ok = true;
-    for (int j = 0; j < n_kv && ok; ++j) {
-        const int st = j % S::kStages;
-        const uint32_t par = ((j / S::kStages) & 1) ^ 1;
-        ok = ptx::mbar_wait(A(sy.k_empty[st]), par);
+    for (int w = blockIdx.x; w < g.n_items && ok; w += gridDim.x) {
+        const PfItem I = pf_item(w, g.n_pairs, g.B, g.T, g.Hq, g.Hkv);
+        // The previous item's last S MMA has released the Q tiles.
+        ok = ptx::mbar_wait(A(sy.q_empty), (qc & 1) ^ 1);
         if (!ok) break;
-        ptx::mbar_arrive_expect_tx(A(sy.k_full[st]), S::kTileBytes);
-        for (int kb = 0; kb < S::kBlocks; ++kb)
-            ptx::tma_load_3d(ptx::smem_addr(smem + S::kOffK + st * S::kTileBytes + kb * S::kBlockBytes),
-                             &maps.k, A(sy.k_full[st]), kb * 64, j * 128, b * Hkv + kvh);
-        issued_k = j + 1;
-        ok = ptx::mbar_wait(A(sy.v_empty[st]), par);
-        if (!ok) break;
-        ptx::mbar_arrive_expect_tx(A(sy.v_full[st]), S::kTileBytes);
-        for (int kb = 0; kb < S::kBlocks; ++kb)
-            ptx::tma_load_3d(ptx::smem_addr(smem + S::kOffV + st * S::kTileBytes + kb * S::kBlockBytes),
-                             &maps.v, A(sy.v_full[st]), kb * 64, j * 128, b * Hkv + kvh);
-        issued_v = j + 1;
+        ptx::mbar_arrive_expect_tx(A(sy.q_full), S::kTileBytes * (I.has1 ? 2 : 1));
+        for (int t = 0; t < (I.has1 ? 2 : 1); ++t)
+            for (int kb = 0; kb < S::kBlocks; ++kb)
+                ptx::tma_load_4d(ptx::smem_addr(smem + S::kOffQ + t * S::kTileBytes + kb * S::kBlockBytes),
+                                 &maps.q, A(sy.q_full), kb * 64, I.h, I.q0 + 128 * t, I.b);
+        ++qc;
+        // K tiles run ahead of V tiles: S(j) needs K(j) one MMA pair before
+        // PV(j) needs V(j), and the K ring is the deeper one.
+        int jk = 0, jv = 0;
+        while (ok && jv < I.n_kv) {
+            if (jk < I.n_kv && jk < jv + S::kStagesK) {
+                const int st = kc % S::kStagesK;
+                ok = ptx::mbar_wait(A(sy.k_empty[st]), ((kc / S::kStagesK) & 1) ^ 1);
+                if (!ok) break;
+                ptx::mbar_arrive_expect_tx(A(sy.k_full[st]), S::kTileBytes);
+                for (int kb = 0; kb < S::kBlocks; ++kb)
+                    ptx::tma_load_3d(ptx::smem_addr(smem + S::kOffK + st * S::kTileBytes + kb * S::kBlockBytes),
+                                     &maps.k, A(sy.k_full[st]), kb * 64, jk * 128, I.b * g.Hkv + I.kvh);
+                ++kc;
+                ++jk;
+            }
+            if (jv < jk) {
+                const int st = vc % S::kStagesV;
+                ok = ptx::mbar_wait(A(sy.v_empty[st]), ((vc / S::kStagesV) & 1) ^ 1);
+                if (!ok) break;
+                ptx::mbar_arrive_expect_tx(A(sy.v_full[st]), S::kTileBytes);
+                for (int kb = 0; kb < S::kBlocks; ++kb)
+                    ptx::tma_load_3d(ptx::smem_addr(smem + S::kOffV + st * S::kTileBytes + kb * S::kBlockBytes),
+                                     &maps.v, A(sy.v_full[st]), kb * 64, jv * 128, I.b * g.Hkv + I.kvh);
+                ++vc;
+                ++jv;
+            }
+        }
     }
     if (!ok) {
         report(status, GQA_DEV_TIMEOUT);
         // Let every copy already issued land before the CTA can retire.
-        ptx::mbar_wait(A(sy.q_full), 0);
-        for (int j = (issued_k > S::kStages ? issued_k - S::kStages : 0); j < issued_k; ++j)
-            ptx::mbar_wait(A(sy.k_full[j % S::kStages]), (j / S::kStages) & 1);
-        for (int j = (issued_v > S::kStages ? issued_v - S::kStages : 0); j < issued_v; ++j)
-            ptx::mbar_wait(A(sy.v_full[j % S::kStages]), (j / S::kStages) & 1);
+        if (qc > 0) ptx::mbar_wait(A(sy.q_full), (qc - 1) & 1);
+        for (int j = (kc > S::kStagesK ? kc - S::kStagesK : 0); j < kc; ++j)
+            ptx::mbar_wait(A(sy.k_full[j % S::kStagesK]), (j / S::kStagesK) & 1);
+        for (int j = (vc > S::kStagesV ? vc - S::kStagesV : 0); j < vc; ++j)
+            ptx::mbar_wait(A(sy.v_full[j % S::kStagesV]), (j / S::kStagesV) & 1);
     }
 }
 
 template <int D>
-__device__ void mma_issuer(PfSync &sy, uint8_t *smem, uint32_t tmem, bool has1, int n0, int n1,
-                           int n_kv, int32_t *status) {
+__device__ void mma_issuer(PfSync &sy, uint8_t *smem, uint32_t tmem, const PfGrid &g,
+                           int32_t *status) {
     using S = PfShape<D>;
     constexpr uint32_t idS = ptx::idesc_bf16_f32(128, 128, false);
     constexpr uint32_t idO = ptx::idesc_bf16_f32(128, D, true);
@@ -131,9 +178,9 @@ __device__ void mma_issuer(PfSync &sy, uint8_t *smem, uint32_t tmem, bool has1, 
     const uint32_t k_base = ptx::smem_addr(smem + S::kOffK);
     const uint32_t v_base = ptx::smem_addr(smem + S::kOffV);
 
-    auto issue_s = [&](int t, int j) {
+    auto issue_s = [&](int t, int kst) {
         const uint32_t qa = q_base + t * S::kTileBytes;
-        const uint32_t ka = k_base + (j % S::kStages) * S::kTileBytes;
+        const uint32_t ka = k_base + kst * S::kTileBytes;
 #pragma unroll
         for (int ks = 0; ks < S::kKSteps; ++ks) {
             const uint32_t off = (ks >> 2) * S::kBlockBytes + (ks & 3) * 32;
@@ -142,61 +189,78 @@ __device__ void mma_issuer(PfSync &sy, uint8_t *smem, uint32_t tmem, bool has1, 
         }
         ptx::mma_commit(A(sy.s_full[t]));
     };
-    auto issue_pv = [&](int t, int j) {
-        const uint32_t va = v_base + (j % S::kStages) * S::kTileBytes;
+    auto issue_pv = [&](int t, int vst, bool acc) {
+        const uint32_t va = v_base + vst * S::kTileBytes;
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
             ptx::mma_ts(tmem + 256 + t * 128, tmem + t * 128 + ks * 8,
                         ptx::smem_desc_sw128(va + ks * 2048, S::kBlockBytes, 1024), idO,
-                        (j > 0 || ks > 0) ? 1u : 0u);
+                        (acc || ks > 0) ? 1u : 0u);
     };
 
-    bool ok = ptx::mbar_wait(A(sy.q_full), 0) && ptx::mbar_wait(A(sy.k_full[0]), 0);
-    if (ok) {
-        ptx::tc_fence_after();
-        issue_s(0, 0);
-        if (has1) issue_s(1, 0);
-        ptx::mma_commit(A(sy.k_empty[0]));
-    }
-    for (int j = 0; j < n_kv && ok; ++j) {
-        const int st = j % S::kStages;
-        ok = ptx::mbar_wait(A(sy.v_full[st]), (j / S::kStages) & 1);
+    int kc = 0, vc = 0, qc = 0;     // K, V tiles and Q pairs consumed
+    int pc0 = 0, pc1 = 0;           // P hand-overs received from each softmax group
+    bool ok = true;
+    for (int w = blockIdx.x; w < g.n_items && ok; w += gridDim.x) {
+        const PfItem I = pf_item(w, g.n_pairs, g.B, g.T, g.Hq, g.Hkv);
+        const int kc0 = kc;
+        ok = ptx::mbar_wait(A(sy.q_full), qc & 1) &&
+             ptx::mbar_wait(A(sy.k_full[kc0 % S::kStagesK]), (kc0 / S::kStagesK) & 1);
         if (!ok) break;
-        const int jn = j + 1;
-        const int stn = jn % S::kStages;
-        bool k_next = false;
-        if (j < n0) {
-            ok = ptx::mbar_wait(A(sy.p_full[0]), j & 1);
+        ++qc;
+        ptx::tc_fence_after();
+        issue_s(0, kc0 % S::kStagesK);
+        if (I.has1) issue_s(1, kc0 % S::kStagesK);
+        ptx::mma_commit(A(sy.k_empty[kc0 % S::kStagesK]));
+        if (I.n_kv == 1) ptx::mma_commit(A(sy.q_empty));   // Q no longer read
+        for (int j = 0; j < I.n_kv && ok; ++j) {
+            const int vst = vc % S::kStagesV;
+            ok = ptx::mbar_wait(A(sy.v_full[vst]), (vc / S::kStagesV) & 1);
             if (!ok) break;
-            ptx::tc_fence_after();
-            issue_pv(0, j);
-            if (jn < n0) {
-                ok = ptx::mbar_wait(A(sy.k_full[stn]), (jn / S::kStages) & 1);
+            const int jn = j + 1;
+            const int kidx = kc0 + jn;
+            const int kst = kidx % S::kStagesK;
+            bool k_next = false;
+            if (j < I.n0) {
+                ok = ptx::mbar_wait(A(sy.p_full[0]), pc0 & 1);
                 if (!ok) break;
-                k_next = true;
-                issue_s(0, jn);
-            } else {
-                ptx::mma_commit(A(sy.o_final[0]));
-            }
-        }
-        if (has1 && j < n1) {
-            ok = ptx::mbar_wait(A(sy.p_full[1]), j & 1);
-            if (!ok) break;
-            ptx::tc_fence_after();
-            issue_pv(1, j);
-            if (jn < n1) {
-                if (!k_next) {
-                    ok = ptx::mbar_wait(A(sy.k_full[stn]), (jn / S::kStages) & 1);
+                ++pc0;
+                ptx::tc_fence_after();
+                issue_pv(0, vst, j > 0);
+                if (jn < I.n0) {
+                    ok = ptx::mbar_wait(A(sy.k_full[kst]), (kidx / S::kStagesK) & 1);
                     if (!ok) break;
                     k_next = true;
+                    issue_s(0, kst);
+                } else {
+                    ptx::mma_commit(A(sy.o_final[0]));
                 }
-                issue_s(1, jn);
-            } else {
-                ptx::mma_commit(A(sy.o_final[1]));
+            }
+            if (I.has1 && j < I.n1) {
+                ok = ptx::mbar_wait(A(sy.p_full[1]), pc1 & 1);
+                if (!ok) break;
+                ++pc1;
+                ptx::tc_fence_after();
+                issue_pv(1, vst, j > 0);
+                if (jn < I.n1) {
+                    if (!k_next) {
+                        ok = ptx::mbar_wait(A(sy.k_full[kst]), (kidx / S::kStagesK) & 1);
+                        if (!ok) break;
+                        k_next = true;
+                    }
+                    issue_s(1, kst);
+                } else {
+                    ptx::mma_commit(A(sy.o_final[1]));
+                }
+            }
+            ptx::mma_commit(A(sy.v_empty[vst]));
+            ++vc;
+            if (k_next) {
+                ptx::mma_commit(A(sy.k_empty[kst]));
+                if (jn == I.n_kv - 1) ptx::mma_commit(A(sy.q_empty));   // last S of the item
             }
         }
-        ptx::mma_commit(A(sy.v_empty[st]));
-        if (k_next) ptx::mma_commit(A(sy.k_empty[stn]));
+        kc = kc0 + I.n_kv;
     }
     if (!ok) report(status, GQA_DEV_TIMEOUT);
     // No MMA may still be writing tensor memory when it is released.
@@ -205,117 +269,126 @@ __device__ void mma_issuer(PfSync &sy, uint8_t *smem, uint32_t tmem, bool has1, 
 }
 
 template <int D>
-__device__ void softmax_tile(PfSync &sy, uint32_t tmem, int t, int q_first, int nt, int T,
-                             float scale_log2, uint16_t *out_row_base, size_t row_stride,
-                             int32_t *status) {
+__device__ void softmax_tile(PfSync &sy, uint32_t tmem, int t, const PfGrid &g, float scale_log2,
+                             uint16_t *__restrict__ out, int32_t *status) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int row = (warp & 3) * 32 + lane;
-    const int qrow = q_first + row;
     const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const uint32_t s_col = t * 128, o_col = 256 + t * 128;
-    const int diag = q_first / 128;
-
-    float m = -INFINITY, l = 0.f;
+    const int T = g.T;
+    int sc = 0, oc = 0;             // scores and outputs of this tile received
     bool ok = true;
-    for (int j = 0; j < nt; ++j) {
-        ok = __all_sync(0xffffffffu, ptx::mbar_wait(A(sy.s_full[t]), j & 1));
-        if (!ok) break;
-        ptx::tc_fence_after();
-        uint32_t sv[4][32];
+    for (int w = blockIdx.x; w < g.n_items && ok; w += gridDim.x) {
+        const PfItem I = pf_item(w, g.n_pairs, g.B, g.T, g.Hq, g.Hkv);
+        if (t == 1 && !I.has1) continue;
+        const int q_first = I.q0 + 128 * t;
+        const int nt = t == 0 ? I.n0 : I.n1;
+        const int qrow = q_first + row;
+        const int diag = q_first / 128;
+        float m = -INFINITY, l = 0.f;
+        for (int j = 0; j < nt; ++j) {
+            ok = __all_sync(0xffffffffu, ptx::mbar_wait(A(sy.s_full[t]), sc & 1));
+            if (!ok) break;
+            ++sc;
+            ptx::tc_fence_after();
+            uint32_t sv[4][32];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) ptx::tmem_ld32(lane_addr + s_col + 32 * c, sv[c]);
-        ptx::tmem_wait_ld();
+            for (int c = 0; c < 4; ++c) ptx::tmem_ld32(lane_addr + s_col + 32 * c, sv[c]);
+            ptx::tmem_wait_ld();
 #define SV(c) __uint_as_float(sv[(c) >> 5][(c) & 31])
-
-        const int key0 = j * 128;
-        if (j == diag || key0 + 128 > T) {
+            const int key0 = j * 128;
+            if (j == diag || key0 + 128 > T) {
 #pragma unroll
-            for (int c = 0; c < 128; ++c) {
-                const int key = key0 + c;
-                if (key > qrow || key >= T) sv[c >> 5][c & 31] = __float_as_uint(-INFINITY);
+                for (int c = 0; c < 128; ++c) {
+                    const int key = key0 + c;
+                    if (key > qrow || key >= T) sv[c >> 5][c & 31] = __float_as_uint(-INFINITY);
+                }
             }
-        }
-        // Row maximum: four independent chains of three-input max.
-        float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+            // Row maximum: four independent chains of three-input max.
+            float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < 128; c += 8) {
-            mx0 = ptx::fmax3(mx0, SV(c), SV(c + 1));
-            mx1 = ptx::fmax3(mx1, SV(c + 2), SV(c + 3));
-            mx2 = ptx::fmax3(mx2, SV(c + 4), SV(c + 5));
-            mx3 = ptx::fmax3(mx3, SV(c + 6), SV(c + 7));
-        }
-        const float smax = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
-        const float m_new = fmaxf(m, smax * scale_log2);
-        const bool resc = m_new > m + kRescaleThreshold;
-        const float alpha = resc ? ex2(m - m_new) : 1.f;
-        if (resc) {
-            l *= alpha;
-            m = m_new;
-        }
-        if (j > 0 && __any_sync(0xffffffffu, resc)) {
-#pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-                uint32_t o[32];
-                ptx::tmem_ld32(lane_addr + o_col + 32 * c, o);
-                ptx::tmem_wait_ld();
-#pragma unroll
-                for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-                ptx::tmem_st32(lane_addr + o_col + 32 * c, o);
+            for (int c = 0; c < 128; c += 8) {
+                mx0 = ptx::fmax3(mx0, SV(c), SV(c + 1));
+                mx1 = ptx::fmax3(mx1, SV(c + 2), SV(c + 3));
+                mx2 = ptx::fmax3(mx2, SV(c + 4), SV(c + 5));
+                mx3 = ptx::fmax3(mx3, SV(c + 6), SV(c + 7));
             }
-        }
-        // p = 2^(s * scale_log2 - m): packed FMA for the exponent argument, the
-        // special-function unit for 2^x, four independent partial row sums.
-        const float neg_m = -m;
-        float la0 = 0.f, la1 = 0.f, lb0 = 0.f, lb1 = 0.f;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            uint32_t p[16];
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-                float x0, x1;
-                ptx::ffma2(x0, x1, SV(32 * c + 2 * e), SV(32 * c + 2 * e + 1), scale_log2,
-                           scale_log2, neg_m, neg_m);
-                const float p0 = ex2(x0), p1 = ex2(x1);
-                p[e] = pack_bf16x2(p0, p1);
-                if (e & 1)
-                    ptx::fadd2(la0, la1, la0, la1, p0, p1);
-                else
-                    ptx::fadd2(lb0, lb1, lb0, lb1, p0, p1);
+            const float smax = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+            const float m_new = fmaxf(m, smax * scale_log2);
+            const bool resc = m_new > m + kRescaleThreshold;
+            const float alpha = resc ? ex2(m - m_new) : 1.f;
+            if (resc) {
+                l *= alpha;
+                m = m_new;
             }
-            ptx::tmem_st16(lane_addr + s_col + 16 * c, p);
-        }
+            if (j > 0 && __any_sync(0xffffffffu, resc)) {
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t o[32];
+                    ptx::tmem_ld32(lane_addr + o_col + 32 * c, o);
+                    ptx::tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                    ptx::tmem_st32(lane_addr + o_col + 32 * c, o);
+                }
+            }
+            // p = 2^(s * scale_log2 - m): packed FMA for the exponent argument, the
+            // special-function unit for 2^x, four independent partial row sums.
+            const float neg_m = -m;
+            float la0 = 0.f, la1 = 0.f, lb0 = 0.f, lb1 = 0.f;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint32_t p[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    float x0, x1;
+                    ptx::ffma2(x0, x1, SV(32 * c + 2 * e), SV(32 * c + 2 * e + 1), scale_log2,
+                               scale_log2, neg_m, neg_m);
+                    const float p0 = ex2(x0), p1 = ex2(x1);
+                    p[e] = pack_bf16x2(p0, p1);
+                    if (e & 1)
+                        ptx::fadd2(la0, la1, la0, la1, p0, p1);
+                    else
+                        ptx::fadd2(lb0, lb1, lb0, lb1, p0, p1);
+                }
+                ptx::tmem_st16(lane_addr + s_col + 16 * c, p);
+            }
 #undef SV
-        l += (la0 + la1) + (lb0 + lb1);
-        ptx::tmem_wait_st();
-        ptx::tc_fence_before();
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(A(sy.p_full[t]));
-    }
-    if (ok) ok = __all_sync(0xffffffffu, ptx::mbar_wait(A(sy.o_final[t]), 0));
-    if (!ok) {
-        if (lane == 0) report(status, GQA_DEV_TIMEOUT);
-        return;
-    }
-    ptx::tc_fence_after();
-    const float inv_l = 1.f / l;
-    uint16_t *dst = out_row_base + (size_t)qrow * row_stride;
-#pragma unroll
-    for (int c = 0; c < D / 32; ++c) {
-        uint32_t o[32];
-        ptx::tmem_ld32(lane_addr + o_col + 32 * c, o);
-        ptx::tmem_wait_ld();
-        uint32_t w[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e)
-            w[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
-        if (qrow < T) {
-            uint4 *d4 = reinterpret_cast<uint4 *>(dst + 32 * c);
-            d4[0] = make_uint4(w[0], w[1], w[2], w[3]);
-            d4[1] = make_uint4(w[4], w[5], w[6], w[7]);
-            d4[2] = make_uint4(w[8], w[9], w[10], w[11]);
-            d4[3] = make_uint4(w[12], w[13], w[14], w[15]);
+            l += (la0 + la1) + (lb0 + lb1);
+            ptx::tmem_wait_st();
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(A(sy.p_full[t]));
         }
+        if (ok) ok = __all_sync(0xffffffffu, ptx::mbar_wait(A(sy.o_final[t]), oc & 1));
+        if (!ok) break;
+        ++oc;
+        ptx::tc_fence_after();
+        const float inv_l = 1.f / l;
+        uint16_t *dst = out + (((size_t)I.b * T + qrow) * g.Hq + I.h) * D;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            ptx::tmem_ld32(lane_addr + o_col + 32 * c, o);
+            ptx::tmem_wait_ld();
+            uint32_t w4[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+                w4[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l,
+                                    __uint_as_float(o[2 * e + 1]) * inv_l);
+            if (qrow < T) {
+                uint4 *d4 = reinterpret_cast<uint4 *>(dst + 32 * c);
+                d4[0] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                d4[1] = make_uint4(w4[4], w4[5], w4[6], w4[7]);
+                d4[2] = make_uint4(w4[8], w4[9], w4[10], w4[11]);
+                d4[3] = make_uint4(w4[12], w4[13], w4[14], w4[15]);
+            }
+        }
+        // the next item's first P hand-over (after this read of O) lets the
+        // MMA overwrite O with that item's first product
+        ptx::tc_fence_before();
     }
+    if (!ok && lane == 0) report(status, GQA_DEV_TIMEOUT);
 }
 
 template <int D>
@@ -327,25 +400,23 @@ prefill_kernel(const __grid_constant__ PfMaps maps, uint16_t *__restrict__ out, 
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     __shared__ PfSync sy;
-
-    // Longest query pairs first; the heads of one KV group run side by side.
-    const int per_pair = Hq * B;
-    const int pair = n_pairs - 1 - (int)(blockIdx.x / per_pair);
-    const int rest = (int)(blockIdx.x % per_pair);
-    const int h = rest % Hq, b = rest / Hq;
-    const int kvh = h / (Hq / Hkv);
-    const int q0 = pair * 256;
-    const bool has1 = q0 + 128 < T;
-    const int n0 = (min(T, q0 + 128) + 127) / 128;
-    const int n1 = has1 ? (min(T, q0 + 256) + 127) / 128 : 0;
-    const int n_kv = has1 ? n1 : n0;
+    PfGrid g;
+    g.n_pairs = n_pairs;
+    g.B = B;
+    g.T = T;
+    g.Hq = Hq;
+    g.Hkv = Hkv;
+    g.n_items = n_pairs * Hq * B;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         ptx::mbar_init(A(sy.q_full), 1);
-        for (int i = 0; i < S::kStages; ++i) {
+        ptx::mbar_init(A(sy.q_empty), 1);
+        for (int i = 0; i < S::kStagesK; ++i) {
             ptx::mbar_init(A(sy.k_full[i]), 1);
             ptx::mbar_init(A(sy.k_empty[i]), 1);
+        }
+        for (int i = 0; i < S::kStagesV; ++i) {
             ptx::mbar_init(A(sy.v_full[i]), 1);
             ptx::mbar_init(A(sy.v_empty[i]), 1);
         }
@@ -374,20 +445,15 @@ prefill_kernel(const __grid_constant__ PfMaps maps, uint16_t *__restrict__ out, 
     if (warp >= 8) {
         ptx::regs_dec<kControlRegs>();
         if (warp == kTmaWarp) {
-            if (lane == 0) producer<D>(maps, sy, smem, b, h, kvh, Hkv, q0, has1, n_kv, status);
+            if (lane == 0) producer<D>(maps, sy, smem, g, status);
             __syncwarp();
         } else if (warp == kMmaWarp) {
-            if (lane == 0) mma_issuer<D>(sy, smem, tmem, has1, n0, n1, n_kv, status);
+            if (lane == 0) mma_issuer<D>(sy, smem, tmem, g, status);
             __syncwarp();
         }
     } else {
         ptx::regs_inc<kSoftmaxRegs>();
-        const int t = warp >> 2;
-        if (t == 0 || has1) {
-            uint16_t *base = out + ((size_t)b * T * Hq + h) * D;
-            softmax_tile<D>(sy, tmem, t, q0 + 128 * t, t == 0 ? n0 : n1, T, scale_log2, base,
-                            (size_t)Hq * D, status);
-        }
+        softmax_tile<D>(sy, tmem, warp >> 2, g, scale_log2, out, status);
     }
     ptx::tc_fence_before();
     __syncthreads();
@@ -461,7 +527,12 @@ gqa_status launch_prefill(const void *q, const void *kc, const void *vc, void *o
     if (cudaFuncGetAttributes(&attr, kern) != cudaSuccess) return GQA_ERR_CUDA;
     if (attr.numRegs != kLaunchRegs) return GQA_ERR_UNSUPPORTED;
     const int n_pairs = (T + 255) / 256;
-    const long long grid = (long long)n_pairs * Hq * B;
+    const long long items = (long long)n_pairs * Hq * B;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return GQA_ERR_CUDA;
+    const long long grid = items < sms ? items : sms;   // persistent: one CTA per SM
     // Programmatic dependent launch: the prologue (barriers, tensor memory,
     // descriptor prefetch) overlaps the tail of the preceding kernel; the TMA
     // producer waits for that kernel before its first load.

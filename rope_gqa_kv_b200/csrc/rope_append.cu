@@ -5,10 +5,11 @@
 // QK-norm: page "训练3.8B LLM至0.384 CORE，成本998美元 – Hugo Vergnes", section "设置";
 // KV-cache append: first page, section "V3：扩容与推理优化".
 //
-// One CTA per token (b, t).  The CTA issues the loads of its first head vectors,
-// then turns the token's position into the D/2 rotation angles (float64 angle
-// p * base^(-2i/D) reduced to [-pi, pi] in float64, cos/sin in fp32) in shared
-// memory, shared by all of the token's heads.  Each head vector
+// One CTA per block of 4 consecutive tokens of a sequence (1 token in decode).
+// The CTA issues the loads of its first head vectors, then turns each token's
+// position into the D/2 rotation angles (float64 angle p * base^(-2i/D) reduced
+// to [-pi, pi] in float64, cos/sin in fp32) in shared memory, shared by all of
+// the token's heads.  Each head vector
 // is then owned by TPV threads: thread j holds the 16-byte chunk j of the first
 // half (coordinates 8j..8j+7) and the matching chunk of the second half
 // (coordinates D/2+8j..), i.e. exactly the 8 rotation pairs it needs, so every
@@ -89,8 +90,13 @@ __device__ __forceinline__ void rotate_vector(const uint4 a_in, const uint4 b_in
 
 // Vectors of one token, in order: Hq query heads (if q), Hkv key heads and Hkv
 // value heads (if k).  Query heads are rotated in place; key heads are rotated
-// into the cache; value heads are copied into the cache bit for bit.
-template <int D>
+// into the cache; value heads are copied into the cache bit for bit.  A CTA
+// takes TB consecutive tokens of one sequence: its global loads go out in
+// batches of kBatch passes (the first batch before the angles are computed),
+// so every lane has several 32-byte loads in flight.
+constexpr int kBatch = 4;
+
+template <int D, int TB>
 __global__ void __launch_bounds__(kThreads)
 rope_append_kernel(uint16_t *__restrict__ q, const uint16_t *__restrict__ k,
                    const uint16_t *__restrict__ v, uint16_t *__restrict__ kc,
@@ -98,18 +104,19 @@ rope_append_kernel(uint16_t *__restrict__ q, const uint16_t *__restrict__ k,
                    int32_t *__restrict__ new_len, int T, int Hq, int Hkv, int Lmax,
                    int qk_norm, float eps, float base, int32_t *status) {
     using S = RopeShape<D>;
-    __shared__ float cs[S::kHalf];
-    __shared__ float sn[S::kHalf];
+    __shared__ float cs[TB][S::kHalf];
+    __shared__ float sn[TB][S::kHalf];
+    __shared__ double theta_d[S::kHalf];
     // A kernel launched after this one as a programmatic dependent (the prefill
     // or the decode) may start its prologue now; it waits for this grid to
     // complete before it reads anything written here.
     asm volatile("griddepcontrol.launch_dependents;");
 
-    const int token = blockIdx.x;              // b * T + t
-    const int b = token / T;
-    const int t = token - b * T;
+    const int nblk = (T + TB - 1) / TB;
+    const int b = blockIdx.x / nblk;
+    const int t0 = (blockIdx.x - b * nblk) * TB;
+    const int nt = min(TB, T - t0);
     const int p0 = pos0 ? pos0[b] : 0;
-    const int p = p0 + t;
 
     bool write_cache = (k != nullptr);
     if (threadIdx.x == 0) {
@@ -118,124 +125,132 @@ rope_append_kernel(uint16_t *__restrict__ q, const uint16_t *__restrict__ k,
         } else if (write_cache && p0 + T > Lmax) {
             report(status, GQA_DEV_CAPACITY);
         }
-        if (new_len && t == 0) new_len[b] = p0 + T;
+        if (new_len && t0 == 0) new_len[b] = p0 + T;
     }
     if (p0 < 0) return;
     if (write_cache && p0 + T > Lmax) write_cache = false;
 
     const int nq = q ? Hq : 0;
     const int nk = write_cache ? Hkv : 0;
-    const int nvec = nq + 2 * nk;
+    const int per_tok = nq + 2 * nk;
+    const int nvec = nt * per_tok;
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
     const int j = lane % S::kTPV;
     const int slot = lane / S::kTPV;
     const bool active = j < S::kChunks;
     constexpr int kSlots = (kThreads / 32) * S::kVecPerWarp;
+    const int npass = (nvec + kSlots - 1) / kSlots;
 
-    const size_t tok_q = (size_t)token * Hq * D;
-    const size_t tok_kv = (size_t)token * Hkv * D;
-
-    // Where vector vi comes from and goes to; `rotate` is false for value heads.
-    auto locate = [&](int vi, const uint16_t *&src, uint16_t *&dst, bool &rotate) {
-        if (vi < nq) {
-            src = q + tok_q + (size_t)vi * D;
-            dst = q + tok_q + (size_t)vi * D;
+    // Where vector vi of the block comes from and goes to; `rotate` is false for
+    // value heads, `tl` is its token within the block.
+    auto locate = [&](int vi, const uint16_t *&src, uint16_t *&dst, bool &rotate, int &tl) {
+        tl = vi / per_tok;
+        const int r = vi - tl * per_tok;
+        const int t = t0 + tl;
+        const int p = p0 + t;
+        const size_t token = (size_t)b * T + t;
+        if (r < nq) {
+            src = q + (token * Hq + r) * D;
+            dst = q + (token * Hq + r) * D;
             rotate = true;
-        } else if (vi < nq + nk) {
-            const int h = vi - nq;
-            src = k + tok_kv + (size_t)h * D;
+        } else if (r < nq + nk) {
+            const int h = r - nq;
+            src = k + (token * Hkv + h) * D;
             dst = kc + (((size_t)b * Hkv + h) * Lmax + p) * D;
             rotate = true;
         } else {
-            const int h = min(vi - nq - nk, Hkv - 1);
-            src = v + tok_kv + (size_t)h * D;
+            const int h = r - nq - nk;
+            src = v + (token * Hkv + h) * D;
             dst = vc + (((size_t)b * Hkv + h) * Lmax + p) * D;
             rotate = false;
         }
     };
 
-    // The first kPre passes of loads are issued before the angles are computed,
-    // so their memory latency overlaps the trigonometry and the barrier.
-    constexpr int kPre = 2;
-    uint4 ra[kPre], rb[kPre];
+    for (int pb = 0; pb < npass; pb += kBatch) {
+        uint4 ra[kBatch], rb[kBatch];
 #pragma unroll
-    for (int u = 0; u < kPre; ++u) {
-        const int vi = u * kSlots + warp * S::kVecPerWarp + slot;
-        ra[u] = make_uint4(0, 0, 0, 0);
-        rb[u] = make_uint4(0, 0, 0, 0);
-        if (vi < nvec && active) {
+        for (int u = 0; u < kBatch; ++u) {
+            const int vi = (pb + u) * kSlots + warp * S::kVecPerWarp + slot;
+            ra[u] = make_uint4(0, 0, 0, 0);
+            rb[u] = make_uint4(0, 0, 0, 0);
+            if (vi < nvec && active) {
+                const uint16_t *src;
+                uint16_t *dst;
+                bool rot;
+                int tl;
+                locate(vi, src, dst, rot, tl);
+                ra[u] = *reinterpret_cast<const uint4 *>(src + 8 * j);
+                rb[u] = *reinterpret_cast<const uint4 *>(src + S::kHalf + 8 * j);
+            }
+        }
+        if (pb == 0) {
+            // Angle p * base^(-2i/D) in float64, reduced to [-pi, pi] in float64
+            // (subtracting the nearest multiple of 2*pi), then sin/cos in fp32.
+            for (int i = threadIdx.x; i < S::kHalf; i += kThreads)
+                theta_d[i] = pow((double)base, -2.0 * (double)i / (double)D);
+            __syncthreads();
+            for (int i = threadIdx.x; i < TB * S::kHalf; i += kThreads) {
+                const int tl = i / S::kHalf, pi = i - tl * S::kHalf;
+                const double a = (double)(p0 + t0 + tl) * theta_d[pi];
+                const double two_pi = 6.283185307179586476925286766559;
+                const double r = a - rint(a * (1.0 / two_pi)) * two_pi;
+                float sf, cf;
+                sincosf((float)r, &sf, &cf);
+                cs[tl][pi] = cf;
+                sn[tl][pi] = sf;
+            }
+            __syncthreads();
+        }
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            if (pb + u >= npass) break;                    // uniform across the CTA
+            const int vi = (pb + u) * kSlots + warp * S::kVecPerWarp + slot;
+            const bool live = vi < nvec;
             const uint16_t *src;
             uint16_t *dst;
-            bool rot;
-            locate(vi, src, dst, rot);
-            ra[u] = *reinterpret_cast<const uint4 *>(src + 8 * j);
-            rb[u] = *reinterpret_cast<const uint4 *>(src + S::kHalf + 8 * j);
-        }
-    }
-
-    // Angle p * base^(-2i/D) in float64, reduced to [-pi, pi] in float64
-    // (subtracting the nearest multiple of 2*pi), then sin/cos in fp32.
-    for (int i = threadIdx.x; i < S::kHalf; i += kThreads) {
-        const double theta = pow((double)base, -2.0 * (double)i / (double)D);
-        const double a = (double)p * theta;
-        const double two_pi = 6.283185307179586476925286766559;
-        const double r = a - rint(a * (1.0 / two_pi)) * two_pi;
-        float sf, cf;
-        sincosf((float)r, &sf, &cf);
-        cs[i] = cf;
-        sn[i] = sf;
-    }
-    __syncthreads();
-
-    // Every lane of a group runs the loop the same number of times (the shuffle
-    // in the norm needs the whole warp); inactive lanes just skip memory.
-    for (int pass = 0; pass * kSlots < nvec; ++pass) {
-        const int vi = pass * kSlots + warp * S::kVecPerWarp + slot;
-        const bool live = vi < nvec;
-        const uint16_t *src;
-        uint16_t *dst;
-        bool rotate;
-        locate(live ? vi : 0, src, dst, rotate);
-        const bool mem = live && active;
-        uint4 a = make_uint4(0, 0, 0, 0), bb = make_uint4(0, 0, 0, 0);
-        if (pass < kPre) {
-#pragma unroll
-            for (int u = 0; u < kPre; ++u)
-                if (u == pass) {
-                    a = ra[u];
-                    bb = rb[u];
-                }
-        } else if (mem) {
-            a = *reinterpret_cast<const uint4 *>(src + 8 * j);
-            bb = *reinterpret_cast<const uint4 *>(src + S::kHalf + 8 * j);
-        }
-        // Every lane computes the rotation (the norm's shuffle spans the whole
-        // warp); value vectors keep their loaded bits.
-        uint4 oa, ob;
-        rotate_vector<D>(a, bb, oa, ob, cs, sn, j, mem, qk_norm != 0, eps);
-        if (rotate) {
-            a = oa;
-            bb = ob;
-        }
-        if (mem) {
-            *reinterpret_cast<uint4 *>(dst + 8 * j) = a;
-            *reinterpret_cast<uint4 *>(dst + S::kHalf + 8 * j) = bb;
+            bool rotate;
+            int tl;
+            locate(live ? vi : 0, src, dst, rotate, tl);
+            const bool mem = live && active;
+            // Every lane computes the rotation (the norm's shuffle spans the
+            // whole warp); value vectors keep their loaded bits.
+            uint4 a = ra[u], bb = rb[u], oa, ob;
+            rotate_vector<D>(a, bb, oa, ob, cs[tl], sn[tl], j, mem, qk_norm != 0, eps);
+            if (rotate) {
+                a = oa;
+                bb = ob;
+            }
+            if (mem) {
+                *reinterpret_cast<uint4 *>(dst + 8 * j) = a;
+                *reinterpret_cast<uint4 *>(dst + S::kHalf + 8 * j) = bb;
+            }
         }
     }
 }
 
-template <int D>
+template <int D, int TB>
 cudaError_t launch(void *q, const void *k, const void *v, void *kc, void *vc,
                    const int32_t *pos0, int32_t *new_len, int B, int T, int Hq, int Hkv,
                    int Lmax, const gqa_rope_params &p, int32_t *status, cudaStream_t s) {
-    const unsigned grid = (unsigned)B * (unsigned)T;
-    rope_append_kernel<D><<<grid, kThreads, 0, s>>>(
+    const unsigned grid = (unsigned)B * (unsigned)((T + TB - 1) / TB);
+    rope_append_kernel<D, TB><<<grid, kThreads, 0, s>>>(
         static_cast<uint16_t *>(q), static_cast<const uint16_t *>(k),
         static_cast<const uint16_t *>(v), static_cast<uint16_t *>(kc),
         static_cast<uint16_t *>(vc), pos0, new_len, T, Hq, Hkv, Lmax, p.qk_norm, p.eps,
         p.rope_base, status);
     return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_tb(void *q, const void *k, const void *v, void *kc, void *vc,
+                      const int32_t *pos0, int32_t *new_len, int B, int T, int Hq, int Hkv,
+                      int Lmax, const gqa_rope_params &p, int32_t *status, cudaStream_t s) {
+    // Blocks of 4 tokens once a sequence has that many; one token otherwise
+    // (decode), so that the grid still covers the batch.
+    if (T >= 4)
+        return launch<D, 4>(q, k, v, kc, vc, pos0, new_len, B, T, Hq, Hkv, Lmax, p, status, s);
+    return launch<D, 1>(q, k, v, kc, vc, pos0, new_len, B, T, Hq, Hkv, Lmax, p, status, s);
 }
 
 gqa_status dispatch(void *q, const void *k, const void *v, void *kc, void *vc,
@@ -245,9 +260,9 @@ gqa_status dispatch(void *q, const void *k, const void *v, void *kc, void *vc,
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e;
     switch (D) {
-        case 64: e = launch<64>(q, k, v, kc, vc, pos0, new_len, B, T, Hq, Hkv, Lmax, p, status, s); break;
-        case 96: e = launch<96>(q, k, v, kc, vc, pos0, new_len, B, T, Hq, Hkv, Lmax, p, status, s); break;
-        case 128: e = launch<128>(q, k, v, kc, vc, pos0, new_len, B, T, Hq, Hkv, Lmax, p, status, s); break;
+        case 64: e = launch_tb<64>(q, k, v, kc, vc, pos0, new_len, B, T, Hq, Hkv, Lmax, p, status, s); break;
+        case 96: e = launch_tb<96>(q, k, v, kc, vc, pos0, new_len, B, T, Hq, Hkv, Lmax, p, status, s); break;
+        case 128: e = launch_tb<128>(q, k, v, kc, vc, pos0, new_len, B, T, Hq, Hkv, Lmax, p, status, s); break;
         default: return GQA_ERR_UNSUPPORTED;
     }
     return e == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
