@@ -41,6 +41,8 @@ PREFILL = inputs.BY_NAME["prefill_3p8b"]
 DECODE = inputs.BY_NAME["batched_decode"]
 WORKLOAD = ("3.8B-style attention layer: prefill B=8 T=2048 Hq=24 Hkv=8 D=128 QK-norm, "
             "then one decode step B=64 Hq=24 Hkv=8 D=128 with cached lengths U[256,2048]")
+# kernels of libgqa launched per step: rope/append + prefill, rope/append + decode split + merge
+LAUNCHES_PER_STEP = 5
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -362,7 +364,7 @@ def run_ours(args, rank, world, dev, dist_on):
         "e2e": {"value": round(tok / (ms_e2e / K * 1e-3), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": round(ms_e2e / K, 4)},
-        "gpu_launches": 4 * K,
+        "gpu_launches": LAUNCHES_PER_STEP * K,
         "clocks": clocks,
         "device_status": status,
     }
