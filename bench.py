@@ -54,6 +54,14 @@ def prefill_flops(w=PREFILL) -> float:
     return 4.0 * w.D * (w.T * (w.T + 1) / 2) * w.B * w.Hq
 
 
+def chunk_flops(pos0, w) -> float:
+    """Causal FLOPs of a continuation chunk: 4*D per (query, visible key, query
+    head), query t of sequence b seeing pos0[b] + t + 1 keys."""
+    T = w.T
+    per_b = [T * int(p) + T * (T + 1) / 2.0 for p in pos0]
+    return 4.0 * w.D * w.Hq * sum(per_b)
+
+
 def decode_bytes(lens_new, w=DECODE) -> float:
     """K and V of every visible slot, once per KV head, plus q in and o out."""
     kv = float(np.sum(lens_new)) * w.Hkv * w.D * 2 * 2
@@ -368,9 +376,48 @@ def run_ours(args, rank, world, dev, dist_on):
         "clocks": clocks,
         "device_status": status,
     }
+    line["next_rows"] = {"chunked_prefill": measure_chunk(dev, peaks, tag)}
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
     return line
+
+
+def measure_chunk(dev, peaks, tag, reps: int = 30):
+    """Continuation chunk (gqa_prefill_chunk), outside the timed step: 8 sequences
+    with cached prefixes U[512, 1536] and 1024 new tokens each, 24/8 heads,
+    D = 128.  Each launch is timed alone with CUDA events after a 256 MB write
+    that evicts the L2."""
+    import rope_gqa_kv_b200 as gqa
+    w = inputs.BY_NAME["chunked_prefill_3p8b"]
+    x = inputs.make_inputs(w)
+    d = lambda t: t.to(dev)  # noqa: E731
+    q, k, v, kc, vc = d(x["q"]), d(x["k"]), d(x["v"]), d(x["k_cache"]), d(x["v_cache"])
+    pos0 = d(x["lens"])
+    max_pos0 = int(x["lens"].max())
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    gqa.gqa_rope_append(q, k, v, kc, vc, pos0=pos0, max_pos0=max_pos0, qk_norm=True,
+                        status=status)
+    out = torch.empty_like(q)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for _ in range(3):
+        gqa.gqa_prefill_chunk(q, kc, vc, pos0, max_pos0, out=out, status=status)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(reps)]
+    for i in range(reps):
+        flush.fill_(i & 255)
+        ev[i][0].record()
+        gqa.gqa_prefill_chunk(q, kc, vc, pos0, max_pos0, out=out, status=status)
+        ev[i][1].record()
+    torch.cuda.synchronize()
+    ms = sorted(a.elapsed_time(b) for a, b in ev)[reps // 2]
+    fl = chunk_flops(x["lens"].tolist(), w)
+    tf = fl / (ms * 1e-3) / 1e12
+    return {"workload": "8 x (prefix U[512,1536] + 1024 new tokens), 24q/8kv, D=128, QK-norm",
+            "kernel": "gqa_prefill_chunk", "bound": "tensor", "us_median": round(ms * 1e3, 2),
+            "achieved": round(tf, 1), "unit": "TFLOP/s", "peak": peaks["bf16_tflops"],
+            "frac": round(tf / peaks["bf16_tflops"], 4), "peak_kind": "bf16 burst " + tag,
+            "algorithmic_per_launch": fl, "l2": "flushed (256 MB write) before each launch",
+            "device_status": int(status.item())}
 
 
 # ---------------------------------------------------------------------------

@@ -125,6 +125,33 @@ gqa_status gqa_prefill(const void *q, const void *k_cache, const void *v_cache, 
                        int32_t *status_dev, void *stream);
 
 /*
+ * gqa_prefill_chunk -- causal attention of T new tokens per sequence that
+ * continue a cached prefix (chunked prefill, multi-turn continuation, a batch of
+ * prompts of different cached lengths): query t of sequence b sits at position
+ * p = pos0[b] + t and attends to every cache slot s <= p,
+ *     out[b, t, h, :] = sum_{s <= pos0[b]+t} softmax_s(q[b,t,h,:] . K[b, h/g, s, :] * scale)
+ *                                            * V[b, h/g, s, :]
+ * the KV-cache step of page "750美元从零训练3个LLM" (section "V3：扩容与推理优化")
+ * taken T tokens at a time.  q must be rotated at those positions and the
+ * caches must hold the prefix (slots < pos0[b]) and the chunk's own rotated K
+ * and raw V (slots pos0[b] .. pos0[b] + n_tok[b] - 1): gqa_rope_append with the
+ * same pos0 does both.  Cache slots from pos0[b] + n_tok[b] on are never used and
+ * may hold anything (NaN included).  Same kernel as gqa_prefill.
+ *   pos0: device int32 [B] (required); n_tok: device int32 [B], the number of
+ *     valid new tokens of sequence b (0 .. T), or NULL for T everywhere.  Rows
+ *     t >= n_tok[b] of out are not written.  A sequence with pos0[b] < 0, n_tok
+ *     outside 0 .. T or pos0[b] + n_tok[b] > Lmax raises GQA_DEV_BAD_LEN or
+ *     GQA_DEV_CAPACITY and none of its rows is written.
+ *   max_pos0_host: host-known upper bound of pos0 (max_pos0_host + T <= Lmax,
+ *     else GQA_ERR_CAPACITY).  pos0, n_tok 4-byte aligned, the rest 16.
+ * pos0 all zero and n_tok NULL give gqa_prefill's result bit for bit.
+ */
+gqa_status gqa_prefill_chunk(const void *q, const void *k_cache, const void *v_cache,
+                             void *out, const int32_t *pos0, const int32_t *n_tok,
+                             int max_pos0_host, int B, int T, int Hq, int Hkv, int D,
+                             int Lmax, float scale, int32_t *status_dev, void *stream);
+
+/*
  * gqa_decode -- one query token per sequence against the cache:
  *     out[b, h, :] = sum_{s < lens[b]} softmax_s(q[b,h,:] . K[b, h/g, s, :] * scale)
  *                                      * V[b, h/g, s, :]

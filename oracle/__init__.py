@@ -15,7 +15,9 @@ steps together in the order the pages give them:
   same pages, sections "无效的方法" and "V2：引入前沿技术".
 * a decode step appends the new token's rotated k and raw v at position
   ``lens[b]`` and attends over ``lens[b] + 1`` keys -- page "750美元从零训练3个LLM",
-  section "V3：扩容与推理优化".
+  section "V3：扩容与推理优化"; a continuation chunk does the same for T tokens
+  at once, token t at position ``pos0[b] + t`` seeing the cache and the chunk's
+  earlier tokens (the same section, taken a chunk at a time).
 
 Inputs are bfloat16 bit patterns (``numpy.uint16``), widened exactly to float64.
 """
@@ -193,6 +195,44 @@ def prefill(q_bits, k_bits, v_bits, qk_norm: bool, eps: float = 1e-6,
     v = widen(v_bits)
     o = attention(q, k, v, pos, scale, rows, nthreads)
     return o, k, v
+
+
+def prefill_chunk(q_bits, k_bits, v_bits, k_cache_bits, v_cache_bits, pos0,
+                  qk_norm: bool, n_tok=None, eps: float = 1e-6, base: float = 10000.0,
+                  scale: float | None = None, rows=None, nthreads: int = 0):
+    """A continuation chunk of T new tokens per sequence.
+
+    q [B, T, Hq, D], k/v [B, T, Hkv, D] are raw projections; k_cache/v_cache
+    [B, Hkv, Lmax, D] hold rotated K and raw V in slots 0 .. pos0[b]-1 (bf16 bits,
+    or float64).  Token t < n_tok[b] of sequence b is normed and rotated at
+    position pos0[b] + t, joins the cache at that slot, and attends to slots
+    0 .. pos0[b] + t.  Returns (o [B, T, Hq, D], k_rot [B, T, Hkv, D]) in
+    float64; rows t >= n_tok[b] of o are NaN.
+    """
+    B, T = q_bits.shape[:2]
+    Hkv = k_bits.shape[2]
+    D = q_bits.shape[3]
+    pos0 = np.broadcast_to(np.asarray(pos0, dtype=np.int64), (B,))
+    n_tok = np.full(B, T, dtype=np.int64) if n_tok is None else np.asarray(n_tok, np.int64)
+    pos = positions(pos0, B, T)
+    q = prep(q_bits, pos, qk_norm, eps, base)
+    k = prep(k_bits, pos, qk_norm, eps, base)
+    v = widen(v_bits)
+    kc = widen(k_cache_bits)
+    vc = widen(v_cache_bits)
+    Tk = max(1, int((pos0 + n_tok).max()))
+    keys = np.zeros((B, Tk, Hkv, D))
+    vals = np.zeros((B, Tk, Hkv, D))
+    for b in range(B):
+        P, n = int(pos0[b]), int(n_tok[b])
+        keys[b, :P] = kc[b, :, :P].transpose(1, 0, 2)
+        vals[b, :P] = vc[b, :, :P].transpose(1, 0, 2)
+        keys[b, P:P + n] = k[b, :n]
+        vals[b, P:P + n] = v[b, :n]
+    o = attention(q, keys, vals, pos, scale, rows, nthreads)
+    for b in range(B):
+        o[b, int(n_tok[b]):] = np.nan
+    return o, k
 
 
 def decode_step(q_bits, k_bits, v_bits, k_cache_bits, v_cache_bits, lens,

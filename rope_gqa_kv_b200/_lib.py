@@ -38,6 +38,8 @@ SIGNATURES = {
     "gqa_rope_append": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _i,
                              RopeParams, _vp, _vp]),
     "gqa_prefill": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp, _vp]),
+    "gqa_prefill_chunk": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f,
+                               _vp, _vp]),
     "gqa_decode": (_i, [_vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _f, _vp, _sz,
                         _vp, _vp]),
     "gqa_decode_workspace_bytes": (_sz, [_i, _i, _i, _i]),
@@ -183,6 +185,36 @@ def gqa_prefill(q, k_cache, v_cache, out=None, scale=0.0, status=None, stream=No
     _check("gqa_prefill", load().gqa_prefill(
         _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(out), B, T, Hq, Hkv, D, Lmax,
         float(scale), _ptr(status), _stream(stream)))
+    return out
+
+
+def gqa_prefill_chunk(q, k_cache, v_cache, pos0, max_pos0, n_tok=None, out=None, scale=0.0,
+                      status=None, stream=None):
+    """Causal attention of T new tokens per sequence continuing a cached prefix:
+    query t of sequence b sits at position pos0[b] + t.  q [B, T, Hq, D] -> out;
+    rows t >= n_tok[b] of out are left as they were."""
+    _need(q, "q", torch.bfloat16, 4)
+    _need(k_cache, "k_cache", torch.bfloat16, 4)
+    _need(v_cache, "v_cache", torch.bfloat16, 4)
+    _need(pos0, "pos0", torch.int32, 1)
+    B, T, Hq, D = q.shape
+    Hkv, Lmax = k_cache.shape[1], k_cache.shape[2]
+    if k_cache.shape != (B, Hkv, Lmax, D) or v_cache.shape != k_cache.shape:
+        raise ValueError("cache shape disagrees with q")
+    if pos0.shape != (B,):
+        raise ValueError("pos0 must be [B]")
+    if n_tok is not None:
+        _need(n_tok, "n_tok", torch.int32, 1)
+        if n_tok.shape != (B,):
+            raise ValueError("n_tok must be [B]")
+    if out is None:
+        out = torch.empty_like(q)
+    _need(out, "out", torch.bfloat16, 4)
+    if status is not None:
+        _need(status, "status", torch.int32)
+    _check("gqa_prefill_chunk", load().gqa_prefill_chunk(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(out), _ptr(pos0), _ptr(n_tok),
+        int(max_pos0), B, T, Hq, Hkv, D, Lmax, float(scale), _ptr(status), _stream(stream)))
     return out
 
 

@@ -1,20 +1,25 @@
 // prefill.cu -- causal GQA prefill on the 5th-generation tensor cores (tcgen05).
 //
-// out[b,t,h] = sum_{s<=t} softmax_s(q[b,t,h] . K[b,h/g,s] * scale) V[b,h/g,s]:
-// the causal scaled_dot_product_attention of page "训练3.8B LLM至0.384 CORE，
-// 成本998美元 – Hugo Vergnes" (section "无效的方法"), with query heads sharing
-// K/V heads in groups (page "750美元从零训练3个LLM：一位开发者的实战复盘", section
-// "V2：引入前沿技术").  Flash-style: the softmax is taken online over key tiles in
-// fp32, so the T x T score matrix never exists outside the tensor memory.
+// out[b,t,h] = sum_{s<=p(t)} softmax_s(q[b,t,h] . K[b,h/g,s] * scale) V[b,h/g,s]
+// with p(t) = pos0[b] + t: the causal scaled_dot_product_attention of page
+// "训练3.8B LLM至0.384 CORE，成本998美元 – Hugo Vergnes" (section "无效的方法"),
+// with query heads sharing K/V heads in groups (page "750美元从零训练3个LLM：一位
+// 开发者的实战复盘", section "V2：引入前沿技术").  pos0 = 0 is a prompt prefill;
+// pos0 > 0 continues a cached prefix (the new tokens attend to the cache and to
+// each other causally, page "750美元从零训练3个LLM", section "V3：扩容与推理优化").
+// Flash-style: the softmax is taken online over key tiles in fp32, so the score
+// matrix never exists outside the tensor memory.
 //
-// One CTA owns two 128-row query tiles of one (b, h) -- rows [256i, 256i+128)
-// and [256i+128, 256i+256) -- and streams the key/value tiles they need.
+// Persistent: one CTA per SM walks a static list of items; an item is two
+// 128-row query tiles of one (b, h) -- rows [256i, 256i+128) and
+// [256i+128, 256i+256) of the new tokens -- and streams the key/value tiles
+// they need.  Items are numbered longest first.
 // Warp roles (384 threads, three warpgroups):
-//   warps 0-3  softmax of tile 0 (thread = query row = TMEM lane), 232 registers
-//   warps 4-7  softmax of tile 1, 232 registers
-//   warp 8     TMA producer: Q tiles once, then a K ring and a V ring  } 40
-//   warp 9     MMA issuer (one thread): S_t = Q_t K^T and O_t += P_t V } registers
-//   warps 10-11 idle (they complete the third warpgroup)              }
+//   warps 0-3  softmax of tile 0 (thread = query row = TMEM lane), 208 registers
+//   warps 4-7  softmax of tile 1, 208 registers
+//   warp 8     TMA producer: Q tiles, then a K ring and a V ring    } 88
+//   warp 9     MMA issuer (one thread): S_t = Q_t K^T, O_t += P_t V } registers
+//   warps 10-11 idle (they complete the third warpgroup)            }
 // Tensor memory (512 columns): S0 [0,128) S1 [128,256) fp32 scores, with the
 // bf16 probabilities P_t written over the first 64 columns of S_t; O0 [256, 256+D)
 // O1 [384, 384+D) fp32 accumulators.
@@ -24,6 +29,13 @@
 // rescale O_t in TMEM as soon as its next scores are ready.  O_t is only
 // rescaled when the running maximum grows by more than 2^8 (the stale maximum
 // otherwise keeps p <= 256, exact in the final normalisation).
+//
+// Continuation chunks read the cache up to slot pos0 + n_tok - 1 (the last
+// valid key); slots past it in the item's last key tile may hold anything,
+// NaN included.  Their scores are masked, and before the last P . V product
+// the softmax group that owns it zeroes those rows of the V tile in shared
+// memory, so a zero probability never meets a NaN value.  (A prompt prefill
+// needs neither: its tensor maps end at row T and the copies zero-fill.)
 //
 // Every mbarrier wait is bounded; a role that times out raises GQA_DEV_TIMEOUT
 // and stops, the producer then waits (bounded) for its copies in flight and the
@@ -83,33 +95,66 @@ __device__ __forceinline__ uint32_t A(const uint64_t &b) { return ptx::smem_addr
 
 // Work item w of the grid's items: the query-tile pair, head and sequence it
 // covers.  Items are numbered longest first (pairs nearer the end of the
-// prompt see more keys), with the heads of one KV group side by side.
+// chunk see more keys), with the heads of one KV group side by side.
 struct PfItem {
     int b, h, kvh, q0, n0, n1, n_kv;
+    int P, N;          // first position of the chunk, valid new tokens (0: no work)
+    int r_valid;       // valid key rows in the last key tile (128: the tile is full)
     bool has1;
 };
 
-__device__ __forceinline__ PfItem pf_item(int w, int n_pairs, int B, int T, int Hq, int Hkv) {
+struct PfGrid {
+    int n_items, n_pairs, B, T, Hq, Hkv, Lmax;
+    const int32_t *pos0, *n_tok;   // chunk positions / token counts (NULL: 0 / T)
+};
+
+// (pos0[b], n_tok[b]) of a sequence; an invalid pair becomes "no work" (bad set).
+struct PfSeq {
+    int P, N;
+    bool bad;
+};
+template <bool kChunk>
+__device__ __forceinline__ PfSeq pf_seq(const PfGrid &g, int b) {
+    PfSeq q;
+    if constexpr (!kChunk) {
+        q.P = 0;
+        q.N = g.T;
+        q.bad = false;
+        return q;
+    }
+    q.P = g.pos0 ? g.pos0[b] : 0;
+    q.N = g.n_tok ? g.n_tok[b] : g.T;
+    q.bad = q.P < 0 || q.N < 0 || q.N > g.T || (long long)q.P + q.N > g.Lmax;
+    if (q.bad) q.N = 0;
+    return q;
+}
+__device__ __forceinline__ int pf_item_b(int w, int B, int Hq) {
     const int per_pair = Hq * B;
+    return (w % per_pair) / Hq;
+}
+
+__device__ __forceinline__ PfItem pf_item(int w, const PfGrid &g, PfSeq sq) {
+    const int per_pair = g.Hq * g.B;
     const int pi = w / per_pair;
     const int rest = w - pi * per_pair;
     PfItem it;
-    it.h = rest % Hq;
-    it.b = rest / Hq;
-    it.kvh = it.h / (Hq / Hkv);
-    it.q0 = (n_pairs - 1 - pi) * 256;
-    it.has1 = it.q0 + 128 < T;
-    it.n0 = (min(T, it.q0 + 128) + 127) / 128;
-    it.n1 = it.has1 ? (min(T, it.q0 + 256) + 127) / 128 : 0;
+    it.h = rest % g.Hq;
+    it.b = rest / g.Hq;
+    it.kvh = it.h / (g.Hq / g.Hkv);
+    it.q0 = (g.n_pairs - 1 - pi) * 256;
+    it.P = sq.P;
+    it.N = sq.N;
+    const bool has0 = it.q0 < it.N;
+    it.has1 = it.q0 + 128 < it.N;
+    it.n0 = has0 ? (it.P + min(it.N, it.q0 + 128) + 127) / 128 : 0;
+    it.n1 = it.has1 ? (it.P + min(it.N, it.q0 + 256) + 127) / 128 : 0;
     it.n_kv = it.has1 ? it.n1 : it.n0;
+    const int kv_end = it.P + min(it.N, it.q0 + 256);          // keys [0, kv_end) are valid
+    it.r_valid = it.n_kv > 0 ? kv_end - 128 * (it.n_kv - 1) : 128;
     return it;
 }
 
-struct PfGrid {
-    int n_items, n_pairs, B, T, Hq, Hkv;
-};
-
-template <int D>
+template <int D, bool kChunk>
 __device__ void producer(const PfMaps &maps, PfSync &sy, uint8_t *smem, const PfGrid &g,
                          int32_t *status) {
     using S = PfShape<D>;
@@ -118,8 +163,12 @@ __device__ void producer(const PfMaps &maps, PfSync &sy, uint8_t *smem, const Pf
     asm volatile("griddepcontrol.wait;" ::: "memory");
     int kc = 0, vc = 0, qc = 0;     // K, V tiles and Q pairs this CTA has loaded
     bool ok = true;
+    PfSeq nxt = blockIdx.x < g.n_items ? pf_seq<kChunk>(g, pf_item_b(blockIdx.x, g.B, g.Hq)) : PfSeq{0, 0, false};
     for (int w = blockIdx.x; w < g.n_items && ok; w += gridDim.x) {
-        const PfItem I = pf_item(w, g.n_pairs, g.B, g.T, g.Hq, g.Hkv);
+        if (nxt.bad) report(status, nxt.P < 0 || nxt.N < 0 ? GQA_DEV_BAD_LEN : GQA_DEV_CAPACITY);
+        const PfItem I = pf_item(w, g, nxt);
+        if (w + (int)gridDim.x < g.n_items) nxt = pf_seq<kChunk>(g, pf_item_b(w + gridDim.x, g.B, g.Hq));
+        if (I.n_kv == 0) continue;
         // The previous item's last S MMA has released the Q tiles.
         ok = ptx::mbar_wait(A(sy.q_empty), (qc & 1) ^ 1);
         if (!ok) break;
@@ -168,7 +217,7 @@ __device__ void producer(const PfMaps &maps, PfSync &sy, uint8_t *smem, const Pf
     }
 }
 
-template <int D>
+template <int D, bool kChunk>
 __device__ void mma_issuer(PfSync &sy, uint8_t *smem, uint32_t tmem, const PfGrid &g,
                            int32_t *status) {
     using S = PfShape<D>;
@@ -201,8 +250,11 @@ __device__ void mma_issuer(PfSync &sy, uint8_t *smem, uint32_t tmem, const PfGri
     int kc = 0, vc = 0, qc = 0;     // K, V tiles and Q pairs consumed
     int pc0 = 0, pc1 = 0;           // P hand-overs received from each softmax group
     bool ok = true;
+    PfSeq nxt = blockIdx.x < g.n_items ? pf_seq<kChunk>(g, pf_item_b(blockIdx.x, g.B, g.Hq)) : PfSeq{0, 0, false};
     for (int w = blockIdx.x; w < g.n_items && ok; w += gridDim.x) {
-        const PfItem I = pf_item(w, g.n_pairs, g.B, g.T, g.Hq, g.Hkv);
+        const PfItem I = pf_item(w, g, nxt);
+        if (w + (int)gridDim.x < g.n_items) nxt = pf_seq<kChunk>(g, pf_item_b(w + gridDim.x, g.B, g.Hq));
+        if (I.n_kv == 0) continue;
         const int kc0 = kc;
         ok = ptx::mbar_wait(A(sy.q_full), qc & 1) &&
              ptx::mbar_wait(A(sy.k_full[kc0 % S::kStagesK]), (kc0 / S::kStagesK) & 1);
@@ -268,23 +320,34 @@ __device__ void mma_issuer(PfSync &sy, uint8_t *smem, uint32_t tmem, const PfGri
     ptx::mbar_wait(A(sy.mma_done), 0);
 }
 
-template <int D>
-__device__ void softmax_tile(PfSync &sy, uint32_t tmem, int t, const PfGrid &g, float scale_log2,
-                             uint16_t *__restrict__ out, int32_t *status) {
+template <int D, bool kChunk>
+__device__ void softmax_tile(PfSync &sy, uint8_t *smem, uint32_t tmem, int t, const PfGrid &g,
+                             float scale_log2, uint16_t *__restrict__ out, int32_t *status) {
+    using S = PfShape<D>;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int row = (warp & 3) * 32 + lane;
     const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const uint32_t s_col = t * 128, o_col = 256 + t * 128;
     const int T = g.T;
     int sc = 0, oc = 0;             // scores and outputs of this tile received
+    int vc = 0;                     // V tiles of the items before this one
     bool ok = true;
+    PfSeq nxt = blockIdx.x < g.n_items ? pf_seq<kChunk>(g, pf_item_b(blockIdx.x, g.B, g.Hq)) : PfSeq{0, 0, false};
     for (int w = blockIdx.x; w < g.n_items && ok; w += gridDim.x) {
-        const PfItem I = pf_item(w, g.n_pairs, g.B, g.T, g.Hq, g.Hkv);
-        if (t == 1 && !I.has1) continue;
+        const PfItem I = pf_item(w, g, nxt);
+        if (w + (int)gridDim.x < g.n_items) nxt = pf_seq<kChunk>(g, pf_item_b(w + gridDim.x, g.B, g.Hq));
+        const int vc0 = vc;
+        vc += I.n_kv;
+        if (I.n_kv == 0 || (t == 1 && !I.has1)) continue;
         const int q_first = I.q0 + 128 * t;
         const int nt = t == 0 ? I.n0 : I.n1;
         const int qrow = q_first + row;
-        const int diag = q_first / 128;
+        const int lim0 = I.P + q_first;          // the tile's first row sees keys <= lim0
+        const int qlim = I.P + qrow;             // this row sees keys <= qlim
+        // the group whose last key tile is the item's last one clears that V tile's
+        // rows past the last valid key (continuation chunks only)
+        const bool clears = kChunk && I.r_valid < 128 && nt == I.n_kv &&
+                            (t == 0 ? true : I.n0 < I.n_kv);
         float m = -INFINITY, l = 0.f;
         for (int j = 0; j < nt; ++j) {
             ok = __all_sync(0xffffffffu, ptx::mbar_wait(A(sy.s_full[t]), sc & 1));
@@ -297,12 +360,10 @@ __device__ void softmax_tile(PfSync &sy, uint32_t tmem, int t, const PfGrid &g, 
             ptx::tmem_wait_ld();
 #define SV(c) __uint_as_float(sv[(c) >> 5][(c) & 31])
             const int key0 = j * 128;
-            if (j == diag || key0 + 128 > T) {
+            if (key0 + 127 > lim0) {
 #pragma unroll
-                for (int c = 0; c < 128; ++c) {
-                    const int key = key0 + c;
-                    if (key > qrow || key >= T) sv[c >> 5][c & 31] = __float_as_uint(-INFINITY);
-                }
+                for (int c = 0; c < 128; ++c)
+                    if (key0 + c > qlim) sv[c >> 5][c & 31] = __float_as_uint(-INFINITY);
             }
             // Row maximum: four independent chains of three-input max.
             float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
@@ -355,6 +416,24 @@ __device__ void softmax_tile(PfSync &sy, uint32_t tmem, int t, const PfGrid &g, 
             }
 #undef SV
             l += (la0 + la1) + (lb0 + lb1);
+            if (clears && j == nt - 1) {
+                // The last V tile has landed once its barrier's phase completes;
+                // zero its rows past the last valid key, then publish the stores to
+                // the tensor core (async proxy) before P is handed over.
+                const int vidx = vc0 + I.n_kv - 1;
+                ok = __all_sync(0xffffffffu, ptx::mbar_wait(A(sy.v_full[vidx % S::kStagesV]),
+                                                             (vidx / S::kStagesV) & 1));
+                if (ok) {
+                    uint8_t *vt = smem + S::kOffV + (vidx % S::kStagesV) * S::kTileBytes;
+                    const int n16 = (128 - I.r_valid) * 8;   // 16-byte pieces per column block
+                    for (int x = row; x < n16 * S::kBlocks; x += 128) {
+                        const int kb = x / n16, y = x - kb * n16;
+                        *reinterpret_cast<uint4 *>(vt + kb * S::kBlockBytes + I.r_valid * 128 + y * 16) =
+                            make_uint4(0, 0, 0, 0);
+                    }
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                }
+            }
             ptx::tmem_wait_st();
             ptx::tc_fence_before();
             __syncwarp();
@@ -376,7 +455,7 @@ __device__ void softmax_tile(PfSync &sy, uint32_t tmem, int t, const PfGrid &g, 
             for (int e = 0; e < 16; ++e)
                 w4[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l,
                                     __uint_as_float(o[2 * e + 1]) * inv_l);
-            if (qrow < T) {
+            if (qrow < I.N) {
                 uint4 *d4 = reinterpret_cast<uint4 *>(dst + 32 * c);
                 d4[0] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
                 d4[1] = make_uint4(w4[4], w4[5], w4[6], w4[7]);
@@ -391,10 +470,11 @@ __device__ void softmax_tile(PfSync &sy, uint32_t tmem, int t, const PfGrid &g, 
     if (!ok && lane == 0) report(status, GQA_DEV_TIMEOUT);
 }
 
-template <int D>
+template <int D, bool kChunk>
 __global__ void __launch_bounds__(kPfThreads, 1)
 prefill_kernel(const __grid_constant__ PfMaps maps, uint16_t *__restrict__ out, int B, int T,
-               int Hq, int Hkv, float scale_log2, int n_pairs, int32_t *status) {
+               int Hq, int Hkv, int Lmax, const int32_t *__restrict__ pos0,
+               const int32_t *__restrict__ n_tok, float scale_log2, int n_pairs, int32_t *status) {
     using S = PfShape<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -406,6 +486,9 @@ prefill_kernel(const __grid_constant__ PfMaps maps, uint16_t *__restrict__ out, 
     g.T = T;
     g.Hq = Hq;
     g.Hkv = Hkv;
+    g.Lmax = Lmax;
+    g.pos0 = pos0;
+    g.n_tok = n_tok;
     g.n_items = n_pairs * Hq * B;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -445,15 +528,15 @@ prefill_kernel(const __grid_constant__ PfMaps maps, uint16_t *__restrict__ out, 
     if (warp >= 8) {
         ptx::regs_dec<kControlRegs>();
         if (warp == kTmaWarp) {
-            if (lane == 0) producer<D>(maps, sy, smem, g, status);
+            if (lane == 0) producer<D, kChunk>(maps, sy, smem, g, status);
             __syncwarp();
         } else if (warp == kMmaWarp) {
-            if (lane == 0) mma_issuer<D>(sy, smem, tmem, g, status);
+            if (lane == 0) mma_issuer<D, kChunk>(sy, smem, tmem, g, status);
             __syncwarp();
         }
     } else {
         ptx::regs_inc<kSoftmaxRegs>();
-        softmax_tile<D>(sy, tmem, warp >> 2, g, scale_log2, out, status);
+        softmax_tile<D, kChunk>(sy, smem, tmem, warp >> 2, g, scale_log2, out, status);
     }
     ptx::tc_fence_before();
     __syncthreads();
@@ -497,8 +580,8 @@ bool encode(CUtensorMap *m, const void *base, int rank, const cuuint64_t *dims,
 
 template <int D>
 gqa_status launch_prefill(const void *q, const void *kc, const void *vc, void *out, int B, int T,
-                          int Hq, int Hkv, int Lmax, float scale_log2, int32_t *status,
-                          cudaStream_t s) {
+                          int Hq, int Hkv, int Lmax, const int32_t *pos0, const int32_t *n_tok,
+                          float scale_log2, int32_t *status, cudaStream_t s) {
     using S = PfShape<D>;
     PfMaps maps;
     {
@@ -509,15 +592,18 @@ gqa_status launch_prefill(const void *q, const void *kc, const void *vc, void *o
         if (!encode(&maps.q, q, 4, dims, str, box)) return GQA_ERR_CUDA;
     }
     {
-        // Rows beyond T are outside the map, so the copies zero-fill them and
-        // the unused cache slots (whatever they hold) are never read.
-        const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)T, (cuuint64_t)B * Hkv};
+        // A prompt (no pos0): rows beyond T are outside the map, so the copies
+        // zero-fill them and the unused cache slots (whatever they hold) are
+        // never read.  A continuation chunk reads up to slot pos0 + n_tok - 1,
+        // so its maps span the whole cache.
+        const cuuint64_t rows = pos0 ? (cuuint64_t)Lmax : (cuuint64_t)T;
+        const cuuint64_t dims[3] = {(cuuint64_t)D, rows, (cuuint64_t)B * Hkv};
         const cuuint64_t str[2] = {(cuuint64_t)D * 2, (cuuint64_t)Lmax * D * 2};
         const cuuint32_t box[3] = {64, 128, 1};
         if (!encode(&maps.k, kc, 3, dims, str, box)) return GQA_ERR_CUDA;
         if (!encode(&maps.v, vc, 3, dims, str, box)) return GQA_ERR_CUDA;
     }
-    auto kern = prefill_kernel<D>;
+    auto kern = pos0 ? prefill_kernel<D, true> : prefill_kernel<D, false>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kSmem) !=
         cudaSuccess)
         return GQA_ERR_CUDA;
@@ -546,8 +632,8 @@ gqa_status launch_prefill(const void *q, const void *kc, const void *vc, void *o
     cfg.stream = s;
     cfg.attrs = pdl;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, kern, maps, static_cast<uint16_t *>(out), B, T, Hq, Hkv,
-                           scale_log2, n_pairs, status) != cudaSuccess)
+    if (cudaLaunchKernelEx(&cfg, kern, maps, static_cast<uint16_t *>(out), B, T, Hq, Hkv, Lmax,
+                           pos0, n_tok, scale_log2, n_pairs, status) != cudaSuccess)
         return GQA_ERR_CUDA;
     return gqa_host::launch_status();
 }
@@ -563,26 +649,50 @@ bool device_is_sm100() {
 }  // namespace
 }  // namespace gqa
 
-extern "C" gqa_status gqa_prefill(const void *q, const void *k_cache, const void *v_cache,
-                                  void *out, int B, int T, int Hq, int Hkv, int D, int Lmax,
-                                  float scale, int32_t *status_dev, void *stream) {
+namespace {
+
+gqa_status prefill_entry(const void *q, const void *k_cache, const void *v_cache, void *out,
+                         const int32_t *pos0, const int32_t *n_tok, int max_pos0_host, int B,
+                         int T, int Hq, int Hkv, int D, int Lmax, float scale, int32_t *status_dev,
+                         void *stream) {
     using namespace gqa_host;
     if (!q || !k_cache || !v_cache || !out || B < 1 || T < 1 || Hq < 1 || Hkv < 1 || Lmax < 1)
         return GQA_ERR_INVALID_ARG;
     if (Hq % Hkv != 0) return GQA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
         return GQA_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(pos0) & 3u) || (reinterpret_cast<uintptr_t>(n_tok) & 3u))
+        return GQA_ERR_INVALID_ARG;
     if (!head_dim_ok(D)) return GQA_ERR_UNSUPPORTED;
     if (Lmax % 128 != 0) return GQA_ERR_INVALID_ARG;
-    if (T > Lmax) return GQA_ERR_CAPACITY;
+    if (max_pos0_host < 0) return GQA_ERR_INVALID_ARG;
+    if ((long long)max_pos0_host + T > Lmax) return GQA_ERR_CAPACITY;
     if ((long long)((T + 255) / 256) * Hq * B > 0x7fffffffLL) return GQA_ERR_INVALID_ARG;
     if (!gqa::device_is_sm100()) return GQA_ERR_UNSUPPORTED;
     const float sc = scale > 0.f ? scale : 1.0f / sqrtf((float)D);
     const float sl2 = sc * 1.4426950408889634f;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     switch (D) {
-        case 64: return gqa::launch_prefill<64>(q, k_cache, v_cache, out, B, T, Hq, Hkv, Lmax, sl2, status_dev, s);
-        case 96: return gqa::launch_prefill<96>(q, k_cache, v_cache, out, B, T, Hq, Hkv, Lmax, sl2, status_dev, s);
-        default: return gqa::launch_prefill<128>(q, k_cache, v_cache, out, B, T, Hq, Hkv, Lmax, sl2, status_dev, s);
+        case 64: return gqa::launch_prefill<64>(q, k_cache, v_cache, out, B, T, Hq, Hkv, Lmax, pos0, n_tok, sl2, status_dev, s);
+        case 96: return gqa::launch_prefill<96>(q, k_cache, v_cache, out, B, T, Hq, Hkv, Lmax, pos0, n_tok, sl2, status_dev, s);
+        default: return gqa::launch_prefill<128>(q, k_cache, v_cache, out, B, T, Hq, Hkv, Lmax, pos0, n_tok, sl2, status_dev, s);
     }
+}
+
+}  // namespace
+
+extern "C" gqa_status gqa_prefill(const void *q, const void *k_cache, const void *v_cache,
+                                  void *out, int B, int T, int Hq, int Hkv, int D, int Lmax,
+                                  float scale, int32_t *status_dev, void *stream) {
+    return prefill_entry(q, k_cache, v_cache, out, nullptr, nullptr, 0, B, T, Hq, Hkv, D, Lmax,
+                         scale, status_dev, stream);
+}
+
+extern "C" gqa_status gqa_prefill_chunk(const void *q, const void *k_cache, const void *v_cache,
+                                        void *out, const int32_t *pos0, const int32_t *n_tok,
+                                        int max_pos0_host, int B, int T, int Hq, int Hkv, int D,
+                                        int Lmax, float scale, int32_t *status_dev, void *stream) {
+    if (!pos0) return GQA_ERR_INVALID_ARG;
+    return prefill_entry(q, k_cache, v_cache, out, pos0, n_tok, max_pos0_host, B, T, Hq, Hkv, D,
+                         Lmax, scale, status_dev, stream);
 }

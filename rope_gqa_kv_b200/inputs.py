@@ -6,8 +6,8 @@ both the CUDA path and the float64 oracle can take their inputs from it.
 Recipe (the same for every workload):
 * one CPU ``torch.Generator`` seeded with ``seed`` (1000 + workload index for
   the named workloads);
-* draw order: cached lengths (batched decode only), cache K, cache V, prompt
-  q, k, v, then q, k, v of each decode step;
+* draw order: cached lengths (workloads with a cached prefix only), cache K,
+  cache V, prompt (or chunk) q, k, v, then q, k, v of each decode step;
 * values ``torch.randn`` in float32, rounded to bfloat16 (round-to-nearest-even);
   cached lengths ``randint(lo, hi + 1)``;
 * cache capacity Lmax = the longest sequence the workload reaches, rounded up
@@ -18,6 +18,8 @@ Recipe (the same for every workload):
 Shapes follow the models the pages describe: a 12-layer / 768-hidden / 8-head
 decoder (head_dim 96), the 3.8B Llama-style model (24 query heads, 8 KV heads,
 QK-norm, head_dim 128), and a 512-token prompt followed by 100 generated tokens.
+A workload with both a cached prefix and T > 0 is a continuation chunk: T new
+tokens per sequence starting at position lens[b].
 """
 from __future__ import annotations
 
@@ -37,10 +39,10 @@ class Workload:
     Hq: int
     Hkv: int
     D: int
-    T: int                      # prompt tokens prefilled from position 0 (0: none)
+    T: int                      # new tokens: a prompt from 0, or a chunk after the cache
     decode_steps: int           # single-token steps after the prompt
     qk_norm: bool
-    cached_len_range: Optional[tuple] = None   # batched decode: lens ~ U[lo, hi]
+    cached_len_range: Optional[tuple] = None   # cached prefix: lens ~ U[lo, hi]
     rope_base: float = 10000.0
     eps: float = 1e-6
 
@@ -62,7 +64,7 @@ class Workload:
     @property
     def max_len(self) -> int:
         if self.cached_len_range is not None:
-            return self.cached_len_range[1] + self.decode_steps
+            return self.cached_len_range[1] + self.T + self.decode_steps
         return self.T + self.decode_steps
 
     @property
@@ -81,6 +83,9 @@ WORKLOADS = [
     Workload("prefill_3p8b", 3, B=8, Hq=24, Hkv=8, D=128, T=2048, decode_steps=0, qk_norm=True),
     Workload("batched_decode", 4, B=64, Hq=24, Hkv=8, D=128, T=0, decode_steps=1, qk_norm=True,
              cached_len_range=(256, 2048)),
+    # continuation chunk: 1024 new tokens after cached prefixes of 512 .. 1536
+    Workload("chunked_prefill_3p8b", 5, B=8, Hq=24, Hkv=8, D=128, T=1024, decode_steps=0,
+             qk_norm=True, cached_len_range=(512, 1536)),
 ]
 BY_NAME = {w.name: w for w in WORKLOADS}
 
@@ -94,7 +99,7 @@ def make_inputs(w: Workload, decode_steps: Optional[int] = None, seed: Optional[
     """Draw one workload's inputs on the CPU (bfloat16 unless noted).
 
     Returns a dict with
-      lens     int32 [B]   cached lengths (batched decode) or None
+      lens     int32 [B]   cached lengths (workloads with a prefix) or None
       k_cache, v_cache     [B, Hkv, Lmax, D]: random in slots < lens, NaN after
       q, k, v              prompt projections [B, T, H, D] (None when T == 0)
       steps                list of (q [B, Hq, D], k [B, Hkv, D], v [B, Hkv, D])

@@ -32,7 +32,8 @@ def declared_functions():
 
 def test_header_declares_the_four_entry_points():
     names = declared_functions()
-    for n in ("gqa_rope_apply", "kv_cache_append", "gqa_prefill", "gqa_decode"):
+    for n in ("gqa_rope_apply", "kv_cache_append", "gqa_prefill", "gqa_decode",
+              "gqa_prefill_chunk"):
         assert n in names
 
 
@@ -94,6 +95,27 @@ def test_prefill_validation(lib):
     assert lib.gqa_prefill(f, f, f, f, 1, 300, 4, 2, 64, 256, 0.0, None, None) == 3
     assert lib.gqa_prefill(f, f, f, ODD, 1, 10, 4, 2, 64, 128, 0.0, None, None) == 1
     assert lib.gqa_prefill(f, f, f, f, 1, 0, 4, 2, 64, 128, 0.0, None, None) == 1
+
+
+def test_prefill_chunk_validation(lib):
+    f = FAKE
+    odd4 = ctypes.c_void_p(0x10002)      # not 4-byte aligned
+    # pos0 is required
+    assert lib.gqa_prefill_chunk(f, f, f, f, None, None, 0, 1, 10, 4, 2, 64, 128, 0.0,
+                                 None, None) == 1
+    # max_pos0 + T beyond the cache
+    assert lib.gqa_prefill_chunk(f, f, f, f, f, None, 100, 1, 29, 4, 2, 64, 128, 0.0,
+                                 None, None) == 3
+    assert lib.gqa_prefill_chunk(f, f, f, f, f, None, -1, 1, 10, 4, 2, 64, 128, 0.0,
+                                 None, None) == 1
+    assert lib.gqa_prefill_chunk(f, f, f, f, odd4, None, 0, 1, 10, 4, 2, 64, 128, 0.0,
+                                 None, None) == 1
+    assert lib.gqa_prefill_chunk(f, f, f, f, f, odd4, 0, 1, 10, 4, 2, 64, 128, 0.0,
+                                 None, None) == 1
+    assert lib.gqa_prefill_chunk(f, f, f, f, f, None, 0, 1, 10, 4, 2, 48, 128, 0.0,
+                                 None, None) == 2
+    assert lib.gqa_prefill_chunk(f, f, f, f, f, None, 0, 1, 10, 6, 4, 64, 128, 0.0,
+                                 None, None) == 1
 
 
 def test_decode_validation(lib):

@@ -4,7 +4,9 @@ The batched-decode workload at full size (B=64, 24/8 heads, D=128, cached
 lengths U[256, 2048], QK-norm, NaN in every slot past each length), the
 generation loops of the tiny and 512+100 workloads, and the edge cases: a
 cache of one token, a full cache, MHA and MQA groupings, head_dim 96, and
-invalid lengths.
+invalid lengths; and the shapes that stress the split over 64-slot chunks: one
+long sequence of 313 chunks per row, problems with fewer chunks than SMs, and
+lengths on and around multiples of 64.
 """
 import numpy as np
 import pytest
@@ -186,3 +188,40 @@ def test_workspace_reuse_and_garbage_contents(cuda_lib):
                             oracle.bf16_to_f64(bits(x["v_cache"])).transpose(0, 2, 1, 3),
                             (x["lens"].numpy() - 1)[:, None].astype(np.int64))[:, 0]
     assert_close(outs[0], want, "decode with a reused workspace")
+
+
+def _decode_vs_oracle(B, Hq, Hkv, D, L, lens_list, seed, label):
+    g = torch.Generator().manual_seed(seed)
+    q = torch.randn(B, Hq, D, generator=g).to(torch.bfloat16)
+    kc = torch.randn(B, Hkv, L, D, generator=g).to(torch.bfloat16)
+    vc = torch.randn(B, Hkv, L, D, generator=g).to(torch.bfloat16)
+    lens = torch.tensor(lens_list, dtype=torch.int32)
+    for b, n in enumerate(lens_list):          # NaN past every length
+        kc[b, :, n:] = float("nan")
+        vc[b, :, n:] = float("nan")
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    out = gqa.gqa_decode(q.to(DEV), kc.to(DEV), vc.to(DEV), lens.to(DEV), max(lens_list),
+                         status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    want = oracle.attention(oracle.bf16_to_f64(bits(q))[:, None],
+                            oracle.bf16_to_f64(bits(kc)).transpose(0, 2, 1, 3),
+                            oracle.bf16_to_f64(bits(vc)).transpose(0, 2, 1, 3),
+                            (lens.numpy() - 1)[:, None].astype(np.int64))[:, 0]
+    assert_close(out, want, label)
+
+
+def test_long_sequence_many_chunks(cuda_lib):
+    # one sequence of 20000 slots, MQA with 8 query heads (4 subgroups of 2
+    # heads): 313 chunks per subgroup for the merge to combine
+    _decode_vs_oracle(1, 8, 1, 128, 20096, [20000], 91, "one long MQA sequence")
+
+
+def test_fewer_chunks_than_sms(cuda_lib):
+    # 2 sequences of 1 and 2 chunks, 2 KV heads each: 6 chunk CTAs in all
+    _decode_vs_oracle(2, 4, 2, 64, 256, [30, 70], 92, "six chunks")
+
+
+def test_lengths_around_unit_edges(cuda_lib):
+    lens = [1, 63, 64, 65, 127, 128, 129, 191, 192, 640, 1, 2]
+    _decode_vs_oracle(len(lens), 12, 4, 96, 640, lens, 93, "lengths around multiples of 64")

@@ -14,8 +14,9 @@ def test_named_workloads_and_capacities():
         "generation": (1, 16, 4, 64, 512, 100, False, 640),
         "prefill_3p8b": (8, 24, 8, 128, 2048, 0, True, 2048),
         "batched_decode": (64, 24, 8, 128, 0, 1, True, 2176),
+        "chunked_prefill_3p8b": (8, 24, 8, 128, 1024, 0, True, 2560),
     }
-    assert [w.seed for w in inputs.WORKLOADS] == [1000, 1001, 1002, 1003, 1004]
+    assert [w.seed for w in inputs.WORKLOADS] == [1000, 1001, 1002, 1003, 1004, 1005]
 
 
 def test_config_assertions():
@@ -49,3 +50,14 @@ def test_prefill_workload_cache_starts_empty():
     assert a["q"].shape == (2, 70, 4, 96) and a["q"].dtype == torch.bfloat16
     assert (a["k_cache"].view(torch.int16) == inputs.BF16_QNAN_BITS).all()
     assert a["k_cache"].shape == (2, 2, 128, 96)
+
+
+def test_chunk_workload_has_prefix_and_new_tokens():
+    w = inputs.custom("k", B=3, Hq=4, Hkv=2, D=64, T=50, cached_len_range=(10, 100))
+    a = inputs.make_inputs(w)
+    assert w.Lmax == 256                    # 100 cached + 50 new, rounded up to 128
+    assert a["q"].shape == (3, 50, 4, 64)
+    for bi, n in enumerate(a["lens"].tolist()):
+        assert 10 <= n <= 100
+        assert not torch.isnan(a["k_cache"][bi, :, :n].float()).any()
+        assert torch.isnan(a["k_cache"][bi, :, n:].float()).all()

@@ -311,3 +311,56 @@ def test_decode_ignores_slots_beyond_length():
         vc[b, :, lens[b]:] = np.nan
     o2, _ = oracle.decode_step(q, k, v, kc, vc, lens, True)
     np.testing.assert_array_equal(o1, o2)
+
+
+# ---------------------------------------------------------------------------
+# continuation chunks: the same check a chunk of tokens at a time
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("qk_norm", [False, True])
+def test_chunked_prefill_equals_one_prefill(qk_norm):
+    """A prompt taken in chunks (different cut points per sequence, the last
+    chunk ragged) gives the rows and the rotated keys of one prefill."""
+    rng = np.random.default_rng(12)
+    B, T, Hq, Hkv, D, Lmax = 2, 37, 6, 2, 16, 64
+    q = _rand_bits(rng, B, T, Hq, D)
+    k = _rand_bits(rng, B, T, Hkv, D)
+    v = _rand_bits(rng, B, T, Hkv, D)
+    o_full, k_rot, v_all = oracle.prefill(q, k, v, qk_norm)
+    cuts = [[0, 15, 30, 37], [0, 22, 37]]
+    kc = np.full((B, Hkv, Lmax, D), np.nan)     # slots past the prefix are never read
+    vc = np.full((B, Hkv, Lmax, D), np.nan)
+    got = np.full(o_full.shape, np.nan)
+    pos0 = np.zeros(B, dtype=np.int64)
+    for step in range(3):
+        n_tok = np.array([max(0, (c[step + 1] - c[step]) if step + 1 < len(c) else 0)
+                          for c in cuts])
+        Tc = int(n_tok.max())
+        qc = np.zeros((B, Tc, Hq, D), np.uint16)
+        kc_new = np.zeros((B, Tc, Hkv, D), np.uint16)
+        vc_new = np.zeros((B, Tc, Hkv, D), np.uint16)
+        for b in range(B):
+            P, n = int(pos0[b]), int(n_tok[b])
+            qc[b, :n], kc_new[b, :n], vc_new[b, :n] = q[b, P:P + n], k[b, P:P + n], v[b, P:P + n]
+        o, kr = oracle.prefill_chunk(qc, kc_new, vc_new, kc, vc, pos0, qk_norm, n_tok=n_tok)
+        for b in range(B):
+            P, n = int(pos0[b]), int(n_tok[b])
+            got[b, P:P + n] = o[b, :n]
+            assert np.isnan(o[b, n:]).all()
+            np.testing.assert_allclose(kr[b, :n], k_rot[b, P:P + n], rtol=0, atol=1e-15)
+            kc[b, :, P:P + n] = kr[b, :n].transpose(1, 0, 2)
+            vc[b, :, P:P + n] = v_all[b, P:P + n].transpose(1, 0, 2)
+        pos0 = pos0 + n_tok
+    np.testing.assert_allclose(got, o_full, rtol=0, atol=1e-13)
+
+
+def test_chunk_of_one_token_is_a_decode_step():
+    rng = np.random.default_rng(13)
+    B, Hq, Hkv, D, L = 3, 4, 1, 32, 48
+    lens = np.array([1, 20, 47])
+    kc = rng.standard_normal((B, Hkv, L, D))
+    vc = rng.standard_normal((B, Hkv, L, D))
+    q, k, v = (_rand_bits(rng, B, Hq, D), _rand_bits(rng, B, Hkv, D), _rand_bits(rng, B, Hkv, D))
+    o_dec, k_dec = oracle.decode_step(q, k, v, kc, vc, lens, True)
+    o_chk, k_chk = oracle.prefill_chunk(q[:, None], k[:, None], v[:, None], kc, vc, lens, True)
+    np.testing.assert_array_equal(o_chk[:, 0], o_dec)
+    np.testing.assert_array_equal(k_chk[:, 0], k_dec)
