@@ -376,10 +376,37 @@ def run_ours(args, rank, world, dev, dist_on):
         "clocks": clocks,
         "device_status": status,
     }
-    line["next_rows"] = {"chunked_prefill": measure_chunk(dev, peaks, tag)}
+    line["next_rows"] = {"chunked_prefill": measure_chunk(dev, peaks, tag),
+                         "rope_scaling": measure_scaled_append(layer, peaks, tag)}
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
     return line
+
+
+def measure_scaled_append(layer, peaks, tag, reps: int = 30):
+    """The prefill-sized fused QK-norm + RoPE + append with YaRN (s = 4 over a
+    2048-token trained length), outside the timed step: the same HBM-bound
+    kernel as plain RoPE with a different frequency table and a scale."""
+    import rope_gqa_kv_b200 as gqa
+    sc = gqa.RopeScaling("yarn", 4.0, original_max_pos=2048)
+    args = (layer.pq, layer.pk, layer.pv, layer.pkc, layer.pvc)
+    for _ in range(3):
+        gqa.gqa_rope_append(*args, qk_norm=True, max_pos0=0, status=layer.status, scaling=sc)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(reps)]
+    for i in range(reps):
+        ev[i][0].record()
+        gqa.gqa_rope_append(*args, qk_norm=True, max_pos0=0, status=layer.status, scaling=sc)
+        ev[i][1].record()
+    torch.cuda.synchronize()
+    ms = sorted(a.elapsed_time(b) for a, b in ev)[reps // 2]
+    gbs = append_bytes() / (ms * 1e-3) / 1e9
+    return {"workload": "prefill-sized append, YaRN s=4 over 2048 trained positions",
+            "kernel": "gqa_rope_append", "bound": "hbm", "us_median": round(ms * 1e3, 2),
+            "achieved": round(gbs, 1), "unit": "GB/s", "peak": peaks["hbm_gbs"],
+            "frac": round(gbs / peaks["hbm_gbs"], 4), "peak_kind": "hbm copy " + tag,
+            "algorithmic_per_launch": append_bytes(),
+            "l2": "inputs (335 MB moved per launch) exceed L2"}
 
 
 def measure_chunk(dev, peaks, tag, reps: int = 30):

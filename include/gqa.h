@@ -67,10 +67,34 @@ typedef enum {
 #define GQA_DEV_TIMEOUT 0x2    /* a bounded wait inside a kernel gave up: output invalid */
 #define GQA_DEV_BAD_LEN 0x4    /* a length or position < 0 (or 0 where >= 1 is needed) */
 
+/*
+ * RoPE for contexts longer than the one a model was trained on.  Page "750美元
+ * 从零训练3个LLM" (section "V1：现代架构基线") names NTK-aware scaling and YaRN as
+ * the length-extension methods RoPE works with; the formulas are those of the
+ * published methods (pair i, theta_i = base^(-2i/D), extension factor s):
+ *   GQA_ROPE_LINEAR  position interpolation: theta_i / s
+ *   GQA_ROPE_NTK     NTK-aware: the base becomes base * s^(D/(D-2)), so the
+ *                    fastest pair keeps its angle and the slowest is divided by s
+ *   GQA_ROPE_YARN    YaRN: with r_i = L theta_i / (2 pi) (turns of pair i over the
+ *                    trained length L) and g_i = clamp((r_i - alpha)/(beta - alpha),
+ *                    0, 1), theta_i' = (1 - g_i) theta_i / s + g_i theta_i; both
+ *                    rotated q and k are multiplied by 0.1 ln(s) + 1, which
+ *                    divides the logits by the temperature t of the method.
+ */
+#define GQA_ROPE_PLAIN 0
+#define GQA_ROPE_LINEAR 1
+#define GQA_ROPE_NTK 2
+#define GQA_ROPE_YARN 3
+
 typedef struct {
-    int qk_norm;       /* nonzero: unit-gain RMSNorm over D before RoPE */
-    float eps;         /* RMSNorm epsilon inside the root (1e-6 in the pages' model) */
-    float rope_base;   /* RoPE base (10000) */
+    int qk_norm;          /* nonzero: unit-gain RMSNorm over D before RoPE */
+    float eps;            /* RMSNorm epsilon inside the root (1e-6 in the pages' model) */
+    float rope_base;      /* RoPE base (10000) */
+    int scaling;          /* GQA_ROPE_*; zero-filled = plain RoPE */
+    float factor;         /* s >= 1 (used when scaling != GQA_ROPE_PLAIN) */
+    int original_max_pos; /* YaRN: L, the trained context length (>= 1) */
+    float yarn_alpha;     /* YaRN: 0 <= alpha < beta (the method's defaults: 1, 32) */
+    float yarn_beta;
 } gqa_rope_params;
 
 /*

@@ -67,6 +67,8 @@ def _load():
                                        ctypes.c_double]
         lib.oracle_rope.argtypes = [_f64p, _f64p, _i64p, ctypes.c_int64, ctypes.c_int,
                                     ctypes.c_int, ctypes.c_double, ctypes.c_int]
+        lib.oracle_rope_theta.argtypes = [_f64p, _f64p, _i64p, ctypes.c_int64, ctypes.c_int,
+                                          ctypes.c_int, _f64p, ctypes.c_int]
         lib.oracle_attention.argtypes = [_f64p, _f64p, _f64p, _i64p, _f64p,
                                          ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                          ctypes.c_int, ctypes.c_int, ctypes.c_int,
@@ -113,7 +115,49 @@ def rmsnorm(x, eps: float = 1e-6) -> np.ndarray:
     return y
 
 
-def rope(x, pos, base: float = 10000.0, interleaved: bool = False) -> np.ndarray:
+class RopeScaling:
+    """A RoPE context-extension method.  Page "750美元从零训练3个LLM", section
+    "V1：现代架构基线", names NTK-aware scaling and YaRN as the methods RoPE works
+    with; the pages give no formulas, so these follow the published methods:
+
+    * ``linear`` (position interpolation): every frequency divided by s;
+    * ``ntk`` (NTK-aware): the base raised to base * s^(D/(D-2)), so the fastest
+      pair keeps its frequency and the slowest one is divided by s;
+    * ``yarn``: pair i makes r_i = L theta_i / (2 pi) turns over the trained
+      length L; with the ramp g = 0 below r = alpha, 1 above r = beta and linear
+      between, theta_i' = (1 - g) theta_i / s + g theta_i (long wavelengths
+      interpolated, short ones kept), and the rotated vectors are multiplied by
+      0.1 ln(s) + 1 (the attention temperature).
+    """
+
+    def __init__(self, kind: str, factor: float, original_max_pos: int = 0,
+                 alpha: float = 1.0, beta: float = 32.0):
+        assert kind in ("linear", "ntk", "yarn")
+        self.kind, self.factor = kind, float(factor)
+        self.original_max_pos, self.alpha, self.beta = int(original_max_pos), float(alpha), float(beta)
+
+    def theta(self, D: int, base: float) -> np.ndarray:
+        """The D/2 frequencies theta_i' of the method."""
+        i = np.arange(D // 2, dtype=np.float64)
+        s = self.factor
+        if self.kind == "ntk":
+            base = base * s ** (D / (D - 2.0))
+        theta = base ** (-2.0 * i / D)
+        if self.kind == "linear":
+            return theta / s
+        if self.kind == "yarn":
+            turns = self.original_max_pos * theta / (2.0 * math.pi)
+            ramp = np.clip((turns - self.alpha) / (self.beta - self.alpha), 0.0, 1.0)
+            return (1.0 - ramp) * theta / s + ramp * theta
+        return theta
+
+    def mscale(self) -> float:
+        """Factor on the rotated q and k (YaRN only)."""
+        return 0.1 * math.log(self.factor) + 1.0 if self.kind == "yarn" else 1.0
+
+
+def rope(x, pos, base: float = 10000.0, interleaved: bool = False,
+         scaling: RopeScaling | None = None) -> np.ndarray:
     """Rotate x [..., N, H, D] (leading axes flattened into N) at positions pos [N]."""
     x = _f64(x)
     H, D = x.shape[-2], x.shape[-1]
@@ -121,9 +165,14 @@ def rope(x, pos, base: float = 10000.0, interleaved: bool = False) -> np.ndarray
     pos = np.ascontiguousarray(np.broadcast_to(pos, x.shape[:-2]), dtype=np.int64)
     assert pos.size == N
     y = np.empty_like(x)
-    _load().oracle_rope(_ptr(x, _f64p), _ptr(y, _f64p), _ptr(pos, _i64p), N, H, D,
-                        base, 1 if interleaved else 0)
-    return y
+    if scaling is None:
+        _load().oracle_rope(_ptr(x, _f64p), _ptr(y, _f64p), _ptr(pos, _i64p), N, H, D,
+                            base, 1 if interleaved else 0)
+        return y
+    theta = np.ascontiguousarray(scaling.theta(D, base))
+    _load().oracle_rope_theta(_ptr(x, _f64p), _ptr(y, _f64p), _ptr(pos, _i64p), N, H, D,
+                              _ptr(theta, _f64p), 1 if interleaved else 0)
+    return y * scaling.mscale()
 
 
 def attention(q, k, v, qpos, scale: float | None = None, rows=None,
@@ -159,12 +208,12 @@ def attention(q, k, v, qpos, scale: float | None = None, rows=None,
 # the path, step by step
 # --------------------------------------------------------------------------
 def prep(x_bits, pos, qk_norm: bool, eps: float = 1e-6, base: float = 10000.0,
-         interleaved: bool = False) -> np.ndarray:
+         interleaved: bool = False, scaling: RopeScaling | None = None) -> np.ndarray:
     """RoPE(RMSNorm?(x)) for x [B, T, H, D] bf16 bits at positions pos [B, T]."""
     x = widen(x_bits)
     if qk_norm:
         x = rmsnorm(x, eps)
-    return rope(x, pos, base, interleaved)
+    return rope(x, pos, base, interleaved, scaling)
 
 
 def positions(pos0, B: int, T: int) -> np.ndarray:
@@ -174,15 +223,15 @@ def positions(pos0, B: int, T: int) -> np.ndarray:
 
 
 def rope_apply(q_bits, pos0, qk_norm: bool, eps: float = 1e-6,
-               base: float = 10000.0) -> np.ndarray:
+               base: float = 10000.0, scaling: RopeScaling | None = None) -> np.ndarray:
     """What gqa_rope_apply computes: q [B, T, H, D] rotated at pos0[b] + t."""
     B, T = q_bits.shape[:2]
-    return prep(q_bits, positions(pos0, B, T), qk_norm, eps, base)
+    return prep(q_bits, positions(pos0, B, T), qk_norm, eps, base, scaling=scaling)
 
 
 def prefill(q_bits, k_bits, v_bits, qk_norm: bool, eps: float = 1e-6,
             base: float = 10000.0, scale: float | None = None, rows=None,
-            nthreads: int = 0):
+            nthreads: int = 0, scaling: RopeScaling | None = None):
     """Prompt prefill from position 0.
 
     Returns (o [B, T, Hq, D], k_rot [B, T, Hkv, D], v [B, T, Hkv, D]) in float64:
@@ -190,8 +239,8 @@ def prefill(q_bits, k_bits, v_bits, qk_norm: bool, eps: float = 1e-6,
     """
     B, T = q_bits.shape[:2]
     pos = positions(0, B, T)
-    q = prep(q_bits, pos, qk_norm, eps, base)
-    k = prep(k_bits, pos, qk_norm, eps, base)
+    q = prep(q_bits, pos, qk_norm, eps, base, scaling=scaling)
+    k = prep(k_bits, pos, qk_norm, eps, base, scaling=scaling)
     v = widen(v_bits)
     o = attention(q, k, v, pos, scale, rows, nthreads)
     return o, k, v

@@ -84,9 +84,11 @@ void oracle_rmsnorm(const double *x, double *y, int64_t rows, int D, double eps)
  * pairing) or (2i, 2i + 1) when interleaved != 0; the rotation is
  *   x_a' = x_a cos(p th_i) - x_b sin(p th_i)
  *   x_b' = x_a sin(p th_i) + x_b cos(p th_i).
+ * oracle_rope_theta takes the table th_i (the context-extension variants change
+ * only the table); oracle_rope builds the plain one, th_i = base^(-2i/D).
  */
-void oracle_rope(const double *x, double *y, const int64_t *pos, int64_t N, int H,
-                 int D, double base, int interleaved)
+void oracle_rope_theta(const double *x, double *y, const int64_t *pos, int64_t N, int H,
+                       int D, const double *theta, int interleaved)
 {
     int half = D / 2;
     for (int64_t n = 0; n < N; ++n) {
@@ -95,8 +97,7 @@ void oracle_rope(const double *x, double *y, const int64_t *pos, int64_t N, int 
             const double *xr = x + (n * H + h) * D;
             double *yr = y + (n * H + h) * D;
             for (int i = 0; i < half; ++i) {
-                double theta = pow(base, -2.0 * (double)i / (double)D);
-                double ang = p * theta;
+                double ang = p * theta[i];
                 double c = cos(ang), s = sin(ang);
                 int ia = interleaved ? 2 * i : i;
                 int ib = interleaved ? 2 * i + 1 : i + half;
@@ -106,6 +107,18 @@ void oracle_rope(const double *x, double *y, const int64_t *pos, int64_t N, int 
             }
         }
     }
+}
+
+/* Plain RoPE: the table theta_i = base^(-2i/D). */
+void oracle_rope(const double *x, double *y, const int64_t *pos, int64_t N, int H,
+                 int D, double base, int interleaved)
+{
+    int half = D / 2;
+    double *theta = (double *)malloc(sizeof(double) * (size_t)(half > 0 ? half : 1));
+    for (int i = 0; i < half; ++i)
+        theta[i] = pow(base, -2.0 * (double)i / (double)D);
+    oracle_rope_theta(x, y, pos, N, H, D, theta, interleaved);
+    free(theta);
 }
 
 /* One output row: softmax over visible keys, then the weighted sum of values. */

@@ -28,7 +28,25 @@ _vp, _i, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_
 
 class RopeParams(ctypes.Structure):
     _fields_ = [("qk_norm", ctypes.c_int), ("eps", ctypes.c_float),
-                ("rope_base", ctypes.c_float)]
+                ("rope_base", ctypes.c_float), ("scaling", ctypes.c_int),
+                ("factor", ctypes.c_float), ("original_max_pos", ctypes.c_int),
+                ("yarn_alpha", ctypes.c_float), ("yarn_beta", ctypes.c_float)]
+
+
+ROPE_KINDS = {"plain": 0, "linear": 1, "ntk": 2, "yarn": 3}
+
+
+class RopeScaling:
+    """A RoPE context-extension variant (see gqa.h): kind 'linear', 'ntk' or
+    'yarn', the extension factor s >= 1 and, for YaRN, the trained context
+    length and the ramp bounds alpha < beta."""
+
+    def __init__(self, kind: str, factor: float, original_max_pos: int = 0,
+                 alpha: float = 1.0, beta: float = 32.0):
+        if kind not in ROPE_KINDS:
+            raise ValueError("unknown RoPE scaling %r" % kind)
+        self.kind, self.factor = kind, float(factor)
+        self.original_max_pos, self.alpha, self.beta = int(original_max_pos), float(alpha), float(beta)
 
 
 SIGNATURES = {
@@ -104,26 +122,32 @@ def _need(t, name, dtype, ndim=None):
         raise ValueError("%s must have %d dims, got %s" % (name, ndim, tuple(t.shape)))
 
 
-def _params(qk_norm, eps, rope_base):
-    return RopeParams(1 if qk_norm else 0, float(eps), float(rope_base))
+def _params(qk_norm, eps, rope_base, scaling=None):
+    if scaling is None:
+        return RopeParams(1 if qk_norm else 0, float(eps), float(rope_base))
+    return RopeParams(1 if qk_norm else 0, float(eps), float(rope_base), ROPE_KINDS[scaling.kind],
+                      scaling.factor, scaling.original_max_pos, scaling.alpha, scaling.beta)
 
 
 # ---------------------------------------------------------------------------
 # entry points (same names as the C ABI)
 # ---------------------------------------------------------------------------
-def gqa_rope_apply(q, pos0=None, qk_norm=False, eps=1e-6, rope_base=10000.0, stream=None):
+def gqa_rope_apply(q, pos0=None, qk_norm=False, eps=1e-6, rope_base=10000.0, stream=None,
+                   scaling=None):
     """In place: q [B, T, H, D] <- RoPE(RMSNorm?(q)) at positions pos0[b] + t."""
     _need(q, "q", torch.bfloat16, 4)
     if pos0 is not None:
         _need(pos0, "pos0", torch.int32, 1)
     B, T, H, D = q.shape
     _check("gqa_rope_apply", load().gqa_rope_apply(
-        _ptr(q), _ptr(pos0), B, T, H, D, _params(qk_norm, eps, rope_base), _stream(stream)))
+        _ptr(q), _ptr(pos0), B, T, H, D, _params(qk_norm, eps, rope_base, scaling),
+        _stream(stream)))
     return q
 
 
 def kv_cache_append(k, v, k_cache, v_cache, pos0=None, max_pos0=-1, new_len=None,
-                    qk_norm=False, eps=1e-6, rope_base=10000.0, status=None, stream=None):
+                    qk_norm=False, eps=1e-6, rope_base=10000.0, status=None, stream=None,
+                    scaling=None):
     """Write RoPE(RMSNorm?(k)) and v of the new tokens [B, T, Hkv, D] into the caches."""
     _need(k, "k", torch.bfloat16, 4)
     _need(v, "v", torch.bfloat16, 4)
@@ -138,12 +162,13 @@ def kv_cache_append(k, v, k_cache, v_cache, pos0=None, max_pos0=-1, new_len=None
             _need(t, name, torch.int32)
     _check("kv_cache_append", load().kv_cache_append(
         _ptr(k), _ptr(v), _ptr(k_cache), _ptr(v_cache), _ptr(pos0), int(max_pos0),
-        _ptr(new_len), B, T, Hkv, D, k_cache.shape[2], _params(qk_norm, eps, rope_base),
+        _ptr(new_len), B, T, Hkv, D, k_cache.shape[2], _params(qk_norm, eps, rope_base, scaling),
         _ptr(status), _stream(stream)))
 
 
 def gqa_rope_append(q, k, v, k_cache, v_cache, pos0=None, max_pos0=-1, new_len=None,
-                    qk_norm=False, eps=1e-6, rope_base=10000.0, status=None, stream=None):
+                    qk_norm=False, eps=1e-6, rope_base=10000.0, status=None, stream=None,
+                    scaling=None):
     """gqa_rope_apply on q and kv_cache_append of k, v in one launch."""
     _need(q, "q", torch.bfloat16)
     _need(k, "k", torch.bfloat16)
@@ -164,7 +189,7 @@ def gqa_rope_append(q, k, v, k_cache, v_cache, pos0=None, max_pos0=-1, new_len=N
             _need(t, name, torch.int32)
     _check("gqa_rope_append", load().gqa_rope_append(
         _ptr(q), _ptr(k), _ptr(v), _ptr(k_cache), _ptr(v_cache), _ptr(pos0), int(max_pos0),
-        _ptr(new_len), B, T, Hq, Hkv, D, k_cache.shape[2], _params(qk_norm, eps, rope_base),
+        _ptr(new_len), B, T, Hq, Hkv, D, k_cache.shape[2], _params(qk_norm, eps, rope_base, scaling),
         _ptr(status), _stream(stream)))
 
 

@@ -14,4 +14,4 @@ extern "C" const char *gqa_status_string(gqa_status s) {
     return "unknown status";
 }
 
-extern "C" int gqa_version(void) { return 100; }
+extern "C" int gqa_version(void) { return 200; }

@@ -7,14 +7,19 @@
 //
 // One CTA per block of 4 consecutive tokens of a sequence (1 token in decode).
 // The CTA issues the loads of its first head vectors, then turns each token's
-// position into the D/2 rotation angles (float64 angle p * base^(-2i/D) reduced
-// to [-pi, pi] in float64, cos/sin in fp32) in shared memory, shared by all of
-// the token's heads.  Each head vector
+// position into the D/2 rotation angles (float64 angle p * theta_i reduced to
+// [-pi, pi] in float64, cos/sin in fp32) in shared memory, shared by all of the
+// token's heads.  The float64 table theta_i -- base^(-2i/D), or one of the
+// context-extension variants (linear interpolation, NTK-aware, YaRN, see
+// gqa.h) -- is computed once per call on the host and passed as a kernel
+// parameter, together with YaRN's scale of the rotated vectors.  Each head vector
 // is then owned by TPV threads: thread j holds the 16-byte chunk j of the first
 // half (coordinates 8j..8j+7) and the matching chunk of the second half
 // (coordinates D/2+8j..), i.e. exactly the 8 rotation pairs it needs, so every
 // global access is a coalesced 16-byte vector and no data crosses threads except
 // the RMSNorm sum of squares (an xor-shuffle within the TPV-lane group).
+#include <cmath>
+
 #include "common.cuh"
 
 namespace gqa {
@@ -22,6 +27,13 @@ namespace gqa {
 namespace {
 
 constexpr int kThreads = 256;
+
+// Rotation frequencies theta_i of the D/2 pairs (float64) and the factor the
+// rotated vectors are multiplied by (1 except for YaRN).
+struct RopeTable {
+    double theta[64];
+    float mscale;
+};
 
 template <int D>
 struct RopeShape {
@@ -102,11 +114,11 @@ rope_append_kernel(uint16_t *__restrict__ q, const uint16_t *__restrict__ k,
                    const uint16_t *__restrict__ v, uint16_t *__restrict__ kc,
                    uint16_t *__restrict__ vc, const int32_t *__restrict__ pos0,
                    int32_t *__restrict__ new_len, int T, int Hq, int Hkv, int Lmax,
-                   int qk_norm, float eps, float base, int32_t *status) {
+                   int qk_norm, float eps, const __grid_constant__ RopeTable tab,
+                   int32_t *status) {
     using S = RopeShape<D>;
     __shared__ float cs[TB][S::kHalf];
     __shared__ float sn[TB][S::kHalf];
-    __shared__ double theta_d[S::kHalf];
     // A kernel launched after this one as a programmatic dependent (the prefill
     // or the decode) may start its prologue now; it waits for this grid to
     // complete before it reads anything written here.
@@ -185,20 +197,17 @@ rope_append_kernel(uint16_t *__restrict__ q, const uint16_t *__restrict__ k,
             }
         }
         if (pb == 0) {
-            // Angle p * base^(-2i/D) in float64, reduced to [-pi, pi] in float64
+            // Angle p * theta_i in float64, reduced to [-pi, pi] in float64
             // (subtracting the nearest multiple of 2*pi), then sin/cos in fp32.
-            for (int i = threadIdx.x; i < S::kHalf; i += kThreads)
-                theta_d[i] = pow((double)base, -2.0 * (double)i / (double)D);
-            __syncthreads();
             for (int i = threadIdx.x; i < TB * S::kHalf; i += kThreads) {
                 const int tl = i / S::kHalf, pi = i - tl * S::kHalf;
-                const double a = (double)(p0 + t0 + tl) * theta_d[pi];
+                const double a = (double)(p0 + t0 + tl) * tab.theta[pi];
                 const double two_pi = 6.283185307179586476925286766559;
                 const double r = a - rint(a * (1.0 / two_pi)) * two_pi;
                 float sf, cf;
                 sincosf((float)r, &sf, &cf);
-                cs[tl][pi] = cf;
-                sn[tl][pi] = sf;
+                cs[tl][pi] = cf * tab.mscale;
+                sn[tl][pi] = sf * tab.mscale;
             }
             __syncthreads();
         }
@@ -229,6 +238,32 @@ rope_append_kernel(uint16_t *__restrict__ q, const uint16_t *__restrict__ k,
     }
 }
 
+// theta_i for the chosen variant, in float64 on the host (formulas in gqa.h).
+RopeTable make_table(int D, const gqa_rope_params &p) {
+    RopeTable t;
+    const int half = D / 2;
+    const double base = (double)p.rope_base, s = (double)p.factor;
+    const double two_pi = 6.283185307179586476925286766559;
+    double eff_base = base;
+    if (p.scaling == GQA_ROPE_NTK) eff_base = base * std::pow(s, (double)D / (double)(D - 2));
+    for (int i = 0; i < 64; ++i) t.theta[i] = 0.0;
+    for (int i = 0; i < half; ++i) {
+        const double th = std::pow(eff_base, -2.0 * (double)i / (double)D);
+        double out = th;
+        if (p.scaling == GQA_ROPE_LINEAR) {
+            out = th / s;
+        } else if (p.scaling == GQA_ROPE_YARN) {
+            const double r = (double)p.original_max_pos * th / two_pi;
+            double gmix = (r - (double)p.yarn_alpha) / ((double)p.yarn_beta - (double)p.yarn_alpha);
+            gmix = gmix < 0.0 ? 0.0 : (gmix > 1.0 ? 1.0 : gmix);
+            out = (1.0 - gmix) * th / s + gmix * th;
+        }
+        t.theta[i] = out;
+    }
+    t.mscale = p.scaling == GQA_ROPE_YARN ? (float)(0.1 * std::log(s) + 1.0) : 1.0f;
+    return t;
+}
+
 template <int D, int TB>
 cudaError_t launch(void *q, const void *k, const void *v, void *kc, void *vc,
                    const int32_t *pos0, int32_t *new_len, int B, int T, int Hq, int Hkv,
@@ -238,7 +273,7 @@ cudaError_t launch(void *q, const void *k, const void *v, void *kc, void *vc,
         static_cast<uint16_t *>(q), static_cast<const uint16_t *>(k),
         static_cast<const uint16_t *>(v), static_cast<uint16_t *>(kc),
         static_cast<uint16_t *>(vc), pos0, new_len, T, Hq, Hkv, Lmax, p.qk_norm, p.eps,
-        p.rope_base, status);
+        make_table(D, p), status);
     return cudaGetLastError();
 }
 
@@ -269,7 +304,16 @@ gqa_status dispatch(void *q, const void *k, const void *v, void *kc, void *vc,
 }
 
 bool params_ok(const gqa_rope_params &p) {
-    return p.eps >= 0.f && p.rope_base > 1.f;
+    if (!(p.eps >= 0.f && p.rope_base > 1.f)) return false;
+    switch (p.scaling) {
+        case GQA_ROPE_PLAIN: return true;
+        case GQA_ROPE_LINEAR:
+        case GQA_ROPE_NTK: return p.factor >= 1.f;
+        case GQA_ROPE_YARN:
+            return p.factor >= 1.f && p.original_max_pos >= 1 && p.yarn_alpha >= 0.f &&
+                   p.yarn_beta > p.yarn_alpha;
+        default: return false;
+    }
 }
 
 }  // namespace

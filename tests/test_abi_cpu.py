@@ -76,6 +76,19 @@ def test_rope_apply_validation(lib):
     assert lib.gqa_rope_apply(FAKE, None, 1, 1, 1, 64, bad, None) == 1
 
 
+def test_rope_scaling_validation(lib):
+    f = FAKE
+    def params(kind, factor=2.0, L=2048, alpha=1.0, beta=32.0):
+        return _lib.RopeParams(0, 1e-6, 10000.0, kind, factor, L, alpha, beta)
+    assert lib.gqa_rope_apply(f, None, 1, 1, 1, 64, params(9), None) == 1          # unknown kind
+    assert lib.gqa_rope_apply(f, None, 1, 1, 1, 64, params(1, 0.5), None) == 1     # factor < 1
+    assert lib.gqa_rope_apply(f, None, 1, 1, 1, 64, params(2, 0.9), None) == 1
+    assert lib.gqa_rope_apply(f, None, 1, 1, 1, 64, params(3, L=0), None) == 1     # no trained length
+    assert lib.gqa_rope_apply(f, None, 1, 1, 1, 64, params(3, alpha=32.0, beta=1.0), None) == 1
+    assert lib.kv_cache_append(f, f, f, f, None, 0, None, 1, 16, 2, 64, 128, params(3, 0.5),
+                               None, None) == 1
+
+
 def test_append_validation(lib):
     f = FAKE
     # capacity known on the host: max_pos0 + T > Lmax

@@ -364,3 +364,88 @@ def test_chunk_of_one_token_is_a_decode_step():
     o_chk, k_chk = oracle.prefill_chunk(q[:, None], k[:, None], v[:, None], kc, vc, lens, True)
     np.testing.assert_array_equal(o_chk[:, 0], o_dec)
     np.testing.assert_array_equal(k_chk[:, 0], k_dec)
+
+
+# ---------------------------------------------------------------------------
+# RoPE context-extension variants (linear interpolation, NTK-aware, YaRN)
+# ---------------------------------------------------------------------------
+def test_theta_table_path_reproduces_plain_rope():
+    rng = np.random.default_rng(20)
+    x = rng.standard_normal((5, 3, 64))
+    pos = np.array([0, 1, 7, 100, 4095])
+    plain = oracle.rope(x, pos)
+    class Plain(oracle.RopeScaling):        # the plain table through the table path
+        def theta(self, D, base):
+            return base ** (-2.0 * np.arange(D // 2) / D)
+    # numpy's power and C's pow may round theta differently by an ulp, which the
+    # position multiplies: allow |p| * 2^-52 on top of the rotation's rounding
+    np.testing.assert_allclose(oracle.rope(x, pos, scaling=Plain("linear", 1.0)), plain,
+                               rtol=0, atol=4e-16 * pos.max() + 1e-15)
+
+
+@pytest.mark.parametrize("kind", ["linear", "ntk", "yarn"])
+def test_scaling_with_factor_one_is_plain_rope(kind):
+    rng = np.random.default_rng(21)
+    x = rng.standard_normal((4, 2, 128))
+    pos = np.array([3, 64, 1000, 9000])
+    sc = oracle.RopeScaling(kind, 1.0, original_max_pos=2048)
+    np.testing.assert_allclose(oracle.rope(x, pos, scaling=sc), oracle.rope(x, pos),
+                               rtol=0, atol=4e-16 * pos.max() + 1e-15)
+
+
+def test_linear_interpolation_closed_form():
+    """Position interpolation by s: position s*m rotates like position m."""
+    rng = np.random.default_rng(22)
+    x = rng.standard_normal((6, 2, 96))
+    m = np.array([0, 1, 5, 77, 512, 2047])
+    s = 4
+    got = oracle.rope(x, s * m, scaling=oracle.RopeScaling("linear", s))
+    np.testing.assert_allclose(got, oracle.rope(x, m), rtol=0, atol=1e-11)
+
+
+def test_ntk_is_plain_rope_with_the_larger_base():
+    rng = np.random.default_rng(23)
+    D, s, base = 64, 8.0, 10000.0
+    x = rng.standard_normal((5, 2, D))
+    pos = np.array([0, 9, 300, 5000, 30000])
+    got = oracle.rope(x, pos, base, scaling=oracle.RopeScaling("ntk", s))
+    np.testing.assert_allclose(got, oracle.rope(x, pos, base * s ** (D / (D - 2))),
+                               rtol=0, atol=1e-10)
+    th = oracle.RopeScaling("ntk", s).theta(D, base)
+    # the fastest pair keeps its frequency; the slowest is divided by exactly s
+    assert th[0] == 1.0
+    np.testing.assert_allclose(th[-1], base ** (-(D - 2) / D) / s, rtol=1e-13)
+
+
+def test_yarn_limits_and_temperature():
+    D, s, base, L = 128, 8.0, 10000.0, 4096
+    sc = oracle.RopeScaling("yarn", s, original_max_pos=L, alpha=1.0, beta=32.0)
+    plain = base ** (-2.0 * np.arange(D // 2) / D)
+    turns = L * plain / (2 * math.pi)
+    th = sc.theta(D, base)
+    fast, slow = turns >= 32.0, turns <= 1.0
+    assert fast.any() and slow.any() and (~fast & ~slow).any()
+    np.testing.assert_allclose(th[fast], plain[fast], rtol=1e-15)        # kept
+    np.testing.assert_allclose(th[slow], plain[slow] / s, rtol=1e-15)    # interpolated
+    mid = ~fast & ~slow                                                   # in between
+    assert ((th[mid] < plain[mid]) & (th[mid] > plain[mid] / s)).all()
+    rng = np.random.default_rng(24)
+    x = rng.standard_normal((3, 4, D))
+    y = oracle.rope(x, np.array([0, 17, 40000]), base, scaling=sc)
+    mscale = 0.1 * math.log(s) + 1.0
+    np.testing.assert_allclose(np.linalg.norm(y, axis=-1), mscale * np.linalg.norm(x, axis=-1),
+                               rtol=1e-13)
+
+
+@pytest.mark.parametrize("kind", ["linear", "ntk", "yarn"])
+def test_scaled_scores_depend_on_distance_only(kind):
+    rng = np.random.default_rng(25)
+    D = 64
+    sc = oracle.RopeScaling(kind, 4.0, original_max_pos=1024)
+    qv, kv = rng.standard_normal((1, 1, D)), rng.standard_normal((1, 1, D))
+    def score(m, n):
+        return float((oracle.rope(qv, np.array([m]), scaling=sc) *
+                      oracle.rope(kv, np.array([n]), scaling=sc)).sum())
+    for m, n in [(10, 3), (700, 5), (40, 40)]:
+        for shift in (1, 333, 20000):
+            assert abs(score(m + shift, n + shift) - score(m, n)) < 1e-9
