@@ -176,6 +176,31 @@ gqa_status gqa_prefill_chunk(const void *q, const void *k_cache, const void *v_c
                              int Lmax, float scale, int32_t *status_dev, void *stream);
 
 /*
+ * gqa_doc_start -- for packed documents: doc_start[b, t] = the first position
+ * t' <= t of token t's document, from per-token document ids doc_id [B, T]
+ * that do not decrease along a sequence (each document contiguous).  A decrease
+ * raises GQA_DEV_BAD_LEN.  Both arrays device int32, 4-byte aligned.
+ */
+gqa_status gqa_doc_start(const int32_t *doc_id, int32_t *doc_start, int B, int T,
+                         int32_t *status_dev, void *stream);
+
+/*
+ * gqa_prefill_docs -- causal attention of a prompt of packed documents: query t
+ * sees only the keys of its own document,
+ *     out[b, t, h, :] = sum_{doc_start[b,t] <= s <= t} softmax_s(q . K[b, h/g, s] * scale)
+ *                                                      * V[b, h/g, s]
+ * the document-boundary mask of page "训练3.8B LLM…" (section "无效的方法", flex
+ * attention with per-token document ids).  doc_start from gqa_doc_start (non-
+ * decreasing along each sequence, doc_start[b, t] <= t; a value outside 0 .. t
+ * raises GQA_DEV_BAD_LEN and the row attends to itself only).  Key tiles that
+ * lie wholly before a query tile's first document are skipped.  Otherwise as
+ * gqa_prefill (positions from 0, caches filled by gqa_rope_append).
+ */
+gqa_status gqa_prefill_docs(const void *q, const void *k_cache, const void *v_cache,
+                            void *out, const int32_t *doc_start, int B, int T, int Hq, int Hkv,
+                            int D, int Lmax, float scale, int32_t *status_dev, void *stream);
+
+/*
  * gqa_decode -- one query token per sequence against the cache:
  *     out[b, h, :] = sum_{s < lens[b]} softmax_s(q[b,h,:] . K[b, h/g, s, :] * scale)
  *                                      * V[b, h/g, s, :]

@@ -18,6 +18,9 @@ steps together in the order the pages give them:
   section "V3：扩容与推理优化"; a continuation chunk does the same for T tokens
   at once, token t at position ``pos0[b] + t`` seeing the cache and the chunk's
   earlier tokens (the same section, taken a chunk at a time).
+* packed documents (``doc_id``): a query sees only the earlier keys of its own
+  document -- page "训练3.8B LLM…", section "无效的方法" (document-boundary
+  masking with flex attention).
 
 Inputs are bfloat16 bit patterns (``numpy.uint16``), widened exactly to float64.
 """
@@ -75,6 +78,12 @@ def _load():
                                          ctypes.c_double, _i64p, ctypes.c_int64,
                                          ctypes.c_int]
         lib.oracle_attention.restype = ctypes.c_int
+        lib.oracle_attention_docs.argtypes = [_f64p, _f64p, _f64p, _i64p, _i64p, _i64p, _f64p,
+                                              ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                              ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                              ctypes.c_double, _i64p, ctypes.c_int64,
+                                              ctypes.c_int]
+        lib.oracle_attention_docs.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -176,12 +185,14 @@ def rope(x, pos, base: float = 10000.0, interleaved: bool = False,
 
 
 def attention(q, k, v, qpos, scale: float | None = None, rows=None,
-              nthreads: int = 0) -> np.ndarray:
+              nthreads: int = 0, qdoc=None, kdoc=None) -> np.ndarray:
     """Causal GQA attention.
 
     q [B, Tq, Hq, D]; k, v [B, Tk, Hkv, D]; qpos [B, Tq] = absolute position of
     each query (keys 0..qpos are visible).  ``rows`` optionally lists flat
     (b, t, h) row indices, r = (b*Tq + t)*Hq + h; other output rows stay NaN.
+    qdoc [B, Tq] / kdoc [B, Tk]: document ids; a key is then visible only inside
+    the query's own document.
     """
     q, k, v = _f64(q), _f64(k), _f64(v)
     B, Tq, Hq, D = q.shape
@@ -196,9 +207,17 @@ def attention(q, k, v, qpos, scale: float | None = None, rows=None,
     else:
         rows = np.ascontiguousarray(rows, dtype=np.int64)
         rp, nr = _ptr(rows, _i64p), rows.size
-    rc = _load().oracle_attention(_ptr(q, _f64p), _ptr(k, _f64p), _ptr(v, _f64p),
-                                  _ptr(qpos, _i64p), _ptr(o, _f64p), B, Tq, Tk, Hq,
-                                  Hkv, D, scale, rp, nr, nthreads)
+    if qdoc is None:
+        rc = _load().oracle_attention(_ptr(q, _f64p), _ptr(k, _f64p), _ptr(v, _f64p),
+                                      _ptr(qpos, _i64p), _ptr(o, _f64p), B, Tq, Tk, Hq,
+                                      Hkv, D, scale, rp, nr, nthreads)
+    else:
+        qdoc = np.ascontiguousarray(np.broadcast_to(qdoc, (B, Tq)), dtype=np.int64)
+        kdoc = np.ascontiguousarray(np.broadcast_to(kdoc, (B, Tk)), dtype=np.int64)
+        rc = _load().oracle_attention_docs(_ptr(q, _f64p), _ptr(k, _f64p), _ptr(v, _f64p),
+                                           _ptr(qpos, _i64p), _ptr(qdoc, _i64p),
+                                           _ptr(kdoc, _i64p), _ptr(o, _f64p), B, Tq, Tk, Hq,
+                                           Hkv, D, scale, rp, nr, nthreads)
     if rc != 0:
         raise ValueError("oracle_attention rejected its arguments (Hq %% Hkv != 0?)")
     return o
@@ -231,7 +250,7 @@ def rope_apply(q_bits, pos0, qk_norm: bool, eps: float = 1e-6,
 
 def prefill(q_bits, k_bits, v_bits, qk_norm: bool, eps: float = 1e-6,
             base: float = 10000.0, scale: float | None = None, rows=None,
-            nthreads: int = 0, scaling: RopeScaling | None = None):
+            nthreads: int = 0, scaling: RopeScaling | None = None, doc_id=None):
     """Prompt prefill from position 0.
 
     Returns (o [B, T, Hq, D], k_rot [B, T, Hkv, D], v [B, T, Hkv, D]) in float64:
@@ -242,7 +261,7 @@ def prefill(q_bits, k_bits, v_bits, qk_norm: bool, eps: float = 1e-6,
     q = prep(q_bits, pos, qk_norm, eps, base, scaling=scaling)
     k = prep(k_bits, pos, qk_norm, eps, base, scaling=scaling)
     v = widen(v_bits)
-    o = attention(q, k, v, pos, scale, rows, nthreads)
+    o = attention(q, k, v, pos, scale, rows, nthreads, qdoc=doc_id, kdoc=doc_id)
     return o, k, v
 
 

@@ -121,10 +121,16 @@ void oracle_rope(const double *x, double *y, const int64_t *pos, int64_t N, int 
     free(theta);
 }
 
-/* One output row: softmax over visible keys, then the weighted sum of values. */
+/*
+ * One output row: softmax over visible keys, then the weighted sum of values.
+ * With document ids (qdoc [B, Tq], kdoc [B, Tk]; NULL for none) a key is
+ * visible only if it also belongs to the query's document -- page "训练3.8B
+ * LLM…", section "无效的方法" (masking at document boundaries, flex attention).
+ */
 static void attend_row(const double *q, const double *k, const double *v,
-                       const int64_t *qpos, double *o, int Tq, int Tk, int Hq,
-                       int Hkv, int D, double scale, int64_t r, double *scores)
+                       const int64_t *qpos, const int64_t *qdoc, const int64_t *kdoc,
+                       double *o, int Tq, int Tk, int Hq, int Hkv, int D, double scale,
+                       int64_t r, double *scores)
 {
     int64_t h = r % Hq;
     int64_t bt = r / Hq;
@@ -139,6 +145,10 @@ static void attend_row(const double *q, const double *k, const double *v,
 
     double m = -INFINITY;
     for (int64_t u = 0; u < nvis; ++u) {
+        if (kdoc && kdoc[b * Tk + u] != qdoc[bt]) {
+            scores[u] = -INFINITY;       /* another document: exp gives 0 */
+            continue;
+        }
         const double *kr = k + ((b * Tk + u) * Hkv + kvh) * D;
         double s = 0.0;
         for (int d = 0; d < D; ++d)
@@ -166,12 +176,13 @@ static void attend_row(const double *q, const double *k, const double *v,
 /*
  * Causal GQA attention.  rows == NULL computes every (b, t, h) row; otherwise
  * only the nrows flat row indices listed.  nthreads <= 0 uses the OpenMP default.
+ * qdoc / kdoc: document ids of queries and keys, or NULL (no document mask).
  * Returns 0, or -1 when Hq is not a multiple of Hkv or an allocation fails.
  */
-int oracle_attention(const double *q, const double *k, const double *v,
-                     const int64_t *qpos, double *o, int B, int Tq, int Tk, int Hq,
-                     int Hkv, int D, double scale, const int64_t *rows,
-                     int64_t nrows, int nthreads)
+int oracle_attention_docs(const double *q, const double *k, const double *v,
+                          const int64_t *qpos, const int64_t *qdoc, const int64_t *kdoc,
+                          double *o, int B, int Tq, int Tk, int Hq, int Hkv, int D,
+                          double scale, const int64_t *rows, int64_t nrows, int nthreads)
 {
     if (Hkv <= 0 || Hq % Hkv != 0)
         return -1;
@@ -185,8 +196,17 @@ int oracle_attention(const double *q, const double *k, const double *v,
     for (int64_t i = 0; i < total; ++i) {
         int64_t r = rows ? rows[i] : i;
         double *scores = scratch + per * (size_t)omp_get_thread_num();
-        attend_row(q, k, v, qpos, o, Tq, Tk, Hq, Hkv, D, scale, r, scores);
+        attend_row(q, k, v, qpos, qdoc, kdoc, o, Tq, Tk, Hq, Hkv, D, scale, r, scores);
     }
     free(scratch);
     return 0;
+}
+
+int oracle_attention(const double *q, const double *k, const double *v,
+                     const int64_t *qpos, double *o, int B, int Tq, int Tk, int Hq,
+                     int Hkv, int D, double scale, const int64_t *rows,
+                     int64_t nrows, int nthreads)
+{
+    return oracle_attention_docs(q, k, v, qpos, NULL, NULL, o, B, Tq, Tk, Hq, Hkv, D, scale,
+                                 rows, nrows, nthreads);
 }

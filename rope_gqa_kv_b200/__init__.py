@@ -7,6 +7,6 @@ workload generator used by the tests and the benchmark.
 from . import inputs  # noqa: F401
 from ._lib import (GQA_DEV_BAD_LEN, GQA_DEV_CAPACITY, GQA_DEV_TIMEOUT,  # noqa: F401
                    LIB_PATH, SIGNATURES, GqaError, RopeScaling, decode_workspace, gqa_decode,
-                   gqa_decode_noalloc, gqa_decode_workspace_bytes, gqa_prefill,
-                   gqa_prefill_chunk, gqa_rope_append, gqa_rope_apply, kv_cache_append, load,
-                   status_string)
+                   gqa_decode_noalloc, gqa_decode_workspace_bytes, gqa_doc_start, gqa_prefill,
+                   gqa_prefill_chunk, gqa_prefill_docs, gqa_rope_append, gqa_rope_apply,
+                   kv_cache_append, load, status_string)

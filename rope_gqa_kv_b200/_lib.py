@@ -58,6 +58,8 @@ SIGNATURES = {
     "gqa_prefill": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp, _vp]),
     "gqa_prefill_chunk": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f,
                                _vp, _vp]),
+    "gqa_doc_start": (_i, [_vp, _vp, _i, _i, _vp, _vp]),
+    "gqa_prefill_docs": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp, _vp]),
     "gqa_decode": (_i, [_vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _f, _vp, _sz,
                         _vp, _vp]),
     "gqa_decode_workspace_bytes": (_sz, [_i, _i, _i, _i]),
@@ -240,6 +242,46 @@ def gqa_prefill_chunk(q, k_cache, v_cache, pos0, max_pos0, n_tok=None, out=None,
     _check("gqa_prefill_chunk", load().gqa_prefill_chunk(
         _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(out), _ptr(pos0), _ptr(n_tok),
         int(max_pos0), B, T, Hq, Hkv, D, Lmax, float(scale), _ptr(status), _stream(stream)))
+    return out
+
+
+def gqa_doc_start(doc_id, out=None, status=None, stream=None):
+    """First position of each token's document, from non-decreasing per-token
+    document ids doc_id [B, T] (int32)."""
+    _need(doc_id, "doc_id", torch.int32, 2)
+    B, T = doc_id.shape
+    if out is None:
+        out = torch.empty_like(doc_id)
+    _need(out, "out", torch.int32, 2)
+    if status is not None:
+        _need(status, "status", torch.int32)
+    _check("gqa_doc_start", load().gqa_doc_start(_ptr(doc_id), _ptr(out), B, T, _ptr(status),
+                                                 _stream(stream)))
+    return out
+
+
+def gqa_prefill_docs(q, k_cache, v_cache, doc_start, out=None, scale=0.0, status=None,
+                     stream=None):
+    """Causal attention of a prompt of packed documents: query t sees keys
+    doc_start[b, t] .. t.  q [B, T, Hq, D] -> out."""
+    _need(q, "q", torch.bfloat16, 4)
+    _need(k_cache, "k_cache", torch.bfloat16, 4)
+    _need(v_cache, "v_cache", torch.bfloat16, 4)
+    _need(doc_start, "doc_start", torch.int32, 2)
+    B, T, Hq, D = q.shape
+    Hkv, Lmax = k_cache.shape[1], k_cache.shape[2]
+    if k_cache.shape != (B, Hkv, Lmax, D) or v_cache.shape != k_cache.shape:
+        raise ValueError("cache shape disagrees with q")
+    if doc_start.shape != (B, T):
+        raise ValueError("doc_start must be [B, T]")
+    if out is None:
+        out = torch.empty_like(q)
+    _need(out, "out", torch.bfloat16, 4)
+    if status is not None:
+        _need(status, "status", torch.int32)
+    _check("gqa_prefill_docs", load().gqa_prefill_docs(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(out), _ptr(doc_start), B, T, Hq, Hkv, D, Lmax,
+        float(scale), _ptr(status), _stream(stream)))
     return out
 
 

@@ -30,6 +30,12 @@
 // rescaled when the running maximum grows by more than 2^8 (the stale maximum
 // otherwise keeps p <= 256, exact in the final normalisation).
 //
+// Documents packed into one sequence (page "训练3.8B LLM…", section "无效的方法":
+// masking at document boundaries, flex-attention style): query t sees only keys
+// doc_start[t] .. t.  Each query tile starts at the key tile holding its first
+// row's doc_start, so tiles wholly before a document are never loaded, and the
+// scores below a row's own start are masked.
+//
 // Continuation chunks read the cache up to slot pos0 + n_tok - 1 (the last
 // valid key); slots past it in the item's last key tile may hold anything,
 // NaN included.  Their scores are masked, and before the last P . V product
@@ -96,8 +102,13 @@ __device__ __forceinline__ uint32_t A(const uint64_t &b) { return ptx::smem_addr
 // Work item w of the grid's items: the query-tile pair, head and sequence it
 // covers.  Items are numbered longest first (pairs nearer the end of the
 // chunk see more keys), with the heads of one KV group side by side.
+// Kernel modes: a prompt from position 0, a continuation chunk after a cached
+// prefix, or a prompt of packed documents.
+constexpr int kPrompt = 0, kChunkMode = 1, kDocs = 2;
+
 struct PfItem {
     int b, h, kvh, q0, n0, n1, n_kv;
+    int lo0, lo1;      // first key tile of each query tile (documents; else 0)
     int P, N;          // first position of the chunk, valid new tokens (0: no work)
     int r_valid;       // valid key rows in the last key tile (128: the tile is full)
     bool has1;
@@ -106,31 +117,54 @@ struct PfItem {
 struct PfGrid {
     int n_items, n_pairs, B, T, Hq, Hkv, Lmax;
     const int32_t *pos0, *n_tok;   // chunk positions / token counts (NULL: 0 / T)
+    const int32_t *doc_start;      // [B, T] first position of each token's document
 };
 
-// (pos0[b], n_tok[b]) of a sequence; an invalid pair becomes "no work" (bad set).
-struct PfSeq {
-    int P, N;
-    bool bad;
-};
-template <bool kChunk>
-__device__ __forceinline__ PfSeq pf_seq(const PfGrid &g, int b) {
-    PfSeq q;
-    if constexpr (!kChunk) {
-        q.P = 0;
-        q.N = g.T;
-        q.bad = false;
-        return q;
-    }
-    q.P = g.pos0 ? g.pos0[b] : 0;
-    q.N = g.n_tok ? g.n_tok[b] : g.T;
-    q.bad = q.P < 0 || q.N < 0 || q.N > g.T || (long long)q.P + q.N > g.Lmax;
-    if (q.bad) q.N = 0;
-    return q;
-}
 __device__ __forceinline__ int pf_item_b(int w, int B, int Hq) {
     const int per_pair = Hq * B;
     return (w % per_pair) / Hq;
+}
+__device__ __forceinline__ int pf_item_q0(int w, const PfGrid &g) {
+    return (g.n_pairs - 1 - w / (g.Hq * g.B)) * 256;
+}
+
+// What an item needs from memory: (pos0[b], n_tok[b]) of a chunk -- an invalid
+// pair becomes "no work" (bad set) -- or the document starts of the first rows
+// of its two query tiles.
+struct PfSeq {
+    int P, N;
+    int lo0, lo1;
+    bool bad;
+};
+template <int kMode>
+__device__ __forceinline__ PfSeq pf_seq(const PfGrid &g, int w) {
+    PfSeq q;
+    q.P = 0;
+    q.N = g.T;
+    q.lo0 = q.lo1 = 0;
+    q.bad = false;
+    if constexpr (kMode == kChunkMode) {
+        const int b = pf_item_b(w, g.B, g.Hq);
+        q.P = g.pos0[b];
+        q.N = g.n_tok ? g.n_tok[b] : g.T;
+        q.bad = q.P < 0 || q.N < 0 || q.N > g.T || (long long)q.P + q.N > g.Lmax;
+        if (q.bad) q.N = 0;
+    } else if constexpr (kMode == kDocs) {
+        const int b = pf_item_b(w, g.B, g.Hq);
+        const int q0 = pf_item_q0(w, g);
+        const int32_t *ds = g.doc_start + (size_t)b * g.T;
+        const int s0 = ds[q0];
+        const int s1 = q0 + 128 < g.T ? ds[q0 + 128] : s0;
+        q.lo0 = max(0, min(s0, q0)) / 128;
+        q.lo1 = q0 + 128 < g.T ? max(0, min(s1, q0 + 128)) / 128 : q.lo0;
+    }
+    return q;
+}
+__device__ __forceinline__ PfSeq pf_seq_none() {
+    PfSeq q;
+    q.P = q.N = q.lo0 = q.lo1 = 0;
+    q.bad = false;
+    return q;
 }
 
 __device__ __forceinline__ PfItem pf_item(int w, const PfGrid &g, PfSeq sq) {
@@ -144,6 +178,8 @@ __device__ __forceinline__ PfItem pf_item(int w, const PfGrid &g, PfSeq sq) {
     it.q0 = (g.n_pairs - 1 - pi) * 256;
     it.P = sq.P;
     it.N = sq.N;
+    it.lo0 = sq.lo0;
+    it.lo1 = sq.lo1;
     const bool has0 = it.q0 < it.N;
     it.has1 = it.q0 + 128 < it.N;
     it.n0 = has0 ? (it.P + min(it.N, it.q0 + 128) + 127) / 128 : 0;
@@ -151,10 +187,11 @@ __device__ __forceinline__ PfItem pf_item(int w, const PfGrid &g, PfSeq sq) {
     it.n_kv = it.has1 ? it.n1 : it.n0;
     const int kv_end = it.P + min(it.N, it.q0 + 256);          // keys [0, kv_end) are valid
     it.r_valid = it.n_kv > 0 ? kv_end - 128 * (it.n_kv - 1) : 128;
+    if (it.lo1 < it.lo0) it.lo1 = it.lo0;
     return it;
 }
 
-template <int D, bool kChunk>
+template <int D, int kMode>
 __device__ void producer(const PfMaps &maps, PfSync &sy, uint8_t *smem, const PfGrid &g,
                          int32_t *status) {
     using S = PfShape<D>;
@@ -163,11 +200,11 @@ __device__ void producer(const PfMaps &maps, PfSync &sy, uint8_t *smem, const Pf
     asm volatile("griddepcontrol.wait;" ::: "memory");
     int kc = 0, vc = 0, qc = 0;     // K, V tiles and Q pairs this CTA has loaded
     bool ok = true;
-    PfSeq nxt = blockIdx.x < g.n_items ? pf_seq<kChunk>(g, pf_item_b(blockIdx.x, g.B, g.Hq)) : PfSeq{0, 0, false};
+    PfSeq nxt = blockIdx.x < g.n_items ? pf_seq<kMode>(g, blockIdx.x) : pf_seq_none();
     for (int w = blockIdx.x; w < g.n_items && ok; w += gridDim.x) {
         if (nxt.bad) report(status, nxt.P < 0 || nxt.N < 0 ? GQA_DEV_BAD_LEN : GQA_DEV_CAPACITY);
         const PfItem I = pf_item(w, g, nxt);
-        if (w + (int)gridDim.x < g.n_items) nxt = pf_seq<kChunk>(g, pf_item_b(w + gridDim.x, g.B, g.Hq));
+        if (w + (int)gridDim.x < g.n_items) nxt = pf_seq<kMode>(g, w + gridDim.x);
         if (I.n_kv == 0) continue;
         // The previous item's last S MMA has released the Q tiles.
         ok = ptx::mbar_wait(A(sy.q_empty), (qc & 1) ^ 1);
@@ -180,7 +217,7 @@ __device__ void producer(const PfMaps &maps, PfSync &sy, uint8_t *smem, const Pf
         ++qc;
         // K tiles run ahead of V tiles: S(j) needs K(j) one MMA pair before
         // PV(j) needs V(j), and the K ring is the deeper one.
-        int jk = 0, jv = 0;
+        int jk = I.lo0, jv = I.lo0;
         while (ok && jv < I.n_kv) {
             if (jk < I.n_kv && jk < jv + S::kStagesK) {
                 const int st = kc % S::kStagesK;
@@ -217,7 +254,7 @@ __device__ void producer(const PfMaps &maps, PfSync &sy, uint8_t *smem, const Pf
     }
 }
 
-template <int D, bool kChunk>
+template <int D, int kMode>
 __device__ void mma_issuer(PfSync &sy, uint8_t *smem, uint32_t tmem, const PfGrid &g,
                            int32_t *status) {
     using S = PfShape<D>;
@@ -250,27 +287,30 @@ __device__ void mma_issuer(PfSync &sy, uint8_t *smem, uint32_t tmem, const PfGri
     int kc = 0, vc = 0, qc = 0;     // K, V tiles and Q pairs consumed
     int pc0 = 0, pc1 = 0;           // P hand-overs received from each softmax group
     bool ok = true;
-    PfSeq nxt = blockIdx.x < g.n_items ? pf_seq<kChunk>(g, pf_item_b(blockIdx.x, g.B, g.Hq)) : PfSeq{0, 0, false};
+    PfSeq nxt = blockIdx.x < g.n_items ? pf_seq<kMode>(g, blockIdx.x) : pf_seq_none();
     for (int w = blockIdx.x; w < g.n_items && ok; w += gridDim.x) {
         const PfItem I = pf_item(w, g, nxt);
-        if (w + (int)gridDim.x < g.n_items) nxt = pf_seq<kChunk>(g, pf_item_b(w + gridDim.x, g.B, g.Hq));
+        if (w + (int)gridDim.x < g.n_items) nxt = pf_seq<kMode>(g, w + gridDim.x);
         if (I.n_kv == 0) continue;
-        const int kc0 = kc;
+        const int kc0 = kc;           // K ring index of key tile lo0
         ok = ptx::mbar_wait(A(sy.q_full), qc & 1) &&
              ptx::mbar_wait(A(sy.k_full[kc0 % S::kStagesK]), (kc0 / S::kStagesK) & 1);
         if (!ok) break;
         ++qc;
         ptx::tc_fence_after();
+        // Query tile t covers key tiles [lo_t, n_t): lo_t = 0 except with
+        // documents, where tile 1 may start later than tile 0.
+        const bool t1_first = I.has1 && I.lo1 == I.lo0;
         issue_s(0, kc0 % S::kStagesK);
-        if (I.has1) issue_s(1, kc0 % S::kStagesK);
+        if (t1_first) issue_s(1, kc0 % S::kStagesK);
         ptx::mma_commit(A(sy.k_empty[kc0 % S::kStagesK]));
-        if (I.n_kv == 1) ptx::mma_commit(A(sy.q_empty));   // Q no longer read
-        for (int j = 0; j < I.n_kv && ok; ++j) {
+        if (I.n_kv - I.lo0 == 1) ptx::mma_commit(A(sy.q_empty));   // Q no longer read
+        for (int j = I.lo0; j < I.n_kv && ok; ++j) {
             const int vst = vc % S::kStagesV;
             ok = ptx::mbar_wait(A(sy.v_full[vst]), (vc / S::kStagesV) & 1);
             if (!ok) break;
             const int jn = j + 1;
-            const int kidx = kc0 + jn;
+            const int kidx = kc0 + (jn - I.lo0);
             const int kst = kidx % S::kStagesK;
             bool k_next = false;
             if (j < I.n0) {
@@ -278,7 +318,7 @@ __device__ void mma_issuer(PfSync &sy, uint8_t *smem, uint32_t tmem, const PfGri
                 if (!ok) break;
                 ++pc0;
                 ptx::tc_fence_after();
-                issue_pv(0, vst, j > 0);
+                issue_pv(0, vst, j > I.lo0);
                 if (jn < I.n0) {
                     ok = ptx::mbar_wait(A(sy.k_full[kst]), (kidx / S::kStagesK) & 1);
                     if (!ok) break;
@@ -288,12 +328,12 @@ __device__ void mma_issuer(PfSync &sy, uint8_t *smem, uint32_t tmem, const PfGri
                     ptx::mma_commit(A(sy.o_final[0]));
                 }
             }
-            if (I.has1 && j < I.n1) {
+            if (I.has1 && j >= I.lo1 && j < I.n1) {
                 ok = ptx::mbar_wait(A(sy.p_full[1]), pc1 & 1);
                 if (!ok) break;
                 ++pc1;
                 ptx::tc_fence_after();
-                issue_pv(1, vst, j > 0);
+                issue_pv(1, vst, j > I.lo1);
                 if (jn < I.n1) {
                     if (!k_next) {
                         ok = ptx::mbar_wait(A(sy.k_full[kst]), (kidx / S::kStagesK) & 1);
@@ -304,6 +344,14 @@ __device__ void mma_issuer(PfSync &sy, uint8_t *smem, uint32_t tmem, const PfGri
                 } else {
                     ptx::mma_commit(A(sy.o_final[1]));
                 }
+            } else if (kMode == kDocs && I.has1 && jn == I.lo1) {
+                // tile 1's first scores, on the next key tile
+                if (!k_next) {
+                    ok = ptx::mbar_wait(A(sy.k_full[kst]), (kidx / S::kStagesK) & 1);
+                    if (!ok) break;
+                    k_next = true;
+                }
+                issue_s(1, kst);
             }
             ptx::mma_commit(A(sy.v_empty[vst]));
             ++vc;
@@ -312,7 +360,7 @@ __device__ void mma_issuer(PfSync &sy, uint8_t *smem, uint32_t tmem, const PfGri
                 if (jn == I.n_kv - 1) ptx::mma_commit(A(sy.q_empty));   // last S of the item
             }
         }
-        kc = kc0 + I.n_kv;
+        kc = kc0 + (I.n_kv - I.lo0);
     }
     if (!ok) report(status, GQA_DEV_TIMEOUT);
     // No MMA may still be writing tensor memory when it is released.
@@ -320,7 +368,7 @@ __device__ void mma_issuer(PfSync &sy, uint8_t *smem, uint32_t tmem, const PfGri
     ptx::mbar_wait(A(sy.mma_done), 0);
 }
 
-template <int D, bool kChunk>
+template <int D, int kMode>
 __device__ void softmax_tile(PfSync &sy, uint8_t *smem, uint32_t tmem, int t, const PfGrid &g,
                              float scale_log2, uint16_t *__restrict__ out, int32_t *status) {
     using S = PfShape<D>;
@@ -332,24 +380,36 @@ __device__ void softmax_tile(PfSync &sy, uint8_t *smem, uint32_t tmem, int t, co
     int sc = 0, oc = 0;             // scores and outputs of this tile received
     int vc = 0;                     // V tiles of the items before this one
     bool ok = true;
-    PfSeq nxt = blockIdx.x < g.n_items ? pf_seq<kChunk>(g, pf_item_b(blockIdx.x, g.B, g.Hq)) : PfSeq{0, 0, false};
+    PfSeq nxt = blockIdx.x < g.n_items ? pf_seq<kMode>(g, blockIdx.x) : pf_seq_none();
     for (int w = blockIdx.x; w < g.n_items && ok; w += gridDim.x) {
         const PfItem I = pf_item(w, g, nxt);
-        if (w + (int)gridDim.x < g.n_items) nxt = pf_seq<kChunk>(g, pf_item_b(w + gridDim.x, g.B, g.Hq));
+        if (w + (int)gridDim.x < g.n_items) nxt = pf_seq<kMode>(g, w + gridDim.x);
         const int vc0 = vc;
-        vc += I.n_kv;
+        vc += I.n_kv - I.lo0;
         if (I.n_kv == 0 || (t == 1 && !I.has1)) continue;
         const int q_first = I.q0 + 128 * t;
         const int nt = t == 0 ? I.n0 : I.n1;
+        const int jlo = t == 0 ? I.lo0 : I.lo1;
         const int qrow = q_first + row;
         const int lim0 = I.P + q_first;          // the tile's first row sees keys <= lim0
         const int qlim = I.P + qrow;             // this row sees keys <= qlim
         // the group whose last key tile is the item's last one clears that V tile's
         // rows past the last valid key (continuation chunks only)
-        const bool clears = kChunk && I.r_valid < 128 && nt == I.n_kv &&
+        const bool clears = kMode == kChunkMode && I.r_valid < 128 && nt == I.n_kv &&
                             (t == 0 ? true : I.n0 < I.n_kv);
+        // documents: this row sees keys [dstart, qrow]
+        int dstart = 0;
+        if constexpr (kMode == kDocs) {
+            if (qrow < T) {
+                dstart = g.doc_start[(size_t)I.b * T + qrow];
+                if (dstart < 0 || dstart > qrow) {
+                    report(status, GQA_DEV_BAD_LEN);
+                    dstart = qrow;
+                }
+            }
+        }
         float m = -INFINITY, l = 0.f;
-        for (int j = 0; j < nt; ++j) {
+        for (int j = jlo; j < nt; ++j) {
             ok = __all_sync(0xffffffffu, ptx::mbar_wait(A(sy.s_full[t]), sc & 1));
             if (!ok) break;
             ++sc;
@@ -360,7 +420,14 @@ __device__ void softmax_tile(PfSync &sy, uint8_t *smem, uint32_t tmem, int t, co
             ptx::tmem_wait_ld();
 #define SV(c) __uint_as_float(sv[(c) >> 5][(c) & 31])
             const int key0 = j * 128;
-            if (key0 + 127 > lim0) {
+            if constexpr (kMode == kDocs) {
+                if (key0 < dstart || key0 + 127 > qlim) {
+#pragma unroll
+                    for (int c = 0; c < 128; ++c)
+                        if (key0 + c < dstart || key0 + c > qlim)
+                            sv[c >> 5][c & 31] = __float_as_uint(-INFINITY);
+                }
+            } else if (key0 + 127 > lim0) {
 #pragma unroll
                 for (int c = 0; c < 128; ++c)
                     if (key0 + c > qlim) sv[c >> 5][c & 31] = __float_as_uint(-INFINITY);
@@ -382,7 +449,7 @@ __device__ void softmax_tile(PfSync &sy, uint8_t *smem, uint32_t tmem, int t, co
                 l *= alpha;
                 m = m_new;
             }
-            if (j > 0 && __any_sync(0xffffffffu, resc)) {
+            if (j > jlo && __any_sync(0xffffffffu, resc)) {
 #pragma unroll
                 for (int c = 0; c < D / 32; ++c) {
                     uint32_t o[32];
@@ -395,7 +462,8 @@ __device__ void softmax_tile(PfSync &sy, uint8_t *smem, uint32_t tmem, int t, co
             }
             // p = 2^(s * scale_log2 - m): packed FMA for the exponent argument, the
             // special-function unit for 2^x, four independent partial row sums.
-            const float neg_m = -m;
+            // (with documents a row may see no key yet: m is -inf, its p must be 0)
+            const float neg_m = (kMode == kDocs && m == -INFINITY) ? 0.f : -m;
             float la0 = 0.f, la1 = 0.f, lb0 = 0.f, lb1 = 0.f;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
@@ -470,11 +538,12 @@ __device__ void softmax_tile(PfSync &sy, uint8_t *smem, uint32_t tmem, int t, co
     if (!ok && lane == 0) report(status, GQA_DEV_TIMEOUT);
 }
 
-template <int D, bool kChunk>
+template <int D, int kMode>
 __global__ void __launch_bounds__(kPfThreads, 1)
 prefill_kernel(const __grid_constant__ PfMaps maps, uint16_t *__restrict__ out, int B, int T,
                int Hq, int Hkv, int Lmax, const int32_t *__restrict__ pos0,
-               const int32_t *__restrict__ n_tok, float scale_log2, int n_pairs, int32_t *status) {
+               const int32_t *__restrict__ n_tok, const int32_t *__restrict__ doc_start,
+               float scale_log2, int n_pairs, int32_t *status) {
     using S = PfShape<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -489,6 +558,7 @@ prefill_kernel(const __grid_constant__ PfMaps maps, uint16_t *__restrict__ out, 
     g.Lmax = Lmax;
     g.pos0 = pos0;
     g.n_tok = n_tok;
+    g.doc_start = doc_start;
     g.n_items = n_pairs * Hq * B;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -528,15 +598,15 @@ prefill_kernel(const __grid_constant__ PfMaps maps, uint16_t *__restrict__ out, 
     if (warp >= 8) {
         ptx::regs_dec<kControlRegs>();
         if (warp == kTmaWarp) {
-            if (lane == 0) producer<D, kChunk>(maps, sy, smem, g, status);
+            if (lane == 0) producer<D, kMode>(maps, sy, smem, g, status);
             __syncwarp();
         } else if (warp == kMmaWarp) {
-            if (lane == 0) mma_issuer<D, kChunk>(sy, smem, tmem, g, status);
+            if (lane == 0) mma_issuer<D, kMode>(sy, smem, tmem, g, status);
             __syncwarp();
         }
     } else {
         ptx::regs_inc<kSoftmaxRegs>();
-        softmax_tile<D, kChunk>(sy, smem, tmem, warp >> 2, g, scale_log2, out, status);
+        softmax_tile<D, kMode>(sy, smem, tmem, warp >> 2, g, scale_log2, out, status);
     }
     ptx::tc_fence_before();
     __syncthreads();
@@ -581,7 +651,8 @@ bool encode(CUtensorMap *m, const void *base, int rank, const cuuint64_t *dims,
 template <int D>
 gqa_status launch_prefill(const void *q, const void *kc, const void *vc, void *out, int B, int T,
                           int Hq, int Hkv, int Lmax, const int32_t *pos0, const int32_t *n_tok,
-                          float scale_log2, int32_t *status, cudaStream_t s) {
+                          const int32_t *doc_start, float scale_log2, int32_t *status,
+                          cudaStream_t s) {
     using S = PfShape<D>;
     PfMaps maps;
     {
@@ -603,7 +674,8 @@ gqa_status launch_prefill(const void *q, const void *kc, const void *vc, void *o
         if (!encode(&maps.k, kc, 3, dims, str, box)) return GQA_ERR_CUDA;
         if (!encode(&maps.v, vc, 3, dims, str, box)) return GQA_ERR_CUDA;
     }
-    auto kern = pos0 ? prefill_kernel<D, true> : prefill_kernel<D, false>;
+    auto kern = pos0 ? prefill_kernel<D, kChunkMode>
+                     : (doc_start ? prefill_kernel<D, kDocs> : prefill_kernel<D, kPrompt>);
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kSmem) !=
         cudaSuccess)
         return GQA_ERR_CUDA;
@@ -633,7 +705,7 @@ gqa_status launch_prefill(const void *q, const void *kc, const void *vc, void *o
     cfg.attrs = pdl;
     cfg.numAttrs = 1;
     if (cudaLaunchKernelEx(&cfg, kern, maps, static_cast<uint16_t *>(out), B, T, Hq, Hkv, Lmax,
-                           pos0, n_tok, scale_log2, n_pairs, status) != cudaSuccess)
+                           pos0, n_tok, doc_start, scale_log2, n_pairs, status) != cudaSuccess)
         return GQA_ERR_CUDA;
     return gqa_host::launch_status();
 }
@@ -652,16 +724,17 @@ bool device_is_sm100() {
 namespace {
 
 gqa_status prefill_entry(const void *q, const void *k_cache, const void *v_cache, void *out,
-                         const int32_t *pos0, const int32_t *n_tok, int max_pos0_host, int B,
-                         int T, int Hq, int Hkv, int D, int Lmax, float scale, int32_t *status_dev,
-                         void *stream) {
+                         const int32_t *pos0, const int32_t *n_tok, const int32_t *doc_start,
+                         int max_pos0_host, int B, int T, int Hq, int Hkv, int D, int Lmax,
+                         float scale, int32_t *status_dev, void *stream) {
     using namespace gqa_host;
     if (!q || !k_cache || !v_cache || !out || B < 1 || T < 1 || Hq < 1 || Hkv < 1 || Lmax < 1)
         return GQA_ERR_INVALID_ARG;
     if (Hq % Hkv != 0) return GQA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
         return GQA_ERR_INVALID_ARG;
-    if ((reinterpret_cast<uintptr_t>(pos0) & 3u) || (reinterpret_cast<uintptr_t>(n_tok) & 3u))
+    if ((reinterpret_cast<uintptr_t>(pos0) & 3u) || (reinterpret_cast<uintptr_t>(n_tok) & 3u) ||
+        (reinterpret_cast<uintptr_t>(doc_start) & 3u))
         return GQA_ERR_INVALID_ARG;
     if (!head_dim_ok(D)) return GQA_ERR_UNSUPPORTED;
     if (Lmax % 128 != 0) return GQA_ERR_INVALID_ARG;
@@ -673,9 +746,9 @@ gqa_status prefill_entry(const void *q, const void *k_cache, const void *v_cache
     const float sl2 = sc * 1.4426950408889634f;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     switch (D) {
-        case 64: return gqa::launch_prefill<64>(q, k_cache, v_cache, out, B, T, Hq, Hkv, Lmax, pos0, n_tok, sl2, status_dev, s);
-        case 96: return gqa::launch_prefill<96>(q, k_cache, v_cache, out, B, T, Hq, Hkv, Lmax, pos0, n_tok, sl2, status_dev, s);
-        default: return gqa::launch_prefill<128>(q, k_cache, v_cache, out, B, T, Hq, Hkv, Lmax, pos0, n_tok, sl2, status_dev, s);
+        case 64: return gqa::launch_prefill<64>(q, k_cache, v_cache, out, B, T, Hq, Hkv, Lmax, pos0, n_tok, doc_start, sl2, status_dev, s);
+        case 96: return gqa::launch_prefill<96>(q, k_cache, v_cache, out, B, T, Hq, Hkv, Lmax, pos0, n_tok, doc_start, sl2, status_dev, s);
+        default: return gqa::launch_prefill<128>(q, k_cache, v_cache, out, B, T, Hq, Hkv, Lmax, pos0, n_tok, doc_start, sl2, status_dev, s);
     }
 }
 
@@ -684,8 +757,8 @@ gqa_status prefill_entry(const void *q, const void *k_cache, const void *v_cache
 extern "C" gqa_status gqa_prefill(const void *q, const void *k_cache, const void *v_cache,
                                   void *out, int B, int T, int Hq, int Hkv, int D, int Lmax,
                                   float scale, int32_t *status_dev, void *stream) {
-    return prefill_entry(q, k_cache, v_cache, out, nullptr, nullptr, 0, B, T, Hq, Hkv, D, Lmax,
-                         scale, status_dev, stream);
+    return prefill_entry(q, k_cache, v_cache, out, nullptr, nullptr, nullptr, 0, B, T, Hq, Hkv, D,
+                         Lmax, scale, status_dev, stream);
 }
 
 extern "C" gqa_status gqa_prefill_chunk(const void *q, const void *k_cache, const void *v_cache,
@@ -693,6 +766,54 @@ extern "C" gqa_status gqa_prefill_chunk(const void *q, const void *k_cache, cons
                                         int max_pos0_host, int B, int T, int Hq, int Hkv, int D,
                                         int Lmax, float scale, int32_t *status_dev, void *stream) {
     if (!pos0) return GQA_ERR_INVALID_ARG;
-    return prefill_entry(q, k_cache, v_cache, out, pos0, n_tok, max_pos0_host, B, T, Hq, Hkv, D,
-                         Lmax, scale, status_dev, stream);
+    return prefill_entry(q, k_cache, v_cache, out, pos0, n_tok, nullptr, max_pos0_host, B, T, Hq,
+                         Hkv, D, Lmax, scale, status_dev, stream);
+}
+
+extern "C" gqa_status gqa_prefill_docs(const void *q, const void *k_cache, const void *v_cache,
+                                       void *out, const int32_t *doc_start, int B, int T, int Hq,
+                                       int Hkv, int D, int Lmax, float scale, int32_t *status_dev,
+                                       void *stream) {
+    if (!doc_start) return GQA_ERR_INVALID_ARG;
+    return prefill_entry(q, k_cache, v_cache, out, nullptr, nullptr, doc_start, 0, B, T, Hq, Hkv,
+                         D, Lmax, scale, status_dev, stream);
+}
+
+// ---------------------------------------------------------------------------
+// gqa_doc_start: per-token document ids -> first position of each document
+// ---------------------------------------------------------------------------
+namespace {
+
+// One thread per token: the first index t' <= t whose id equals id[t], by binary
+// search (ids are non-decreasing along a sequence; a decrease is reported).
+__global__ void __launch_bounds__(256)
+doc_start_kernel(const int32_t *__restrict__ doc_id, int32_t *__restrict__ doc_start, int B,
+                 int T, int32_t *status) {
+    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= (long long)B * T) return;
+    const int b = (int)(i / T), t = (int)(i - (long long)b * T);
+    const int32_t *id = doc_id + (size_t)b * T;
+    const int32_t me = id[t];
+    if (t > 0 && id[t - 1] > me) gqa::report(status, GQA_DEV_BAD_LEN);
+    int lo = 0, hi = t;                    // first index in [0, t] with id >= me
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (id[mid] >= me) hi = mid;
+        else lo = mid + 1;
+    }
+    doc_start[i] = lo;
+}
+
+}  // namespace
+
+extern "C" gqa_status gqa_doc_start(const int32_t *doc_id, int32_t *doc_start, int B, int T,
+                                    int32_t *status_dev, void *stream) {
+    if (!doc_id || !doc_start || B < 1 || T < 1) return GQA_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(doc_id) & 3u) || (reinterpret_cast<uintptr_t>(doc_start) & 3u))
+        return GQA_ERR_INVALID_ARG;
+    const long long n = (long long)B * T;
+    if (n > 0x7fffffffLL * 256LL) return GQA_ERR_INVALID_ARG;
+    doc_start_kernel<<<(unsigned)((n + 255) / 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        doc_id, doc_start, B, T, status_dev);
+    return gqa_host::launch_status();
 }

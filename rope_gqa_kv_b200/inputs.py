@@ -141,6 +141,22 @@ def custom(name: str, B: int, Hq: int, Hkv: int, D: int, T: int = 0, decode_step
                     cached_len_range=cached_len_range)
 
 
+def packed_doc_ids(B: int, T: int, mean_len: float, seed: int) -> torch.Tensor:
+    """Document ids [B, T] (int32, non-decreasing along each row) of documents
+    packed back to back, lengths 1 + an exponential draw of the given mean (the
+    last document cut at T): many short documents and a few long ones."""
+    g = torch.Generator().manual_seed(seed)
+    ids = torch.empty(B, T, dtype=torch.int32)
+    for b in range(B):
+        t, d = 0, 0
+        while t < T:
+            n = 1 + int(torch.empty(1).exponential_(1.0 / mean_len, generator=g).item())
+            ids[b, t:t + n] = d
+            t += n
+            d += 1
+    return ids
+
+
 def bits(t: torch.Tensor):
     """bfloat16 tensor -> numpy uint16 bit patterns (for the oracle)."""
     return t.contiguous().view(torch.int16).numpy().view("uint16")

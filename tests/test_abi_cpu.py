@@ -131,6 +131,18 @@ def test_prefill_chunk_validation(lib):
                                  None, None) == 1
 
 
+def test_docs_validation(lib):
+    f = FAKE
+    odd4 = ctypes.c_void_p(0x10002)
+    assert lib.gqa_prefill_docs(f, f, f, f, None, 1, 10, 4, 2, 64, 128, 0.0, None, None) == 1
+    assert lib.gqa_prefill_docs(f, f, f, f, odd4, 1, 10, 4, 2, 64, 128, 0.0, None, None) == 1
+    assert lib.gqa_prefill_docs(f, f, f, f, f, 1, 10, 4, 2, 80, 128, 0.0, None, None) == 2
+    assert lib.gqa_prefill_docs(f, f, f, f, f, 1, 300, 4, 2, 64, 256, 0.0, None, None) == 3
+    assert lib.gqa_doc_start(None, f, 1, 10, None, None) == 1
+    assert lib.gqa_doc_start(f, odd4, 1, 10, None, None) == 1
+    assert lib.gqa_doc_start(f, f, 0, 10, None, None) == 1
+
+
 def test_decode_validation(lib):
     f = FAKE
     ws = ctypes.c_size_t(1 << 20)

@@ -29,6 +29,9 @@ MUTANTS = {
     "softmax_unnormalised": ("double p = scores[u] / l;", "double p = scores[u];"),
     "values_read_from_keys": ("const double *vr = v + ", "const double *vr = k + "),
     "bf16_shift": ("((uint32_t)bits) << 16", "((uint32_t)bits) << 15"),
+    "document_mask_ignored": ("if (kdoc && kdoc[b * Tk + u] != qdoc[bt]) {", "if (0) {"),
+    "document_mask_by_position": ("if (kdoc && kdoc[b * Tk + u] != qdoc[bt]) {",
+                                  "if (kdoc && kdoc[b * Tk + u] != qdoc[b * Tq + u]) {"),
 }
 
 

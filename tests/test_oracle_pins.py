@@ -449,3 +449,37 @@ def test_scaled_scores_depend_on_distance_only(kind):
     for m, n in [(10, 3), (700, 5), (40, 40)]:
         for shift in (1, 333, 20000):
             assert abs(score(m + shift, n + shift) - score(m, n)) < 1e-9
+
+
+# ---------------------------------------------------------------------------
+# document masking (packed documents, a query sees only its own document)
+# ---------------------------------------------------------------------------
+def test_one_document_is_plain_causal_attention():
+    rng = np.random.default_rng(30)
+    B, T, Hq, Hkv, D = 2, 33, 4, 2, 16
+    q, k, v = (_rand_bits(rng, B, T, Hq, D), _rand_bits(rng, B, T, Hkv, D),
+               _rand_bits(rng, B, T, Hkv, D))
+    o1, _, _ = oracle.prefill(q, k, v, True)
+    o2, _, _ = oracle.prefill(q, k, v, True, doc_id=np.full((B, T), 7))
+    np.testing.assert_array_equal(o1, o2)
+
+
+def test_each_document_is_its_own_prefill():
+    """Rows of a packed document equal a prefill of that document alone, started
+    at position 0: the mask removes the other documents, and RoPE's dependence
+    on position differences alone removes the offset."""
+    rng = np.random.default_rng(31)
+    B, T, Hq, Hkv, D = 2, 60, 6, 2, 32
+    q, k, v = (_rand_bits(rng, B, T, Hq, D), _rand_bits(rng, B, T, Hkv, D),
+               _rand_bits(rng, B, T, Hkv, D))
+    bounds = [[0, 1, 17, 40, 60], [0, 31, 60]]      # a one-token document included
+    doc = np.zeros((B, T), dtype=np.int64)
+    for b, cuts in enumerate(bounds):
+        for i in range(len(cuts) - 1):
+            doc[b, cuts[i]:cuts[i + 1]] = i
+    o, _, _ = oracle.prefill(q, k, v, True, doc_id=doc)
+    for b, cuts in enumerate(bounds):
+        for i in range(len(cuts) - 1):
+            a, e = cuts[i], cuts[i + 1]
+            alone, _, _ = oracle.prefill(q[b:b + 1, a:e], k[b:b + 1, a:e], v[b:b + 1, a:e], True)
+            np.testing.assert_allclose(o[b:b + 1, a:e], alone, rtol=0, atol=1e-12)
