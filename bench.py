@@ -378,7 +378,8 @@ def run_ours(args, rank, world, dev, dist_on):
     }
     line["next_rows"] = {"chunked_prefill": measure_chunk(dev, peaks, tag),
                          "rope_scaling": measure_scaled_append(layer, peaks, tag),
-                         "doc_masked_prefill": measure_docs(layer, peaks, tag)}
+                         "doc_masked_prefill": measure_docs(layer, peaks, tag),
+                         "attention_backward": measure_backward(layer, peaks, tag)}
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
     return line
@@ -408,6 +409,47 @@ def measure_scaled_append(layer, peaks, tag, reps: int = 30):
             "frac": round(gbs / peaks["hbm_gbs"], 4), "peak_kind": "hbm copy " + tag,
             "algorithmic_per_launch": append_bytes(),
             "l2": "inputs (335 MB moved per launch) exceed L2"}
+
+
+def measure_backward(layer, peaks, tag, reps: int = 20):
+    """Attention backward (gqa_attention_backward: rowsum(dO * O), dK/dV, dQ), outside
+    the timed step, on the 3.8B-style prompt (8 x 2048, 24/8 heads, D = 128) with a
+    seeded N(0,1) output gradient.  Work is counted the usual way for attention
+    backwards, 2.5 x the forward's causal FLOPs (five products per (query, key,
+    head) instead of two); the kernels recompute S and dP once more for dQ, so
+    they execute 3.5 x.  Each launch follows an L2-evicting write."""
+    import rope_gqa_kv_b200 as gqa
+    g = torch.Generator().manual_seed(4242)
+    dout = torch.randn(tuple(layer.pq.shape), generator=g).to(torch.bfloat16).to(layer.dev)
+    out, lse = gqa.gqa_prefill_lse(layer.pq, layer.pkc, layer.pvc, status=layer.status)
+    dq = torch.empty_like(layer.pq)
+    dk = torch.empty_like(layer.pkc)
+    dv = torch.empty_like(layer.pvc)
+    ws = torch.empty(gqa.gqa_backward_workspace_bytes(PREFILL.B, PREFILL.T, PREFILL.Hq),
+                     dtype=torch.uint8, device=layer.dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=layer.dev)
+    call = lambda: gqa.gqa_attention_backward(layer.pq, layer.pkc, layer.pvc, out, dout, lse,  # noqa: E731
+                                              dq=dq, dk=dk, dv=dv, workspace=ws,
+                                              status=layer.status)
+    for _ in range(3):
+        call()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(reps)]
+    for i in range(reps):
+        flush.fill_(i & 255)
+        ev[i][0].record()
+        call()
+        ev[i][1].record()
+    torch.cuda.synchronize()
+    ms = sorted(a.elapsed_time(b) for a, b in ev)[reps // 2]
+    fl = 2.5 * prefill_flops()
+    tf = fl / (ms * 1e-3) / 1e12
+    return {"workload": "backward of the 8 x 2048 causal prompt, 24q/8kv, D=128",
+            "kernel": "gqa_attention_backward (3 launches)", "bound": "tensor",
+            "us_median": round(ms * 1e3, 2), "achieved": round(tf, 1), "unit": "TFLOP/s",
+            "peak": peaks["bf16_tflops"], "frac": round(tf / peaks["bf16_tflops"], 4),
+            "peak_kind": "bf16 burst " + tag, "algorithmic_per_launch": fl,
+            "l2": "flushed (256 MB write) before each launch"}
 
 
 def measure_docs(layer, peaks, tag, reps: int = 30):

@@ -176,6 +176,43 @@ gqa_status gqa_prefill_chunk(const void *q, const void *k_cache, const void *v_c
                              int Lmax, float scale, int32_t *status_dev, void *stream);
 
 /*
+ * gqa_prefill_lse -- gqa_prefill that also stores each row's log-sum-exp for
+ * the backward: lse[b, h, t] = ln sum_{s <= t} exp(q[b,t,h] . K[b,h/g,s] * scale),
+ * lse float32 [B, Hq, round_up(T, 4)] (16-byte aligned; the padding is not
+ * written).  Otherwise identical to gqa_prefill.
+ */
+gqa_status gqa_prefill_lse(const void *q, const void *k_cache, const void *v_cache, void *out,
+                           float *lse, int B, int T, int Hq, int Hkv, int D, int Lmax,
+                           float scale, int32_t *status_dev, void *stream);
+
+/*
+ * gqa_attention_backward -- gradients of causal GQA attention for training (the
+ * pages' models train through causal scaled_dot_product_attention: page
+ * "训练3.8B LLM…", section "提高吞吐量"; page "Build a Large Language Model from
+ * Scratch", section 3.1).  With P = softmax(q K^T * scale) (causal) per query
+ * head and the incoming gradient dout of out = P V:
+ *     dv = P^T dout,  dP = dout V^T,  dS = P * (dP - rowsum(dout * out)),
+ *     dq = scale dS K,  dk = scale dS^T q,
+ * dk and dv of a KV head summed over the query heads of its group.
+ *   q, out, dout, dq: bf16 [B, T, Hq, D];  k, v, dk, dv: bf16 [B, Hkv, Lmax, D]
+ *     (the cache layout; slots 0 .. T-1 are read / written, the rest of dk, dv
+ *     is not touched);  lse: the forward's, from gqa_prefill_lse.
+ *   ws, ws_bytes: device scratch of gqa_backward_workspace_bytes(B, T, Hq) bytes
+ *     (16-byte aligned; contents on entry do not matter).
+ * Three launches (rowsum(dout * out); dk and dv per key tile; dq per query
+ * tile), each a programmatic dependent of the one before.  Device errors:
+ * GQA_DEV_TIMEOUT.
+ */
+gqa_status gqa_attention_backward(const void *q, const void *k, const void *v, const void *out,
+                                  const void *dout, const float *lse, void *dq, void *dk,
+                                  void *dv, int B, int T, int Hq, int Hkv, int D, int Lmax,
+                                  float scale, void *ws, size_t ws_bytes, int32_t *status_dev,
+                                  void *stream);
+
+/* Bytes of workspace gqa_attention_backward needs (0 on invalid sizes). */
+size_t gqa_backward_workspace_bytes(int B, int T, int Hq);
+
+/*
  * gqa_doc_start -- for packed documents: doc_start[b, t] = the first position
  * t' <= t of token t's document, from per-token document ids doc_id [B, T]
  * that do not decrease along a sequence (each document contiguous).  A decrease

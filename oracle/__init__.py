@@ -21,6 +21,10 @@ steps together in the order the pages give them:
 * packed documents (``doc_id``): a query sees only the earlier keys of its own
   document -- page "训练3.8B LLM…", section "无效的方法" (document-boundary
   masking with flex attention).
+* the backward of causal GQA attention (the pages' models train through the
+  causal scaled_dot_product_attention -- page "训练3.8B LLM…", section
+  "提高吞吐量"; page "Build a Large Language Model from Scratch", section 3.1):
+  the chain rule through softmax written out with numpy matrix products.
 
 Inputs are bfloat16 bit patterns (``numpy.uint16``), widened exactly to float64.
 """
@@ -335,3 +339,52 @@ def decode_step(q_bits, k_bits, v_bits, k_cache_bits, v_cache_bits, lens,
         vals[b, n] = v[b, 0]
     o = attention(q, keys, vals, pos, scale, rows, nthreads)
     return o[:, 0], k[:, 0]
+
+
+# --------------------------------------------------------------------------
+# backward of causal GQA attention
+# --------------------------------------------------------------------------
+def attention_backward(q, k, v, dout, scale: float | None = None, heads=None):
+    """Gradients of L = sum(dout * o) for o = causal GQA attention(q, k, v).
+
+    q, dout [B, T, Hq, D]; k, v [B, T, Hkv, D] (float64 or bf16 bits); every
+    query t sees keys 0..t.  With P = softmax(q k^T * scale) (causal) per query
+    head:  dV = P^T dO,  dP = dO V^T,  dS = P * (dP - rowsum(P * dP)),
+    dQ = scale dS K,  dK = scale dS^T Q, and the K/V gradients of a KV head are
+    the sums over the query heads of its group.  ``heads`` optionally restricts
+    the work to some (b, query head) pairs (the other gradients stay NaN for dq
+    and hold only those heads' contributions for dk / dv).
+    Returns (dq, dk, dv) in float64, plus the forward output o and the row
+    log-sum-exp lse [B, Hq, T] (natural log of sum_s exp(q.k_s * scale)).
+    """
+    q, k, v, do = widen(q), widen(k), widen(v), widen(dout)
+    B, T, Hq, D = q.shape
+    Hkv = k.shape[2]
+    g = Hq // Hkv
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    dq = np.full(q.shape, np.nan)
+    dk = np.zeros(k.shape)
+    dv = np.zeros(v.shape)
+    o = np.full(q.shape, np.nan)
+    lse = np.full((B, Hq, T), np.nan)
+    future = np.triu(np.ones((T, T), dtype=bool), 1)        # key after query
+    pairs = heads if heads is not None else [(b, h) for b in range(B) for h in range(Hq)]
+    for b, h in pairs:
+        kvh = h // g
+        Q, K, V, dO = q[b, :, h], k[b, :, kvh], v[b, :, kvh], do[b, :, h]
+        S = (Q @ K.T) * scale
+        S[future] = -np.inf
+        m = S.max(axis=1, keepdims=True)
+        E = np.exp(S - m)
+        l = E.sum(axis=1, keepdims=True)
+        P = E / l
+        o[b, :, h] = P @ V
+        lse[b, h] = (m + np.log(l))[:, 0]
+        dV = P.T @ dO
+        dP = dO @ V.T
+        dS = P * (dP - (P * dP).sum(axis=1, keepdims=True))
+        dq[b, :, h] = scale * (dS @ K)
+        dk[b, :, kvh] += scale * (dS.T @ Q)
+        dv[b, :, kvh] += dV
+    return dq, dk, dv, o, lse

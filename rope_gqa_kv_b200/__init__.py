@@ -6,7 +6,8 @@ workload generator used by the tests and the benchmark.
 """
 from . import inputs  # noqa: F401
 from ._lib import (GQA_DEV_BAD_LEN, GQA_DEV_CAPACITY, GQA_DEV_TIMEOUT,  # noqa: F401
-                   LIB_PATH, SIGNATURES, GqaError, RopeScaling, decode_workspace, gqa_decode,
+                   LIB_PATH, SIGNATURES, GqaError, RopeScaling, decode_workspace,
+                   gqa_attention_backward, gqa_backward_workspace_bytes, gqa_decode,
                    gqa_decode_noalloc, gqa_decode_workspace_bytes, gqa_doc_start, gqa_prefill,
-                   gqa_prefill_chunk, gqa_prefill_docs, gqa_rope_append, gqa_rope_apply,
-                   kv_cache_append, load, status_string)
+                   gqa_prefill_chunk, gqa_prefill_docs, gqa_prefill_lse, gqa_rope_append,
+                   gqa_rope_apply, kv_cache_append, load, status_string)

@@ -59,6 +59,10 @@ SIGNATURES = {
     "gqa_prefill_chunk": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f,
                                _vp, _vp]),
     "gqa_doc_start": (_i, [_vp, _vp, _i, _i, _vp, _vp]),
+    "gqa_prefill_lse": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp, _vp]),
+    "gqa_attention_backward": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i,
+                                    _i, _i, _f, _vp, _sz, _vp, _vp]),
+    "gqa_backward_workspace_bytes": (_sz, [_i, _i, _i]),
     "gqa_prefill_docs": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp, _vp]),
     "gqa_decode": (_i, [_vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _f, _vp, _sz,
                         _vp, _vp]),
@@ -243,6 +247,68 @@ def gqa_prefill_chunk(q, k_cache, v_cache, pos0, max_pos0, n_tok=None, out=None,
         _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(out), _ptr(pos0), _ptr(n_tok),
         int(max_pos0), B, T, Hq, Hkv, D, Lmax, float(scale), _ptr(status), _stream(stream)))
     return out
+
+
+def gqa_prefill_lse(q, k_cache, v_cache, out=None, lse=None, scale=0.0, status=None,
+                    stream=None):
+    """gqa_prefill that also returns each row's log-sum-exp: (out, lse) with
+    lse float32 [B, Hq, round_up(T, 4)] (the padding columns are not written)."""
+    _need(q, "q", torch.bfloat16, 4)
+    _need(k_cache, "k_cache", torch.bfloat16, 4)
+    _need(v_cache, "v_cache", torch.bfloat16, 4)
+    B, T, Hq, D = q.shape
+    Hkv, Lmax = k_cache.shape[1], k_cache.shape[2]
+    if k_cache.shape != (B, Hkv, Lmax, D) or v_cache.shape != k_cache.shape:
+        raise ValueError("cache shape disagrees with q")
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(B, Hq, (T + 3) // 4 * 4, dtype=torch.float32, device=q.device)
+    _need(out, "out", torch.bfloat16, 4)
+    _need(lse, "lse", torch.float32, 3)
+    if lse.shape != (B, Hq, (T + 3) // 4 * 4):
+        raise ValueError("lse must be [B, Hq, round_up(T, 4)]")
+    if status is not None:
+        _need(status, "status", torch.int32)
+    _check("gqa_prefill_lse", load().gqa_prefill_lse(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(out), _ptr(lse), B, T, Hq, Hkv, D, Lmax,
+        float(scale), _ptr(status), _stream(stream)))
+    return out, lse
+
+
+def gqa_backward_workspace_bytes(B, T, Hq):
+    return int(load().gqa_backward_workspace_bytes(B, T, Hq))
+
+
+def gqa_attention_backward(q, k, v, out, dout, lse, dq=None, dk=None, dv=None, scale=0.0,
+                           workspace=None, status=None, stream=None):
+    """Gradients (dq, dk, dv) of causal GQA attention.  q, out, dout [B, T, Hq, D];
+    k, v [B, Hkv, Lmax, D] (cache layout, slots < T used); lse from gqa_prefill_lse."""
+    for name, t in (("q", q), ("out", out), ("dout", dout)):
+        _need(t, name, torch.bfloat16, 4)
+    _need(k, "k", torch.bfloat16, 4)
+    _need(v, "v", torch.bfloat16, 4)
+    _need(lse, "lse", torch.float32, 3)
+    B, T, Hq, D = q.shape
+    Hkv, Lmax = k.shape[1], k.shape[2]
+    if k.shape != (B, Hkv, Lmax, D) or v.shape != k.shape or out.shape != q.shape or \
+            dout.shape != q.shape:
+        raise ValueError("q/k/v/out/dout shapes disagree")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.zeros_like(k) if dk is None else dk
+    dv = torch.zeros_like(v) if dv is None else dv
+    for name, t in (("dq", dq), ("dk", dk), ("dv", dv)):
+        _need(t, name, torch.bfloat16, 4)
+    if workspace is None:
+        workspace = torch.empty(max(gqa_backward_workspace_bytes(B, T, Hq), 16), dtype=torch.uint8,
+                                device=q.device)
+    if status is not None:
+        _need(status, "status", torch.int32)
+    _check("gqa_attention_backward", load().gqa_attention_backward(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv),
+        B, T, Hq, Hkv, D, Lmax, float(scale), _ptr(workspace), workspace.numel(), _ptr(status),
+        _stream(stream)))
+    return dq, dk, dv
 
 
 def gqa_doc_start(doc_id, out=None, status=None, stream=None):

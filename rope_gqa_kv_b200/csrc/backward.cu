@@ -1,0 +1,778 @@
+// backward.cu -- the backward of causal GQA attention on the tcgen05 tensor cores.
+//
+// The pages' models train through the causal scaled_dot_product_attention
+// (page "训练3.8B LLM至0.384 CORE，成本998美元 – Hugo Vergnes", sections "无效的方法"
+// and "提高吞吐量"; page "Build a Large Language Model from Scratch", section 3.1),
+// with query heads sharing K/V heads in groups (page "750美元从零训练3个LLM：一位
+// 开发者的实战复盘", section "V2：引入前沿技术").  For one query head, with
+// P = softmax(Q K^T * c) (causal, c the softmax scale) and the incoming gradient
+// dO of the output O = P V:
+//     dV = P^T dO,   dP = dO V^T,   dS = P * (dP - Delta),  Delta = rowsum(dO * O),
+//     dQ = c dS K,   dK = c dS^T Q,
+// and the K/V gradients of a KV head sum over the query heads of its group.  P is
+// recomputed from the forward's row log-sum-exp, never stored.
+//
+// Three launches:
+//   delta_kernel   Delta[b, h, t] = sum_d dO * O (HBM-bound, one warp per row);
+//   bwd_kv_kernel  per (b, KV head, 128-key tile j), persistent: for every query
+//                  head of the group and every query tile i >= j,
+//                    S^T = K_j Q_i^T, dP^T = V_j dO_i^T       (two SS MMAs)
+//                    P^T, dS^T in bf16 over S^T, dP^T in TMEM  (4 warps, thread = key)
+//                    dV_j += P^T dO_i, dK_j += dS^T Q_i         (two TS MMAs)
+//                  dK_j and dV_j stay in tensor memory until the tile is done, so
+//                  the group's sum needs no atomics;
+//   bwd_q_kernel   per (b, query head, 128-query tile i), persistent: for every
+//                  key tile j <= i,  S = Q_i K_j^T, dP = dO_i V_j^T, dS in bf16 over
+//                  dP, dQ_i += dS K_j.
+// The same shared-memory tile serves as a K-major operand (the contraction over
+// D) and as an MN-major one (the contraction over its rows), as in the forward
+// kernel.  Warp roles (192 threads): warps 0-3 elementwise + epilogue (thread =
+// TMEM lane), warp 4 TMA producer, warp 5 MMA issuer.  Every mbarrier wait is
+// bounded (1 s) and raises GQA_DEV_TIMEOUT; tensor memory is released only after
+// the MMA thread has seen its last MMA complete.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "ptx.cuh"
+#include "tmap.cuh"
+
+namespace gqa {
+namespace {
+
+constexpr int kBwThreads = 192;
+constexpr int kBwTmaWarp = 4;
+constexpr int kBwMmaWarp = 5;
+constexpr float kLog2e = 1.4426950408889634f;
+
+template <int D>
+struct BwShape {
+    static constexpr int kBlocks = (D + 63) / 64;           // 128-byte column blocks
+    static constexpr int kBlockBytes = 128 * 128;           // 128 rows x 128 bytes
+    static constexpr int kTileBytes = kBlocks * kBlockBytes;
+    static constexpr int kKSteps = D / 16;
+    static constexpr int kVecBytes = 128 * 4;               // 128 fp32 (lse or delta)
+    static constexpr int kStages = 2;
+    // dK/dV kernel: [K_j | V_j | stages of (Q_i | dO_i | lse_i | delta_i)]
+    static constexpr int kStageBytes = 2 * kTileBytes + 2 * kVecBytes;   // multiple of 1024
+    static constexpr int kOffStage = 2 * kTileBytes;
+    static constexpr int kSmemKV = kOffStage + kStages * kStageBytes + 1024;
+    // dQ kernel: [Q_i | dO_i | stages of (K_j | V_j)]
+    static constexpr int kOffKV = 2 * kTileBytes;
+    static constexpr int kSmemQ = kOffKV + kStages * 2 * kTileBytes + 1024;
+    static_assert(kSmemKV <= 227 * 1024 && kSmemQ <= 227 * 1024, "shared memory per CTA");
+    // tensor memory columns: S [0,128) dP [128,256) then the fp32 accumulators
+    static constexpr uint32_t kColS = 0, kColDP = 128, kColAcc0 = 256, kColAcc1 = 384;
+};
+
+struct BwMaps {
+    CUtensorMap q, dout, k, v, lse, delta;
+};
+
+struct BwSync {
+    uint64_t fixed_full, fixed_empty;          // K_j/V_j (dK/dV kernel) or Q_i/dO_i (dQ kernel)
+    uint64_t st_full[2], st_empty[2];          // the ring
+    uint64_t s_full, p_full, acc_full, acc_empty;
+    uint64_t mma_done;
+    uint32_t tmem_base;
+};
+
+struct BwGrid {
+    int B, T, Hq, Hkv, nT, n_items, lse_stride;
+    float scale_log2, scale;
+    const float *lse, *delta;
+    uint16_t *d0, *d1;                          // dK, dV (dK/dV kernel) or dQ (dQ kernel)
+    int Lmax;
+};
+
+__device__ __forceinline__ uint32_t A(const uint64_t &b) { return ptx::smem_addr(&b); }
+
+template <int D>
+struct BwMma {
+    using S = BwShape<D>;
+    // D(tmem) = A(smem, K-major 128 x D) . B(smem, K-major 128 x D)^T : 128 x 128
+    static __device__ __forceinline__ void ss(uint32_t d, uint32_t a, uint32_t b) {
+        constexpr uint32_t id = ptx::idesc_bf16_f32(128, 128, false);
+#pragma unroll
+        for (int ks = 0; ks < S::kKSteps; ++ks) {
+            const uint32_t off = (ks >> 2) * S::kBlockBytes + (ks & 3) * 32;
+            ptx::mma_ss(d, ptx::smem_desc_sw128(a + off, 16, 1024),
+                        ptx::smem_desc_sw128(b + off, 16, 1024), id, ks > 0);
+        }
+    }
+    // D(tmem, 128 x D) (+)= A(tmem, bf16 128 x 128) . B(smem, 128 rows x D, MN-major)
+    static __device__ __forceinline__ void ts(uint32_t d, uint32_t a_tmem, uint32_t b, bool acc) {
+        constexpr uint32_t id = ptx::idesc_bf16_f32(128, D, true);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+            ptx::mma_ts(d, a_tmem + ks * 8, ptx::smem_desc_sw128(b + ks * 2048, S::kBlockBytes, 1024),
+                        id, (acc || ks > 0) ? 1u : 0u);
+    }
+};
+
+// ---------------------------------------------------------------------------
+// Delta = rowsum(dO * O): one warp per (b, t, h) row
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256)
+delta_kernel(const uint16_t *__restrict__ out, const uint16_t *__restrict__ dout,
+             float *__restrict__ delta, int B, int T, int Hq, int D, int stride) {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;");
+    const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= (long long)B * T * Hq) return;
+    const uint32_t *o2 = reinterpret_cast<const uint32_t *>(out + row * D);
+    const uint32_t *g2 = reinterpret_cast<const uint32_t *>(dout + row * D);
+    float acc = 0.f;
+    for (int d2 = lane; d2 < D / 2; d2 += 32) {
+        const uint32_t a = o2[d2], b = g2[d2];
+        acc = fmaf(bf16lo(a), bf16lo(b), acc);
+        acc = fmaf(bf16hi(a), bf16hi(b), acc);
+    }
+    acc = warp_sum(acc);
+    if (lane == 0) {
+        const int h = (int)(row % Hq);
+        const long long bt = row / Hq;
+        const int t = (int)(bt % T), b = (int)(bt / T);
+        delta[((size_t)b * Hq + h) * stride + t] = acc;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// dK, dV: item = (b, KV head, key tile j), longest first (j ascending)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void kv_item(int w, const BwGrid &g, int &b, int &kvh, int &j) {
+    const int per = g.B * g.Hkv;
+    j = w / per;
+    const int rest = w - j * per;
+    b = rest / g.Hkv;
+    kvh = rest - b * g.Hkv;
+}
+
+template <int D>
+__device__ void kv_producer(const BwMaps &maps, BwSync &sy, uint8_t *smem, const BwGrid &g,
+                            int32_t *status) {
+    using S = BwShape<D>;
+    const int grp = g.Hq / g.Hkv;
+    int ic = 0, sc = 0;
+    bool ok = true;
+    for (int w = blockIdx.x; w < g.n_items && ok; w += gridDim.x) {
+        int b, kvh, j;
+        kv_item(w, g, b, kvh, j);
+        ok = ptx::mbar_wait(A(sy.fixed_empty), (ic & 1) ^ 1);
+        if (!ok) break;
+        ptx::mbar_arrive_expect_tx(A(sy.fixed_full), 2 * S::kTileBytes);
+        for (int kb = 0; kb < S::kBlocks; ++kb) {
+            ptx::tma_load_3d(ptx::smem_addr(smem + kb * S::kBlockBytes), &maps.k, A(sy.fixed_full),
+                             kb * 64, j * 128, b * g.Hkv + kvh);
+            ptx::tma_load_3d(ptx::smem_addr(smem + S::kTileBytes + kb * S::kBlockBytes), &maps.v,
+                             A(sy.fixed_full), kb * 64, j * 128, b * g.Hkv + kvh);
+        }
+        ++ic;
+        for (int hh = 0; hh < grp && ok; ++hh) {
+            const int h = kvh * grp + hh;
+            for (int i = j; i < g.nT; ++i) {
+                const int st = sc % S::kStages;
+                ok = ptx::mbar_wait(A(sy.st_empty[st]), ((sc / S::kStages) & 1) ^ 1);
+                if (!ok) break;
+                uint8_t *base = smem + S::kOffStage + st * S::kStageBytes;
+                const uint32_t bar = A(sy.st_full[st]);
+                ptx::mbar_arrive_expect_tx(bar, 2 * S::kTileBytes + 2 * S::kVecBytes);
+                for (int kb = 0; kb < S::kBlocks; ++kb) {
+                    ptx::tma_load_4d(ptx::smem_addr(base + kb * S::kBlockBytes), &maps.q, bar,
+                                     kb * 64, h, i * 128, b);
+                    ptx::tma_load_4d(ptx::smem_addr(base + S::kTileBytes + kb * S::kBlockBytes),
+                                     &maps.dout, bar, kb * 64, h, i * 128, b);
+                }
+                ptx::tma_load_2d(ptx::smem_addr(base + 2 * S::kTileBytes), &maps.lse, bar, i * 128,
+                                 b * g.Hq + h);
+                ptx::tma_load_2d(ptx::smem_addr(base + 2 * S::kTileBytes + S::kVecBytes), &maps.delta,
+                                 bar, i * 128, b * g.Hq + h);
+                ++sc;
+            }
+        }
+    }
+    if (!ok) {
+        report(status, GQA_DEV_TIMEOUT);
+        if (ic > 0) ptx::mbar_wait(A(sy.fixed_full), (ic - 1) & 1);
+        for (int s = (sc > S::kStages ? sc - S::kStages : 0); s < sc; ++s)
+            ptx::mbar_wait(A(sy.st_full[s % S::kStages]), (s / S::kStages) & 1);
+    }
+}
+
+template <int D>
+__device__ void kv_mma(BwSync &sy, uint8_t *smem, uint32_t tmem, const BwGrid &g, int32_t *status) {
+    using S = BwShape<D>;
+    using M = BwMma<D>;
+    const int grp = g.Hq / g.Hkv;
+    const uint32_t k_base = ptx::smem_addr(smem), v_base = k_base + S::kTileBytes;
+    int ic = 0, sc = 0, pc = 0, ac = 0;
+    bool ok = true;
+    for (int w = blockIdx.x; w < g.n_items && ok; w += gridDim.x) {
+        int b, kvh, j;
+        kv_item(w, g, b, kvh, j);
+        ok = ptx::mbar_wait(A(sy.fixed_full), ic & 1);
+        if (!ok) break;
+        ++ic;
+        ptx::tc_fence_after();
+        bool first = true;
+        const int steps = grp * (g.nT - j);
+        for (int s = 0; s < steps && ok; ++s) {
+            const int st = sc % S::kStages;
+            ok = ptx::mbar_wait(A(sy.st_full[st]), (sc / S::kStages) & 1);
+            if (!ok) break;
+            ptx::tc_fence_after();
+            const uint32_t q_base = ptx::smem_addr(smem + S::kOffStage + st * S::kStageBytes);
+            const uint32_t do_base = q_base + S::kTileBytes;
+            M::ss(tmem + S::kColS, k_base, q_base);      // S^T  = K_j Q_i^T
+            M::ss(tmem + S::kColDP, v_base, do_base);    // dP^T = V_j dO_i^T
+            ptx::mma_commit(A(sy.s_full));
+            ok = ptx::mbar_wait(A(sy.p_full), pc & 1);
+            if (!ok) break;
+            ++pc;
+            if (first) {        // the previous item's epilogue has read dK, dV
+                ok = ptx::mbar_wait(A(sy.acc_empty), (ac & 1) ^ 1);
+                if (!ok) break;
+            }
+            ptx::tc_fence_after();
+            M::ts(tmem + S::kColAcc0, tmem + S::kColS, do_base, !first);   // dV += P^T dO_i
+            M::ts(tmem + S::kColAcc1, tmem + S::kColDP, q_base, !first);   // dK += dS^T Q_i
+            ptx::mma_commit(A(sy.st_empty[st]));
+            first = false;
+            ++sc;
+        }
+        if (!ok) break;
+        ptx::mma_commit(A(sy.acc_full));
+        ptx::mma_commit(A(sy.fixed_empty));
+        ++ac;
+    }
+    if (!ok) report(status, GQA_DEV_TIMEOUT);
+    ptx::mma_commit(A(sy.mma_done));
+    ptx::mbar_wait(A(sy.mma_done), 0);
+}
+
+// Elementwise step of the dK/dV kernel: thread = key row r of tile j; the 128
+// columns are the queries of tile i.
+template <int D>
+__device__ void kv_elementwise(BwSync &sy, uint8_t *smem, uint32_t tmem, const BwGrid &g,
+                               int32_t *status) {
+    using S = BwShape<D>;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int r = warp * 32 + lane;
+    const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+    const int grp = g.Hq / g.Hkv;
+    int sc = 0, ac = 0;
+    bool ok = true;
+    for (int w = blockIdx.x; w < g.n_items && ok; w += gridDim.x) {
+        int b, kvh, j;
+        kv_item(w, g, b, kvh, j);
+        const int key = j * 128 + r;
+        const int steps = grp * (g.nT - j);
+        for (int s = 0; s < steps && ok; ++s) {
+            const int i = j + s % (g.nT - j);
+            ok = __all_sync(0xffffffffu, ptx::mbar_wait(A(sy.s_full), sc & 1));
+            if (!ok) break;
+            const int st = sc % S::kStages;
+            ++sc;
+            ptx::tc_fence_after();
+            const float *lse_v = reinterpret_cast<const float *>(
+                smem + S::kOffStage + st * S::kStageBytes + 2 * S::kTileBytes);
+            const float *del_v = lse_v + 128;
+            const bool edge = i == j || (i + 1) * 128 > g.T;     // some (query, key) masked
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint32_t sv[32], dv[32];
+                ptx::tmem_ld32(lane_addr + S::kColS + 32 * c, sv);
+                ptx::tmem_ld32(lane_addr + S::kColDP + 32 * c, dv);
+                ptx::tmem_wait_ld();
+                uint32_t pp[16], dd[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    float p[2], ds[2];
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        const int col = 32 * c + 2 * e + u;
+                        const float lse2 = lse_v[col] * kLog2e;
+                        float pv = ex2(fmaf(__uint_as_float(sv[2 * e + u]), g.scale_log2, -lse2));
+                        if (edge) {
+                            const int query = i * 128 + col;
+                            if (query < key || query >= g.T) pv = 0.f;
+                        }
+                        p[u] = pv;
+                        ds[u] = pv * (__uint_as_float(dv[2 * e + u]) - del_v[col]);
+                    }
+                    pp[e] = pack_bf16x2(p[0], p[1]);
+                    dd[e] = pack_bf16x2(ds[0], ds[1]);
+                }
+                ptx::tmem_st16(lane_addr + S::kColS + 16 * c, pp);
+                ptx::tmem_st16(lane_addr + S::kColDP + 16 * c, dd);
+            }
+            ptx::tmem_wait_st();
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(A(sy.p_full));
+        }
+        if (!ok) break;
+        // epilogue: dV_j and c dK_j rows to global memory
+        ok = __all_sync(0xffffffffu, ptx::mbar_wait(A(sy.acc_full), ac & 1));
+        if (!ok) break;
+        ++ac;
+        ptx::tc_fence_after();
+        const size_t row = ((size_t)b * g.Hkv + kvh) * g.Lmax + key;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+            uint32_t va[32], ka[32];
+            ptx::tmem_ld32(lane_addr + S::kColAcc0 + 32 * c, va);
+            ptx::tmem_ld32(lane_addr + S::kColAcc1 + 32 * c, ka);
+            ptx::tmem_wait_ld();
+            uint32_t wv[16], wk[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                wv[e] = pack_bf16x2(__uint_as_float(va[2 * e]), __uint_as_float(va[2 * e + 1]));
+                wk[e] = pack_bf16x2(__uint_as_float(ka[2 * e]) * g.scale,
+                                    __uint_as_float(ka[2 * e + 1]) * g.scale);
+            }
+            if (key < g.T) {
+                uint4 *dvp = reinterpret_cast<uint4 *>(g.d1 + row * D + 32 * c);
+                uint4 *dkp = reinterpret_cast<uint4 *>(g.d0 + row * D + 32 * c);
+#pragma unroll
+                for (int x = 0; x < 4; ++x) {
+                    dvp[x] = make_uint4(wv[4 * x], wv[4 * x + 1], wv[4 * x + 2], wv[4 * x + 3]);
+                    dkp[x] = make_uint4(wk[4 * x], wk[4 * x + 1], wk[4 * x + 2], wk[4 * x + 3]);
+                }
+            }
+        }
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(A(sy.acc_empty));
+    }
+    if (!ok && lane == 0) report(status, GQA_DEV_TIMEOUT);
+}
+
+// ---------------------------------------------------------------------------
+// dQ: item = (b, query head, query tile i), longest first (i descending)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void q_item(int w, const BwGrid &g, int &b, int &h, int &i) {
+    const int per = g.B * g.Hq;
+    const int ii = w / per;
+    const int rest = w - ii * per;
+    i = g.nT - 1 - ii;
+    b = rest / g.Hq;
+    h = rest - b * g.Hq;
+}
+
+template <int D>
+__device__ void q_producer(const BwMaps &maps, BwSync &sy, uint8_t *smem, const BwGrid &g,
+                           int32_t *status) {
+    using S = BwShape<D>;
+    const int grp = g.Hq / g.Hkv;
+    int ic = 0, sc = 0;
+    bool ok = true;
+    for (int w = blockIdx.x; w < g.n_items && ok; w += gridDim.x) {
+        int b, h, i;
+        q_item(w, g, b, h, i);
+        const int kvh = h / grp;
+        ok = ptx::mbar_wait(A(sy.fixed_empty), (ic & 1) ^ 1);
+        if (!ok) break;
+        ptx::mbar_arrive_expect_tx(A(sy.fixed_full), 2 * S::kTileBytes);
+        for (int kb = 0; kb < S::kBlocks; ++kb) {
+            ptx::tma_load_4d(ptx::smem_addr(smem + kb * S::kBlockBytes), &maps.q, A(sy.fixed_full),
+                             kb * 64, h, i * 128, b);
+            ptx::tma_load_4d(ptx::smem_addr(smem + S::kTileBytes + kb * S::kBlockBytes), &maps.dout,
+                             A(sy.fixed_full), kb * 64, h, i * 128, b);
+        }
+        ++ic;
+        for (int j = 0; j <= i; ++j) {
+            const int st = sc % S::kStages;
+            ok = ptx::mbar_wait(A(sy.st_empty[st]), ((sc / S::kStages) & 1) ^ 1);
+            if (!ok) break;
+            uint8_t *base = smem + S::kOffKV + st * 2 * S::kTileBytes;
+            const uint32_t bar = A(sy.st_full[st]);
+            ptx::mbar_arrive_expect_tx(bar, 2 * S::kTileBytes);
+            for (int kb = 0; kb < S::kBlocks; ++kb) {
+                ptx::tma_load_3d(ptx::smem_addr(base + kb * S::kBlockBytes), &maps.k, bar, kb * 64,
+                                 j * 128, b * g.Hkv + kvh);
+                ptx::tma_load_3d(ptx::smem_addr(base + S::kTileBytes + kb * S::kBlockBytes), &maps.v,
+                                 bar, kb * 64, j * 128, b * g.Hkv + kvh);
+            }
+            ++sc;
+        }
+    }
+    if (!ok) {
+        report(status, GQA_DEV_TIMEOUT);
+        if (ic > 0) ptx::mbar_wait(A(sy.fixed_full), (ic - 1) & 1);
+        for (int s = (sc > S::kStages ? sc - S::kStages : 0); s < sc; ++s)
+            ptx::mbar_wait(A(sy.st_full[s % S::kStages]), (s / S::kStages) & 1);
+    }
+}
+
+template <int D>
+__device__ void q_mma(BwSync &sy, uint8_t *smem, uint32_t tmem, const BwGrid &g, int32_t *status) {
+    using S = BwShape<D>;
+    using M = BwMma<D>;
+    const uint32_t q_base = ptx::smem_addr(smem), do_base = q_base + S::kTileBytes;
+    int ic = 0, sc = 0, pc = 0, ac = 0;
+    bool ok = true;
+    for (int w = blockIdx.x; w < g.n_items && ok; w += gridDim.x) {
+        int b, h, i;
+        q_item(w, g, b, h, i);
+        ok = ptx::mbar_wait(A(sy.fixed_full), ic & 1);
+        if (!ok) break;
+        ++ic;
+        ptx::tc_fence_after();
+        for (int j = 0; j <= i && ok; ++j) {
+            const int st = sc % S::kStages;
+            ok = ptx::mbar_wait(A(sy.st_full[st]), (sc / S::kStages) & 1);
+            if (!ok) break;
+            ptx::tc_fence_after();
+            const uint32_t k_base = ptx::smem_addr(smem + S::kOffKV + st * 2 * S::kTileBytes);
+            const uint32_t v_base = k_base + S::kTileBytes;
+            M::ss(tmem + S::kColS, q_base, k_base);      // S  = Q_i K_j^T
+            M::ss(tmem + S::kColDP, do_base, v_base);    // dP = dO_i V_j^T
+            ptx::mma_commit(A(sy.s_full));
+            if (j == i) ptx::mma_commit(A(sy.fixed_empty));   // Q_i, dO_i no longer read
+            ok = ptx::mbar_wait(A(sy.p_full), pc & 1);
+            if (!ok) break;
+            ++pc;
+            if (j == 0) {
+                ok = ptx::mbar_wait(A(sy.acc_empty), (ac & 1) ^ 1);
+                if (!ok) break;
+            }
+            ptx::tc_fence_after();
+            M::ts(tmem + S::kColAcc0, tmem + S::kColDP, k_base, j > 0);    // dQ += dS K_j
+            ptx::mma_commit(A(sy.st_empty[st]));
+            ++sc;
+        }
+        if (!ok) break;
+        ptx::mma_commit(A(sy.acc_full));
+        ++ac;
+    }
+    if (!ok) report(status, GQA_DEV_TIMEOUT);
+    ptx::mma_commit(A(sy.mma_done));
+    ptx::mbar_wait(A(sy.mma_done), 0);
+}
+
+template <int D>
+__device__ void q_elementwise(BwSync &sy, uint32_t tmem, const BwGrid &g, int32_t *status) {
+    using S = BwShape<D>;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int r = warp * 32 + lane;
+    const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+    int sc = 0, ac = 0;
+    bool ok = true;
+    // this row's log-sum-exp and Delta, fetched one item ahead
+    auto fetch = [&](int w, float &l2, float &dl) {
+        int b, h, i;
+        q_item(w, g, b, h, i);
+        const int qrow = i * 128 + r;
+        const size_t off = ((size_t)b * g.Hq + h) * g.lse_stride + qrow;
+        l2 = qrow < g.T ? g.lse[off] * kLog2e : 0.f;
+        dl = qrow < g.T ? g.delta[off] : 0.f;
+    };
+    float nl2 = 0.f, ndl = 0.f;
+    if ((int)blockIdx.x < g.n_items) fetch(blockIdx.x, nl2, ndl);
+    for (int w = blockIdx.x; w < g.n_items && ok; w += gridDim.x) {
+        int b, h, i;
+        q_item(w, g, b, h, i);
+        const float lse2 = nl2, dlt = ndl;
+        if (w + (int)gridDim.x < g.n_items) fetch(w + gridDim.x, nl2, ndl);
+        const int qrow = i * 128 + r;
+        for (int j = 0; j <= i && ok; ++j) {
+            ok = __all_sync(0xffffffffu, ptx::mbar_wait(A(sy.s_full), sc & 1));
+            if (!ok) break;
+            ++sc;
+            ptx::tc_fence_after();
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint32_t sv[32], dv[32];
+                ptx::tmem_ld32(lane_addr + S::kColS + 32 * c, sv);
+                ptx::tmem_ld32(lane_addr + S::kColDP + 32 * c, dv);
+                ptx::tmem_wait_ld();
+                uint32_t dd[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    float ds[2];
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        float pv = ex2(fmaf(__uint_as_float(sv[2 * e + u]), g.scale_log2, -lse2));
+                        if (j == i && j * 128 + 32 * c + 2 * e + u > qrow) pv = 0.f;
+                        ds[u] = pv * (__uint_as_float(dv[2 * e + u]) - dlt);
+                    }
+                    dd[e] = pack_bf16x2(ds[0], ds[1]);
+                }
+                ptx::tmem_st16(lane_addr + S::kColDP + 16 * c, dd);
+            }
+            ptx::tmem_wait_st();
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(A(sy.p_full));
+        }
+        if (!ok) break;
+        ok = __all_sync(0xffffffffu, ptx::mbar_wait(A(sy.acc_full), ac & 1));
+        if (!ok) break;
+        ++ac;
+        ptx::tc_fence_after();
+        uint16_t *dst = g.d0 + (((size_t)b * g.T + qrow) * g.Hq + h) * D;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+            uint32_t a[32];
+            ptx::tmem_ld32(lane_addr + S::kColAcc0 + 32 * c, a);
+            ptx::tmem_wait_ld();
+            uint32_t wq[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+                wq[e] = pack_bf16x2(__uint_as_float(a[2 * e]) * g.scale,
+                                    __uint_as_float(a[2 * e + 1]) * g.scale);
+            if (qrow < g.T) {
+                uint4 *d4 = reinterpret_cast<uint4 *>(dst + 32 * c);
+#pragma unroll
+                for (int x = 0; x < 4; ++x)
+                    d4[x] = make_uint4(wq[4 * x], wq[4 * x + 1], wq[4 * x + 2], wq[4 * x + 3]);
+            }
+        }
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(A(sy.acc_empty));
+    }
+    if (!ok && lane == 0) report(status, GQA_DEV_TIMEOUT);
+}
+
+// ---------------------------------------------------------------------------
+// the two tensor-core kernels
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void bw_setup(BwSync &sy) {
+    if (threadIdx.x == 0) {
+        ptx::mbar_init(A(sy.fixed_full), 1);
+        ptx::mbar_init(A(sy.fixed_empty), 1);
+        for (int s = 0; s < 2; ++s) {
+            ptx::mbar_init(A(sy.st_full[s]), 1);
+            ptx::mbar_init(A(sy.st_empty[s]), 1);
+        }
+        ptx::mbar_init(A(sy.s_full), 1);
+        ptx::mbar_init(A(sy.p_full), 4);       // one elected lane per elementwise warp
+        ptx::mbar_init(A(sy.acc_full), 1);
+        ptx::mbar_init(A(sy.acc_empty), 4);
+        ptx::mbar_init(A(sy.mma_done), 1);
+        ptx::fence_barrier_init();
+    }
+    if ((threadIdx.x >> 5) == kBwMmaWarp) {
+        ptx::tmem_alloc(ptx::smem_addr(&sy.tmem_base), 512);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+}
+
+__device__ __forceinline__ void bw_teardown(BwSync &sy) {
+    ptx::tc_fence_before();
+    __syncthreads();
+    if ((threadIdx.x >> 5) == kBwMmaWarp) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(sy.tmem_base, 512);
+    }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kBwThreads, 1)
+bwd_kv_kernel(const __grid_constant__ BwMaps maps, BwGrid g, int32_t *status) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    __shared__ BwSync sy;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    bw_setup(sy);
+    // Delta (and the forward's outputs) come from the kernels before this one.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    const uint32_t tmem = sy.tmem_base;
+    if (warp == kBwTmaWarp) {
+        if (lane == 0) kv_producer<D>(maps, sy, smem, g, status);
+        __syncwarp();
+    } else if (warp == kBwMmaWarp) {
+        if (lane == 0) kv_mma<D>(sy, smem, tmem, g, status);
+        __syncwarp();
+    } else {
+        kv_elementwise<D>(sy, smem, tmem, g, status);
+    }
+    bw_teardown(sy);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kBwThreads, 1)
+bwd_q_kernel(const __grid_constant__ BwMaps maps, BwGrid g, int32_t *status) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    __shared__ BwSync sy;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    bw_setup(sy);
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    const uint32_t tmem = sy.tmem_base;
+    if (warp == kBwTmaWarp) {
+        if (lane == 0) q_producer<D>(maps, sy, smem, g, status);
+        __syncwarp();
+    } else if (warp == kBwMmaWarp) {
+        if (lane == 0) q_mma<D>(sy, smem, tmem, g, status);
+        __syncwarp();
+    } else {
+        q_elementwise<D>(sy, tmem, g, status);
+    }
+    bw_teardown(sy);
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+int lse_stride_of(int T) { return (T + 3) & ~3; }
+
+template <typename K>
+cudaError_t launch_pdl(K kern, dim3 grid, dim3 block, int smem, cudaStream_t s,
+                       const BwMaps &maps, const BwGrid &g, int32_t *status) {
+    cudaLaunchAttribute pdl[1];
+    pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cfg.attrs = pdl;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, maps, g, status);
+}
+
+template <int D>
+gqa_status launch_backward(const void *q, const void *k, const void *v, const void *out,
+                           const void *dout, const float *lse, void *dq, void *dk, void *dv, int B,
+                           int T, int Hq, int Hkv, int Lmax, float scale, float *delta,
+                           int32_t *status, cudaStream_t s) {
+    using S = BwShape<D>;
+    const int ls = lse_stride_of(T);
+    BwMaps maps;
+    {
+        const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)Hq, (cuuint64_t)T, (cuuint64_t)B};
+        const cuuint64_t str[3] = {(cuuint64_t)D * 2, (cuuint64_t)Hq * D * 2,
+                                   (cuuint64_t)T * Hq * D * 2};
+        const cuuint32_t box[4] = {64, 1, 128, 1};
+        if (!encode(&maps.q, q, 4, dims, str, box)) return GQA_ERR_CUDA;
+        if (!encode(&maps.dout, dout, 4, dims, str, box)) return GQA_ERR_CUDA;
+    }
+    {
+        const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)T, (cuuint64_t)B * Hkv};
+        const cuuint64_t str[2] = {(cuuint64_t)D * 2, (cuuint64_t)Lmax * D * 2};
+        const cuuint32_t box[3] = {64, 128, 1};
+        if (!encode(&maps.k, k, 3, dims, str, box)) return GQA_ERR_CUDA;
+        if (!encode(&maps.v, v, 3, dims, str, box)) return GQA_ERR_CUDA;
+    }
+    if (!encode_f32_2d(&maps.lse, lse, (cuuint64_t)T, (cuuint64_t)B * Hq, (cuuint64_t)ls * 4, 128))
+        return GQA_ERR_CUDA;
+    if (!encode_f32_2d(&maps.delta, delta, (cuuint64_t)T, (cuuint64_t)B * Hq, (cuuint64_t)ls * 4,
+                       128))
+        return GQA_ERR_CUDA;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return GQA_ERR_CUDA;
+    BwGrid g;
+    g.B = B;
+    g.T = T;
+    g.Hq = Hq;
+    g.Hkv = Hkv;
+    g.nT = (T + 127) / 128;
+    g.lse_stride = ls;
+    g.scale = scale;
+    g.scale_log2 = scale * kLog2e;
+    g.lse = lse;
+    g.delta = delta;
+    g.Lmax = Lmax;
+
+    // 1. Delta
+    {
+        cudaLaunchAttribute pdl[1];
+        pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        pdl[0].val.programmaticStreamSerializationAllowed = 1;
+        cudaLaunchConfig_t cfg = {};
+        const long long rows = (long long)B * T * Hq;
+        cfg.gridDim = dim3((unsigned)((rows + 7) / 8));
+        cfg.blockDim = dim3(256);
+        cfg.stream = s;
+        cfg.attrs = pdl;
+        cfg.numAttrs = 1;
+        if (cudaLaunchKernelEx(&cfg, delta_kernel, static_cast<const uint16_t *>(out),
+                               static_cast<const uint16_t *>(dout), delta, B, T, Hq, D, ls) !=
+            cudaSuccess)
+            return GQA_ERR_CUDA;
+    }
+    // 2. dK, dV
+    {
+        auto kern = bwd_kv_kernel<D>;
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kSmemKV) !=
+            cudaSuccess)
+            return GQA_ERR_CUDA;
+        BwGrid gk = g;
+        gk.n_items = g.nT * B * Hkv;
+        gk.d0 = static_cast<uint16_t *>(dk);
+        gk.d1 = static_cast<uint16_t *>(dv);
+        const int grid = gk.n_items < sms ? gk.n_items : sms;
+        if (launch_pdl(kern, dim3(grid), dim3(kBwThreads), S::kSmemKV, s, maps, gk, status) !=
+            cudaSuccess)
+            return GQA_ERR_CUDA;
+    }
+    // 3. dQ
+    {
+        auto kern = bwd_q_kernel<D>;
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kSmemQ) !=
+            cudaSuccess)
+            return GQA_ERR_CUDA;
+        BwGrid gq = g;
+        gq.n_items = g.nT * B * Hq;
+        gq.d0 = static_cast<uint16_t *>(dq);
+        gq.d1 = nullptr;
+        const int grid = gq.n_items < sms ? gq.n_items : sms;
+        if (launch_pdl(kern, dim3(grid), dim3(kBwThreads), S::kSmemQ, s, maps, gq, status) !=
+            cudaSuccess)
+            return GQA_ERR_CUDA;
+    }
+    return gqa_host::launch_status();
+}
+
+}  // namespace
+}  // namespace gqa
+
+extern "C" size_t gqa_backward_workspace_bytes(int B, int T, int Hq) {
+    if (B < 1 || T < 1 || Hq < 1) return 0;
+    return (size_t)B * Hq * gqa::lse_stride_of(T) * 4;
+}
+
+extern "C" gqa_status gqa_attention_backward(const void *q, const void *k, const void *v,
+                                             const void *out, const void *dout, const float *lse,
+                                             void *dq, void *dk, void *dv, int B, int T, int Hq,
+                                             int Hkv, int D, int Lmax, float scale, void *ws,
+                                             size_t ws_bytes, int32_t *status_dev, void *stream) {
+    using namespace gqa_host;
+    if (!q || !k || !v || !out || !dout || !lse || !dq || !dk || !dv || B < 1 || T < 1 ||
+        Hq < 1 || Hkv < 1 || Lmax < 1)
+        return GQA_ERR_INVALID_ARG;
+    if (Hq % Hkv != 0) return GQA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(dout) ||
+        !aligned16(lse) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+        return GQA_ERR_INVALID_ARG;
+    if (!head_dim_ok(D)) return GQA_ERR_UNSUPPORTED;
+    if (Lmax % 128 != 0) return GQA_ERR_INVALID_ARG;
+    if (T > Lmax) return GQA_ERR_CAPACITY;
+    if ((long long)((T + 127) / 128) * B * Hq > 0x7fffffffLL) return GQA_ERR_INVALID_ARG;
+    const size_t need = gqa_backward_workspace_bytes(B, T, Hq);
+    if (!ws || ws_bytes < need || !aligned16(ws)) return GQA_ERR_WORKSPACE;
+    int dev = 0, major = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        major != 10)
+        return GQA_ERR_UNSUPPORTED;
+    const float sc = scale > 0.f ? scale : 1.0f / sqrtf((float)D);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    float *delta = static_cast<float *>(ws);
+    switch (D) {
+        case 64: return gqa::launch_backward<64>(q, k, v, out, dout, lse, dq, dk, dv, B, T, Hq, Hkv, Lmax, sc, delta, status_dev, s);
+        case 96: return gqa::launch_backward<96>(q, k, v, out, dout, lse, dq, dk, dv, B, T, Hq, Hkv, Lmax, sc, delta, status_dev, s);
+        default: return gqa::launch_backward<128>(q, k, v, out, dout, lse, dq, dk, dv, B, T, Hq, Hkv, Lmax, sc, delta, status_dev, s);
+    }
+}

@@ -52,6 +52,7 @@
 
 #include "common.cuh"
 #include "ptx.cuh"
+#include "tmap.cuh"
 
 namespace gqa {
 namespace {
@@ -118,6 +119,8 @@ struct PfGrid {
     int n_items, n_pairs, B, T, Hq, Hkv, Lmax;
     const int32_t *pos0, *n_tok;   // chunk positions / token counts (NULL: 0 / T)
     const int32_t *doc_start;      // [B, T] first position of each token's document
+    float *lse;                    // optional [B, Hq, lse_stride] row log-sum-exp (prompts)
+    int lse_stride;
 };
 
 __device__ __forceinline__ int pf_item_b(int w, int B, int Hq) {
@@ -513,6 +516,9 @@ __device__ void softmax_tile(PfSync &sy, uint8_t *smem, uint32_t tmem, int t, co
         ptx::tc_fence_after();
         const float inv_l = 1.f / l;
         uint16_t *dst = out + (((size_t)I.b * T + qrow) * g.Hq + I.h) * D;
+        if (kMode == kPrompt && g.lse && qrow < T)   // natural-log LSE of the scaled scores
+            g.lse[((size_t)I.b * g.Hq + I.h) * g.lse_stride + qrow] =
+                (m + log2f(l)) * 0.69314718055994531f;
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
             uint32_t o[32];
@@ -543,7 +549,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 prefill_kernel(const __grid_constant__ PfMaps maps, uint16_t *__restrict__ out, int B, int T,
                int Hq, int Hkv, int Lmax, const int32_t *__restrict__ pos0,
                const int32_t *__restrict__ n_tok, const int32_t *__restrict__ doc_start,
-               float scale_log2, int n_pairs, int32_t *status) {
+               float *__restrict__ lse, float scale_log2, int n_pairs, int32_t *status) {
     using S = PfShape<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -559,6 +565,8 @@ prefill_kernel(const __grid_constant__ PfMaps maps, uint16_t *__restrict__ out, 
     g.pos0 = pos0;
     g.n_tok = n_tok;
     g.doc_start = doc_start;
+    g.lse = lse;
+    g.lse_stride = (T + 3) & ~3;
     g.n_items = n_pairs * Hq * B;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -619,40 +627,11 @@ prefill_kernel(const __grid_constant__ PfMaps maps, uint16_t *__restrict__ out, 
 // ---------------------------------------------------------------------------
 // host side: tensor maps and launch
 // ---------------------------------------------------------------------------
-typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
-                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
-                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encoder() {
-    static EncodeTiledFn fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-                cudaSuccess && q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    });
-    return fn;
-}
-
-// bf16 tensor map with 128-byte swizzle and a {64, rows...} box; OOB reads are zero.
-bool encode(CUtensorMap *m, const void *base, int rank, const cuuint64_t *dims,
-            const cuuint64_t *strides, const cuuint32_t *box) {
-    EncodeTiledFn fn = encoder();
-    if (!fn) return false;
-    cuuint32_t es[5] = {1, 1, 1, 1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void *>(base), dims, strides,
-              box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <int D>
 gqa_status launch_prefill(const void *q, const void *kc, const void *vc, void *out, int B, int T,
                           int Hq, int Hkv, int Lmax, const int32_t *pos0, const int32_t *n_tok,
-                          const int32_t *doc_start, float scale_log2, int32_t *status,
-                          cudaStream_t s) {
+                          const int32_t *doc_start, float *lse, float scale_log2,
+                          int32_t *status, cudaStream_t s) {
     using S = PfShape<D>;
     PfMaps maps;
     {
@@ -705,7 +684,7 @@ gqa_status launch_prefill(const void *q, const void *kc, const void *vc, void *o
     cfg.attrs = pdl;
     cfg.numAttrs = 1;
     if (cudaLaunchKernelEx(&cfg, kern, maps, static_cast<uint16_t *>(out), B, T, Hq, Hkv, Lmax,
-                           pos0, n_tok, doc_start, scale_log2, n_pairs, status) != cudaSuccess)
+                           pos0, n_tok, doc_start, lse, scale_log2, n_pairs, status) != cudaSuccess)
         return GQA_ERR_CUDA;
     return gqa_host::launch_status();
 }
@@ -725,8 +704,8 @@ namespace {
 
 gqa_status prefill_entry(const void *q, const void *k_cache, const void *v_cache, void *out,
                          const int32_t *pos0, const int32_t *n_tok, const int32_t *doc_start,
-                         int max_pos0_host, int B, int T, int Hq, int Hkv, int D, int Lmax,
-                         float scale, int32_t *status_dev, void *stream) {
+                         float *lse, int max_pos0_host, int B, int T, int Hq, int Hkv, int D,
+                         int Lmax, float scale, int32_t *status_dev, void *stream) {
     using namespace gqa_host;
     if (!q || !k_cache || !v_cache || !out || B < 1 || T < 1 || Hq < 1 || Hkv < 1 || Lmax < 1)
         return GQA_ERR_INVALID_ARG;
@@ -734,7 +713,7 @@ gqa_status prefill_entry(const void *q, const void *k_cache, const void *v_cache
     if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
         return GQA_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(pos0) & 3u) || (reinterpret_cast<uintptr_t>(n_tok) & 3u) ||
-        (reinterpret_cast<uintptr_t>(doc_start) & 3u))
+        (reinterpret_cast<uintptr_t>(doc_start) & 3u) || (reinterpret_cast<uintptr_t>(lse) & 3u))
         return GQA_ERR_INVALID_ARG;
     if (!head_dim_ok(D)) return GQA_ERR_UNSUPPORTED;
     if (Lmax % 128 != 0) return GQA_ERR_INVALID_ARG;
@@ -746,9 +725,9 @@ gqa_status prefill_entry(const void *q, const void *k_cache, const void *v_cache
     const float sl2 = sc * 1.4426950408889634f;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     switch (D) {
-        case 64: return gqa::launch_prefill<64>(q, k_cache, v_cache, out, B, T, Hq, Hkv, Lmax, pos0, n_tok, doc_start, sl2, status_dev, s);
-        case 96: return gqa::launch_prefill<96>(q, k_cache, v_cache, out, B, T, Hq, Hkv, Lmax, pos0, n_tok, doc_start, sl2, status_dev, s);
-        default: return gqa::launch_prefill<128>(q, k_cache, v_cache, out, B, T, Hq, Hkv, Lmax, pos0, n_tok, doc_start, sl2, status_dev, s);
+        case 64: return gqa::launch_prefill<64>(q, k_cache, v_cache, out, B, T, Hq, Hkv, Lmax, pos0, n_tok, doc_start, lse, sl2, status_dev, s);
+        case 96: return gqa::launch_prefill<96>(q, k_cache, v_cache, out, B, T, Hq, Hkv, Lmax, pos0, n_tok, doc_start, lse, sl2, status_dev, s);
+        default: return gqa::launch_prefill<128>(q, k_cache, v_cache, out, B, T, Hq, Hkv, Lmax, pos0, n_tok, doc_start, lse, sl2, status_dev, s);
     }
 }
 
@@ -757,8 +736,16 @@ gqa_status prefill_entry(const void *q, const void *k_cache, const void *v_cache
 extern "C" gqa_status gqa_prefill(const void *q, const void *k_cache, const void *v_cache,
                                   void *out, int B, int T, int Hq, int Hkv, int D, int Lmax,
                                   float scale, int32_t *status_dev, void *stream) {
-    return prefill_entry(q, k_cache, v_cache, out, nullptr, nullptr, nullptr, 0, B, T, Hq, Hkv, D,
-                         Lmax, scale, status_dev, stream);
+    return prefill_entry(q, k_cache, v_cache, out, nullptr, nullptr, nullptr, nullptr, 0, B, T, Hq,
+                         Hkv, D, Lmax, scale, status_dev, stream);
+}
+
+extern "C" gqa_status gqa_prefill_lse(const void *q, const void *k_cache, const void *v_cache,
+                                      void *out, float *lse, int B, int T, int Hq, int Hkv, int D,
+                                      int Lmax, float scale, int32_t *status_dev, void *stream) {
+    if (!lse) return GQA_ERR_INVALID_ARG;
+    return prefill_entry(q, k_cache, v_cache, out, nullptr, nullptr, nullptr, lse, 0, B, T, Hq,
+                         Hkv, D, Lmax, scale, status_dev, stream);
 }
 
 extern "C" gqa_status gqa_prefill_chunk(const void *q, const void *k_cache, const void *v_cache,
@@ -766,8 +753,8 @@ extern "C" gqa_status gqa_prefill_chunk(const void *q, const void *k_cache, cons
                                         int max_pos0_host, int B, int T, int Hq, int Hkv, int D,
                                         int Lmax, float scale, int32_t *status_dev, void *stream) {
     if (!pos0) return GQA_ERR_INVALID_ARG;
-    return prefill_entry(q, k_cache, v_cache, out, pos0, n_tok, nullptr, max_pos0_host, B, T, Hq,
-                         Hkv, D, Lmax, scale, status_dev, stream);
+    return prefill_entry(q, k_cache, v_cache, out, pos0, n_tok, nullptr, nullptr, max_pos0_host, B,
+                         T, Hq, Hkv, D, Lmax, scale, status_dev, stream);
 }
 
 extern "C" gqa_status gqa_prefill_docs(const void *q, const void *k_cache, const void *v_cache,
@@ -775,8 +762,8 @@ extern "C" gqa_status gqa_prefill_docs(const void *q, const void *k_cache, const
                                        int Hkv, int D, int Lmax, float scale, int32_t *status_dev,
                                        void *stream) {
     if (!doc_start) return GQA_ERR_INVALID_ARG;
-    return prefill_entry(q, k_cache, v_cache, out, nullptr, nullptr, doc_start, 0, B, T, Hq, Hkv,
-                         D, Lmax, scale, status_dev, stream);
+    return prefill_entry(q, k_cache, v_cache, out, nullptr, nullptr, doc_start, nullptr, 0, B, T,
+                         Hq, Hkv, D, Lmax, scale, status_dev, stream);
 }
 
 // ---------------------------------------------------------------------------

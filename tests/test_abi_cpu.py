@@ -143,6 +143,22 @@ def test_docs_validation(lib):
     assert lib.gqa_doc_start(f, f, 0, 10, None, None) == 1
 
 
+def test_backward_validation(lib):
+    f = FAKE
+    ws = ctypes.c_size_t(1 << 20)
+    args = lambda D=64, T=100, L=128, Hq=4, wsb=ws, w=f: (f, f, f, f, f, f, f, f, f, 1, T, Hq, 2, D,
+                                                          L, 0.0, w, wsb, None, None)
+    assert lib.gqa_attention_backward(None, *args()[1:]) == 1
+    assert lib.gqa_attention_backward(*args(D=80)) == 2
+    assert lib.gqa_attention_backward(*args(T=300, L=256)) == 3
+    assert lib.gqa_attention_backward(*args(Hq=5)) == 1
+    assert lib.gqa_attention_backward(*args(wsb=ctypes.c_size_t(16))) == 6
+    assert lib.gqa_attention_backward(*args(w=None)) == 6
+    assert lib.gqa_backward_workspace_bytes(2, 1001, 24) == 2 * 24 * 1004 * 4
+    assert lib.gqa_backward_workspace_bytes(0, 10, 1) == 0
+    assert lib.gqa_prefill_lse(f, f, f, f, None, 1, 10, 4, 2, 64, 128, 0.0, None, None) == 1
+
+
 def test_decode_validation(lib):
     f = FAKE
     ws = ctypes.c_size_t(1 << 20)

@@ -1,0 +1,91 @@
+"""GPU parity: the attention backward (gqa_prefill_lse + gqa_attention_backward)
+against the float64 oracle's gradients.
+
+Full gradients at sizes the oracle finishes in seconds (ragged tails, MHA, GQA,
+MQA, every head_dim) and at the 3.8B layer's heads and length (T = 2048, 24/8
+heads, D = 128; one sequence); the forward's log-sum-exp; the forward output of
+gqa_prefill_lse equal to gqa_prefill's bit for bit; cache slots past T of dk /
+dv untouched; repeat runs bit-identical.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import rope_gqa_kv_b200 as gqa
+
+from helpers import assert_grad_close, bits
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _case(B, T, Hq, Hkv, D, seed, L=None):
+    g = torch.Generator().manual_seed(seed)
+    L = L or (T + 127) // 128 * 128
+    q = torch.randn(B, T, Hq, D, generator=g).to(torch.bfloat16)
+    kt = torch.randn(B, T, Hkv, D, generator=g).to(torch.bfloat16)
+    vt = torch.randn(B, T, Hkv, D, generator=g).to(torch.bfloat16)
+    dout = torch.randn(B, T, Hq, D, generator=g).to(torch.bfloat16)
+    kc = torch.full((B, Hkv, L, D), float("nan"), dtype=torch.bfloat16)
+    vc = kc.clone()
+    kc[:, :, :T] = kt.transpose(1, 2)
+    vc[:, :, :T] = vt.transpose(1, 2)
+    return q, kt, vt, dout, kc, vc
+
+
+def _run(q, dout, kc, vc, dk=None, dv=None):
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    dq_, dkc, dvc = q.to(DEV), kc.to(DEV), vc.to(DEV)
+    o, lse = gqa.gqa_prefill_lse(dq_, dkc, dvc, status=st)
+    grads = gqa.gqa_attention_backward(dq_, dkc, dvc, o, dout.to(DEV), lse, dk=dk, dv=dv,
+                                       status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0, "device status %#x" % st.item()
+    return o, lse, grads
+
+
+@pytest.mark.parametrize("B,T,Hq,Hkv,D", [
+    (1, 128, 2, 1, 64),       # one tile
+    (2, 300, 6, 2, 128),      # GQA, ragged last tile
+    (1, 513, 8, 8, 96),       # MHA, one row into the fifth tile
+    (1, 385, 8, 1, 64),       # MQA
+    (2, 1000, 8, 2, 128),
+])
+def test_backward_vs_oracle(cuda_lib, B, T, Hq, Hkv, D):
+    q, kt, vt, dout, kc, vc = _case(B, T, Hq, Hkv, D, seed=T + D)
+    o, lse, (dq, dk, dv) = _run(q, dout, kc, vc)
+    rq, rk, rv, ro, rl = oracle.attention_backward(bits(q), bits(kt), bits(vt), bits(dout))
+    np.testing.assert_allclose(lse[:, :, :T].double().cpu().numpy(), rl, rtol=0, atol=1e-5)
+    assert_grad_close(dq, rq, "dq")
+    assert_grad_close(dk[:, :, :T].transpose(1, 2), rk, "dk")
+    assert_grad_close(dv[:, :, :T].transpose(1, 2), rv, "dv")
+
+
+def test_backward_3p8b_heads_full_length(cuda_lib):
+    """One sequence of the 3.8B layer's shape: T = 2048, 24 query / 8 KV heads, D = 128."""
+    q, kt, vt, dout, kc, vc = _case(1, 2048, 24, 8, 128, seed=2048)
+    _, _, (dq, dk, dv) = _run(q, dout, kc, vc)
+    rq, rk, rv, _, _ = oracle.attention_backward(bits(q), bits(kt), bits(vt), bits(dout))
+    assert_grad_close(dq, rq, "dq")
+    assert_grad_close(dk[:, :, :2048].transpose(1, 2), rk, "dk")
+    assert_grad_close(dv[:, :, :2048].transpose(1, 2), rv, "dv")
+
+
+def test_forward_with_lse_is_prefill_bit_for_bit(cuda_lib):
+    q, _, _, _, kc, vc = _case(2, 333, 6, 2, 128, seed=5)
+    dq_, dkc, dvc = q.to(DEV), kc.to(DEV), vc.to(DEV)
+    a = gqa.gqa_prefill(dq_, dkc, dvc)
+    b, _ = gqa.gqa_prefill_lse(dq_, dkc, dvc)
+    torch.cuda.synchronize()
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+def test_slots_past_t_untouched_and_deterministic(cuda_lib):
+    q, _, _, dout, kc, vc = _case(1, 200, 4, 2, 64, seed=6, L=384)
+    sentinel = torch.full((1, 2, 384, 64), 9.0, dtype=torch.bfloat16, device=DEV)
+    _, _, (dq1, dk1, dv1) = _run(q, dout, kc, vc, dk=sentinel.clone(), dv=sentinel.clone())
+    assert (dk1[:, :, 200:] == 9.0).all() and (dv1[:, :, 200:] == 9.0).all()
+    _, _, (dq2, dk2, dv2) = _run(q, dout, kc, vc, dk=sentinel.clone(), dv=sentinel.clone())
+    for a, b in ((dq1, dq2), (dk1, dk2), (dv1, dv2)):
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16))

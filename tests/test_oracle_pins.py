@@ -483,3 +483,71 @@ def test_each_document_is_its_own_prefill():
             a, e = cuts[i], cuts[i + 1]
             alone, _, _ = oracle.prefill(q[b:b + 1, a:e], k[b:b + 1, a:e], v[b:b + 1, a:e], True)
             np.testing.assert_allclose(o[b:b + 1, a:e], alone, rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# attention backward
+# ---------------------------------------------------------------------------
+def _loss(q, k, v, dout):
+    """L = sum(dout * o) through the forward oracle (no RoPE: q, k as given)."""
+    T = q.shape[1]
+    o = oracle.attention(q, k, v, np.arange(T)[None, :].repeat(q.shape[0], 0))
+    return float((dout * o).sum())
+
+
+def test_backward_matches_finite_differences():
+    rng = np.random.default_rng(40)
+    B, T, Hq, Hkv, D = 1, 5, 4, 2, 4
+    q, k, v = (rng.standard_normal((B, T, Hq, D)), rng.standard_normal((B, T, Hkv, D)),
+               rng.standard_normal((B, T, Hkv, D)))
+    dout = rng.standard_normal((B, T, Hq, D))
+    dq, dk, dv, _, _ = oracle.attention_backward(q, k, v, dout)
+    eps = 1e-6
+    for x, grad in ((q, dq), (k, dk), (v, dv)):
+        num = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += eps
+            xm[idx] -= eps
+            args_p = [xp if a is x else a for a in (q, k, v)]
+            args_m = [xm if a is x else a for a in (q, k, v)]
+            num[idx] = (_loss(*args_p, dout) - _loss(*args_m, dout)) / (2 * eps)
+        np.testing.assert_allclose(grad, num, rtol=0, atol=2e-8)
+
+
+def test_backward_matches_torch_autograd_sdpa():
+    rng = np.random.default_rng(41)
+    B, T, Hq, Hkv, D = 2, 37, 6, 2, 16
+    q, k, v = (rng.standard_normal((B, T, Hq, D)), rng.standard_normal((B, T, Hkv, D)),
+               rng.standard_normal((B, T, Hkv, D)))
+    dout = rng.standard_normal((B, T, Hq, D))
+    dq, dk, dv, o, lse = oracle.attention_backward(q, k, v, dout)
+    tq, tk, tv = (torch.tensor(a, dtype=torch.float64, requires_grad=True) for a in (q, k, v))
+    g = Hq // Hkv
+    out = F.scaled_dot_product_attention(tq.transpose(1, 2),
+                                         tk.repeat_interleave(g, dim=2).transpose(1, 2),
+                                         tv.repeat_interleave(g, dim=2).transpose(1, 2),
+                                         is_causal=True).transpose(1, 2)
+    out.backward(torch.tensor(dout))
+    np.testing.assert_allclose(o, out.detach().numpy(), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(dq, tq.grad.numpy(), rtol=0, atol=1e-11)
+    np.testing.assert_allclose(dk, tk.grad.numpy(), rtol=0, atol=1e-11)
+    np.testing.assert_allclose(dv, tv.grad.numpy(), rtol=0, atol=1e-11)
+    # log-sum-exp of the first row: one key
+    s00 = float(q[0, 0, 0] @ k[0, 0, 0]) / math.sqrt(D)
+    assert abs(lse[0, 0, 0] - s00) < 1e-12
+
+
+def test_backward_sums():
+    """dV summed over keys is dO summed over the group's queries (softmax rows
+    sum to one), and dS rows sum to zero, so dQ is unchanged by adding a
+    constant vector to every key."""
+    rng = np.random.default_rng(42)
+    B, T, Hq, Hkv, D = 1, 20, 4, 1, 8
+    q, k, v = (rng.standard_normal((B, T, Hq, D)), rng.standard_normal((B, T, Hkv, D)),
+               rng.standard_normal((B, T, Hkv, D)))
+    dout = rng.standard_normal((B, T, Hq, D))
+    dq, dk, dv, _, _ = oracle.attention_backward(q, k, v, dout)
+    np.testing.assert_allclose(dv.sum(axis=1)[0, 0], dout.sum(axis=(1, 2))[0], rtol=0, atol=1e-12)
+    dq2, _, _, _, _ = oracle.attention_backward(q, k + rng.standard_normal((1, 1, Hkv, D)), v, dout)
+    np.testing.assert_allclose(dq2, dq, rtol=0, atol=1e-11)
