@@ -13,7 +13,7 @@
 // recomputed from the forward's row log-sum-exp, never stored.
 //
 // Three launches:
-//   delta_kernel   Delta[b, h, t] = sum_d dO * O (HBM-bound, one warp per row);
+//   delta_kernel   Delta[b, h, t] = sum_d dO * O (HBM-bound, 16-byte loads);
 //   bwd_kv_kernel  per (b, KV head, 128-key tile j), persistent: for every query
 //                  head of the group and every query tile i >= j,
 //                    S^T = K_j Q_i^T, dP^T = V_j dO_i^T       (two SS MMAs)
@@ -26,8 +26,10 @@
 //                  dP, dQ_i += dS K_j.
 // The same shared-memory tile serves as a K-major operand (the contraction over
 // D) and as an MN-major one (the contraction over its rows), as in the forward
-// kernel.  Warp roles (192 threads): warps 0-3 elementwise + epilogue (thread =
-// TMEM lane), warp 4 TMA producer, warp 5 MMA issuer.  Every mbarrier wait is
+// kernel.  Warp roles (384 threads, three warpgroups): warps 0-7 elementwise +
+// epilogue (thread = TMEM lane; warps w and w + 4 share lane quadrant w and take
+// 64 of the 128 columns each; 208 registers), warp 8 TMA producer, warp 9 MMA
+// issuer, warps 10-11 idle (88 registers), as in the forward kernel.  Every mbarrier wait is
 // bounded (1 s) and raises GQA_DEV_TIMEOUT; tensor memory is released only after
 // the MMA thread has seen its last MMA complete.
 #include <cuda.h>
@@ -39,9 +41,14 @@
 namespace gqa {
 namespace {
 
-constexpr int kBwThreads = 192;
-constexpr int kBwTmaWarp = 4;
-constexpr int kBwMmaWarp = 5;
+constexpr int kBwThreads = 384;
+constexpr int kBwTmaWarp = 8;
+constexpr int kBwMmaWarp = 9;
+constexpr uint32_t kBwEwRegs = 208, kBwCtlRegs = 88;   // 2 * 208 + 88 = 3 * 168 at launch
+static_assert(2 * kBwEwRegs + kBwCtlRegs == 3 * 168 && kBwThreads == 3 * 128,
+              "register split must balance");
+constexpr int kEwWarps = 8;                 // elementwise warps: 2 per TMEM lane quadrant
+constexpr int kEwBarrier = 1;               // named barrier of the elementwise warps
 constexpr float kLog2e = 1.4426950408889634f;
 
 template <int D>
@@ -86,6 +93,10 @@ struct BwGrid {
 
 __device__ __forceinline__ uint32_t A(const uint64_t &b) { return ptx::smem_addr(&b); }
 
+__device__ __forceinline__ void ew_sync() {
+    asm volatile("bar.sync %0, %1;" ::"n"(kEwBarrier), "n"(kEwWarps * 32) : "memory");
+}
+
 template <int D>
 struct BwMma {
     using S = BwShape<D>;
@@ -110,26 +121,33 @@ struct BwMma {
 };
 
 // ---------------------------------------------------------------------------
-// Delta = rowsum(dO * O): one warp per (b, t, h) row
+// Delta = rowsum(dO * O): TPR lanes per (b, t, h) row, 16-byte loads
 // ---------------------------------------------------------------------------
+template <int D>
 __global__ void __launch_bounds__(256)
 delta_kernel(const uint16_t *__restrict__ out, const uint16_t *__restrict__ dout,
-             float *__restrict__ delta, int B, int T, int Hq, int D, int stride) {
+             float *__restrict__ delta, int B, int T, int Hq, int stride) {
+    constexpr int kChunks = D / 8;                       // 16-byte pieces per row
+    constexpr int kTPR = kChunks > 8 ? 16 : 8;            // lanes per row (power of two)
     asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;");
-    const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
-    const int lane = threadIdx.x & 31;
-    if (row >= (long long)B * T * Hq) return;
-    const uint32_t *o2 = reinterpret_cast<const uint32_t *>(out + row * D);
-    const uint32_t *g2 = reinterpret_cast<const uint32_t *>(dout + row * D);
+    const int lane = threadIdx.x & 31, j = lane % kTPR;
+    const long long row = ((long long)blockIdx.x * 256 + threadIdx.x) / kTPR;
+    const bool live = row < (long long)B * T * Hq;
     float acc = 0.f;
-    for (int d2 = lane; d2 < D / 2; d2 += 32) {
-        const uint32_t a = o2[d2], b = g2[d2];
-        acc = fmaf(bf16lo(a), bf16lo(b), acc);
-        acc = fmaf(bf16hi(a), bf16hi(b), acc);
+    if (live && j < kChunks) {
+        const uint4 a = *reinterpret_cast<const uint4 *>(out + row * D + 8 * j);
+        const uint4 c = *reinterpret_cast<const uint4 *>(dout + row * D + 8 * j);
+        const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, cw[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            acc = fmaf(bf16lo(aw[e]), bf16lo(cw[e]), acc);
+            acc = fmaf(bf16hi(aw[e]), bf16hi(cw[e]), acc);
+        }
     }
-    acc = warp_sum(acc);
-    if (lane == 0) {
+#pragma unroll
+    for (int o = kTPR / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (live && j == 0) {
         const int h = (int)(row % Hq);
         const long long bt = row / Hq;
         const int t = (int)(bt % T), b = (int)(bt / T);
@@ -250,15 +268,50 @@ __device__ void kv_mma(BwSync &sy, uint8_t *smem, uint32_t tmem, const BwGrid &g
     ptx::mbar_wait(A(sy.mma_done), 0);
 }
 
-// Elementwise step of the dK/dV kernel: thread = key row r of tile j; the 128
-// columns are the queries of tile i.
+// Elementwise step of the dK/dV kernel: thread = key row r of tile j, columns =
+// the queries of tile i; warp w takes lane quadrant w % 4 and columns
+// [64 (w / 4), 64 (w / 4) + 64).  Both warps of a quadrant load their S^T and dP^T
+// columns before either writes P^T / dS^T over them (the packed bf16 halves land
+// on the lower columns), hence the barrier between loads and stores.
+template <int D, bool kEdge>
+__device__ __forceinline__ void kv_block(const uint32_t (&sv)[64], const uint32_t (&dv)[64],
+                                         const float *lse_v, const float *del_v, int col0,
+                                         int qbase, int key, int T, float sl2,
+                                         uint32_t (&pp)[32], uint32_t (&dd)[32]) {
+#pragma unroll
+    for (int c4 = 0; c4 < 16; ++c4) {
+        const float4 l4 = *reinterpret_cast<const float4 *>(lse_v + col0 + 4 * c4);
+        const float4 d4 = *reinterpret_cast<const float4 *>(del_v + col0 + 4 * c4);
+        const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+        const float dl[4] = {d4.x, d4.y, d4.z, d4.w};
+        float p[4], ds[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int e = 4 * c4 + u;
+            float pv = ex2(fmaf(__uint_as_float(sv[e]), sl2, -lv[u] * kLog2e));
+            if (kEdge) {
+                const int query = qbase + col0 + e;
+                if (query < key || query >= T) pv = 0.f;
+            }
+            p[u] = pv;
+            ds[u] = pv * (__uint_as_float(dv[e]) - dl[u]);
+        }
+        pp[2 * c4] = pack_bf16x2(p[0], p[1]);
+        pp[2 * c4 + 1] = pack_bf16x2(p[2], p[3]);
+        dd[2 * c4] = pack_bf16x2(ds[0], ds[1]);
+        dd[2 * c4 + 1] = pack_bf16x2(ds[2], ds[3]);
+    }
+}
+
 template <int D>
 __device__ void kv_elementwise(BwSync &sy, uint8_t *smem, uint32_t tmem, const BwGrid &g,
                                int32_t *status) {
     using S = BwShape<D>;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int r = warp * 32 + lane;
-    const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+    const int quad = warp & 3, half = warp >> 2;
+    const int r = quad * 32 + lane;
+    const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
+    const int col0 = 64 * half;                  // this warp's 64 query columns
     const int grp = g.Hq / g.Hkv;
     int sc = 0, ac = 0;
     bool ok = true;
@@ -277,49 +330,35 @@ __device__ void kv_elementwise(BwSync &sy, uint8_t *smem, uint32_t tmem, const B
             const float *lse_v = reinterpret_cast<const float *>(
                 smem + S::kOffStage + st * S::kStageBytes + 2 * S::kTileBytes);
             const float *del_v = lse_v + 128;
-            const bool edge = i == j || (i + 1) * 128 > g.T;     // some (query, key) masked
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                uint32_t sv[32], dv[32];
-                ptx::tmem_ld32(lane_addr + S::kColS + 32 * c, sv);
-                ptx::tmem_ld32(lane_addr + S::kColDP + 32 * c, dv);
-                ptx::tmem_wait_ld();
-                uint32_t pp[16], dd[16];
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    float p[2], ds[2];
-#pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const int col = 32 * c + 2 * e + u;
-                        const float lse2 = lse_v[col] * kLog2e;
-                        float pv = ex2(fmaf(__uint_as_float(sv[2 * e + u]), g.scale_log2, -lse2));
-                        if (edge) {
-                            const int query = i * 128 + col;
-                            if (query < key || query >= g.T) pv = 0.f;
-                        }
-                        p[u] = pv;
-                        ds[u] = pv * (__uint_as_float(dv[2 * e + u]) - del_v[col]);
-                    }
-                    pp[e] = pack_bf16x2(p[0], p[1]);
-                    dd[e] = pack_bf16x2(ds[0], ds[1]);
-                }
-                ptx::tmem_st16(lane_addr + S::kColS + 16 * c, pp);
-                ptx::tmem_st16(lane_addr + S::kColDP + 16 * c, dd);
-            }
+            uint32_t sv[64], dv[64];
+            ptx::tmem_ld32(lane_addr + S::kColS + col0, *reinterpret_cast<uint32_t(*)[32]>(sv));
+            ptx::tmem_ld32(lane_addr + S::kColS + col0 + 32, *reinterpret_cast<uint32_t(*)[32]>(sv + 32));
+            ptx::tmem_ld32(lane_addr + S::kColDP + col0, *reinterpret_cast<uint32_t(*)[32]>(dv));
+            ptx::tmem_ld32(lane_addr + S::kColDP + col0 + 32, *reinterpret_cast<uint32_t(*)[32]>(dv + 32));
+            ptx::tmem_wait_ld();
+            ew_sync();            // every S^T / dP^T column is in registers before any store
+            uint32_t pp[32], dd[32];
+            if (i == j || (i + 1) * 128 > g.T)                   // some (query, key) masked
+                kv_block<D, true>(sv, dv, lse_v, del_v, col0, i * 128, key, g.T, g.scale_log2, pp, dd);
+            else
+                kv_block<D, false>(sv, dv, lse_v, del_v, col0, i * 128, key, g.T, g.scale_log2, pp, dd);
+            ptx::tmem_st16(lane_addr + S::kColS + col0 / 2, *reinterpret_cast<uint32_t(*)[16]>(pp));
+            ptx::tmem_st16(lane_addr + S::kColS + col0 / 2 + 16, *reinterpret_cast<uint32_t(*)[16]>(pp + 16));
+            ptx::tmem_st16(lane_addr + S::kColDP + col0 / 2, *reinterpret_cast<uint32_t(*)[16]>(dd));
+            ptx::tmem_st16(lane_addr + S::kColDP + col0 / 2 + 16, *reinterpret_cast<uint32_t(*)[16]>(dd + 16));
             ptx::tmem_wait_st();
             ptx::tc_fence_before();
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(A(sy.p_full));
         }
         if (!ok) break;
-        // epilogue: dV_j and c dK_j rows to global memory
+        // epilogue: dV_j and c dK_j rows to global memory, half of D per warp
         ok = __all_sync(0xffffffffu, ptx::mbar_wait(A(sy.acc_full), ac & 1));
         if (!ok) break;
         ++ac;
         ptx::tc_fence_after();
         const size_t row = ((size_t)b * g.Hkv + kvh) * g.Lmax + key;
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = half; c < D / 32; c += 2) {
             uint32_t va[32], ka[32];
             ptx::tmem_ld32(lane_addr + S::kColAcc0 + 32 * c, va);
             ptx::tmem_ld32(lane_addr + S::kColAcc1 + 32 * c, ka);
@@ -451,12 +490,32 @@ __device__ void q_mma(BwSync &sy, uint8_t *smem, uint32_t tmem, const BwGrid &g,
     ptx::mbar_wait(A(sy.mma_done), 0);
 }
 
+template <bool kDiag>
+__device__ __forceinline__ void q_block(const uint32_t (&sv)[64], const uint32_t (&dv)[64],
+                                        int key0, int qrow, float sl2, float lse2, float dlt,
+                                        uint32_t (&dd)[32]) {
+#pragma unroll
+    for (int e2 = 0; e2 < 32; ++e2) {
+        float ds[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int e = 2 * e2 + u;
+            float pv = ex2(fmaf(__uint_as_float(sv[e]), sl2, -lse2));
+            if (kDiag && key0 + e > qrow) pv = 0.f;
+            ds[u] = pv * (__uint_as_float(dv[e]) - dlt);
+        }
+        dd[e2] = pack_bf16x2(ds[0], ds[1]);
+    }
+}
+
 template <int D>
 __device__ void q_elementwise(BwSync &sy, uint32_t tmem, const BwGrid &g, int32_t *status) {
     using S = BwShape<D>;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int r = warp * 32 + lane;
-    const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+    const int quad = warp & 3, half = warp >> 2;
+    const int r = quad * 32 + lane;
+    const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
+    const int col0 = 64 * half;                  // this warp's 64 key columns
     int sc = 0, ac = 0;
     bool ok = true;
     // this row's log-sum-exp and Delta, fetched one item ahead
@@ -481,26 +540,20 @@ __device__ void q_elementwise(BwSync &sy, uint32_t tmem, const BwGrid &g, int32_
             if (!ok) break;
             ++sc;
             ptx::tc_fence_after();
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                uint32_t sv[32], dv[32];
-                ptx::tmem_ld32(lane_addr + S::kColS + 32 * c, sv);
-                ptx::tmem_ld32(lane_addr + S::kColDP + 32 * c, dv);
-                ptx::tmem_wait_ld();
-                uint32_t dd[16];
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    float ds[2];
-#pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        float pv = ex2(fmaf(__uint_as_float(sv[2 * e + u]), g.scale_log2, -lse2));
-                        if (j == i && j * 128 + 32 * c + 2 * e + u > qrow) pv = 0.f;
-                        ds[u] = pv * (__uint_as_float(dv[2 * e + u]) - dlt);
-                    }
-                    dd[e] = pack_bf16x2(ds[0], ds[1]);
-                }
-                ptx::tmem_st16(lane_addr + S::kColDP + 16 * c, dd);
-            }
+            uint32_t sv[64], dv[64];
+            ptx::tmem_ld32(lane_addr + S::kColS + col0, *reinterpret_cast<uint32_t(*)[32]>(sv));
+            ptx::tmem_ld32(lane_addr + S::kColS + col0 + 32, *reinterpret_cast<uint32_t(*)[32]>(sv + 32));
+            ptx::tmem_ld32(lane_addr + S::kColDP + col0, *reinterpret_cast<uint32_t(*)[32]>(dv));
+            ptx::tmem_ld32(lane_addr + S::kColDP + col0 + 32, *reinterpret_cast<uint32_t(*)[32]>(dv + 32));
+            ptx::tmem_wait_ld();
+            ew_sync();            // every dP column is in registers before any store
+            uint32_t dd[32];
+            if (j == i)
+                q_block<true>(sv, dv, j * 128 + col0, qrow, g.scale_log2, lse2, dlt, dd);
+            else
+                q_block<false>(sv, dv, j * 128 + col0, qrow, g.scale_log2, lse2, dlt, dd);
+            ptx::tmem_st16(lane_addr + S::kColDP + col0 / 2, *reinterpret_cast<uint32_t(*)[16]>(dd));
+            ptx::tmem_st16(lane_addr + S::kColDP + col0 / 2 + 16, *reinterpret_cast<uint32_t(*)[16]>(dd + 16));
             ptx::tmem_wait_st();
             ptx::tc_fence_before();
             __syncwarp();
@@ -512,8 +565,7 @@ __device__ void q_elementwise(BwSync &sy, uint32_t tmem, const BwGrid &g, int32_
         ++ac;
         ptx::tc_fence_after();
         uint16_t *dst = g.d0 + (((size_t)b * g.T + qrow) * g.Hq + h) * D;
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = half; c < D / 32; c += 2) {
             uint32_t a[32];
             ptx::tmem_ld32(lane_addr + S::kColAcc0 + 32 * c, a);
             ptx::tmem_wait_ld();
@@ -548,9 +600,9 @@ __device__ __forceinline__ void bw_setup(BwSync &sy) {
             ptx::mbar_init(A(sy.st_empty[s]), 1);
         }
         ptx::mbar_init(A(sy.s_full), 1);
-        ptx::mbar_init(A(sy.p_full), 4);       // one elected lane per elementwise warp
+        ptx::mbar_init(A(sy.p_full), kEwWarps);     // one elected lane per elementwise warp
         ptx::mbar_init(A(sy.acc_full), 1);
-        ptx::mbar_init(A(sy.acc_empty), 4);
+        ptx::mbar_init(A(sy.acc_empty), kEwWarps);
         ptx::mbar_init(A(sy.mma_done), 1);
         ptx::fence_barrier_init();
     }
@@ -584,13 +636,17 @@ bwd_kv_kernel(const __grid_constant__ BwMaps maps, BwGrid g, int32_t *status) {
     // Delta (and the forward's outputs) come from the kernels before this one.
     asm volatile("griddepcontrol.wait;" ::: "memory");
     const uint32_t tmem = sy.tmem_base;
-    if (warp == kBwTmaWarp) {
-        if (lane == 0) kv_producer<D>(maps, sy, smem, g, status);
-        __syncwarp();
-    } else if (warp == kBwMmaWarp) {
-        if (lane == 0) kv_mma<D>(sy, smem, tmem, g, status);
-        __syncwarp();
+    if (warp >= kEwWarps) {
+        ptx::regs_dec<kBwCtlRegs>();
+        if (warp == kBwTmaWarp) {
+            if (lane == 0) kv_producer<D>(maps, sy, smem, g, status);
+            __syncwarp();
+        } else if (warp == kBwMmaWarp) {
+            if (lane == 0) kv_mma<D>(sy, smem, tmem, g, status);
+            __syncwarp();
+        }
     } else {
+        ptx::regs_inc<kBwEwRegs>();
         kv_elementwise<D>(sy, smem, tmem, g, status);
     }
     bw_teardown(sy);
@@ -607,13 +663,17 @@ bwd_q_kernel(const __grid_constant__ BwMaps maps, BwGrid g, int32_t *status) {
     bw_setup(sy);
     asm volatile("griddepcontrol.wait;" ::: "memory");
     const uint32_t tmem = sy.tmem_base;
-    if (warp == kBwTmaWarp) {
-        if (lane == 0) q_producer<D>(maps, sy, smem, g, status);
-        __syncwarp();
-    } else if (warp == kBwMmaWarp) {
-        if (lane == 0) q_mma<D>(sy, smem, tmem, g, status);
-        __syncwarp();
+    if (warp >= kEwWarps) {
+        ptx::regs_dec<kBwCtlRegs>();
+        if (warp == kBwTmaWarp) {
+            if (lane == 0) q_producer<D>(maps, sy, smem, g, status);
+            __syncwarp();
+        } else if (warp == kBwMmaWarp) {
+            if (lane == 0) q_mma<D>(sy, smem, tmem, g, status);
+            __syncwarp();
+        }
     } else {
+        ptx::regs_inc<kBwEwRegs>();
         q_elementwise<D>(sy, tmem, g, status);
     }
     bw_teardown(sy);
@@ -692,15 +752,25 @@ gqa_status launch_backward(const void *q, const void *k, const void *v, const vo
         pdl[0].val.programmaticStreamSerializationAllowed = 1;
         cudaLaunchConfig_t cfg = {};
         const long long rows = (long long)B * T * Hq;
-        cfg.gridDim = dim3((unsigned)((rows + 7) / 8));
+        const int tpr = D / 8 > 8 ? 16 : 8;
+        cfg.gridDim = dim3((unsigned)((rows * tpr + 255) / 256));
         cfg.blockDim = dim3(256);
         cfg.stream = s;
         cfg.attrs = pdl;
         cfg.numAttrs = 1;
-        if (cudaLaunchKernelEx(&cfg, delta_kernel, static_cast<const uint16_t *>(out),
-                               static_cast<const uint16_t *>(dout), delta, B, T, Hq, D, ls) !=
+        if (cudaLaunchKernelEx(&cfg, delta_kernel<D>, static_cast<const uint16_t *>(out),
+                               static_cast<const uint16_t *>(dout), delta, B, T, Hq, ls) !=
             cudaSuccess)
             return GQA_ERR_CUDA;
+    }
+    // The warpgroup register split assumes 168 registers per thread at launch;
+    // with any other count the increases could not be met, so refuse.
+    {
+        cudaFuncAttributes a1, a2;
+        if (cudaFuncGetAttributes(&a1, bwd_kv_kernel<D>) != cudaSuccess ||
+            cudaFuncGetAttributes(&a2, bwd_q_kernel<D>) != cudaSuccess)
+            return GQA_ERR_CUDA;
+        if (a1.numRegs != 168 || a2.numRegs != 168) return GQA_ERR_UNSUPPORTED;
     }
     // 2. dK, dV
     {

@@ -296,16 +296,15 @@ decode_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ kc,
 }
 
 // Merge the chunks of one (b, query head): one CTA per row, one thread per output
-// coordinate.  Warp 0 turns the chunks' maxima into weights 2^(m_i - M) in shared
-// memory; then every thread walks the chunks with independent coalesced loads.
-constexpr int kCombMaxStored = 1024;      // chunk weights kept in shared memory
-
+// coordinate.  No barrier and one round trip to memory: each thread issues the
+// loads of its coordinate of up to 32 chunk partials at once, while every warp
+// reduces the chunk maxima and sums on its own with shuffles; the weights
+// 2^(m_i - M) then reach the threads by shuffle.  Rows of more than 32 chunks
+// repeat this per group of 32.
 __global__ void __launch_bounds__(128)
 decode_merge_kernel(const float *__restrict__ ws_ml, const float *__restrict__ ws_o,
                     const int32_t *__restrict__ lens, int max_len, int Hq, int D, int Lmax,
                     int n_splits, uint16_t *__restrict__ out) {
-    __shared__ float wsplit[kCombMaxStored];
-    __shared__ float stats[2];
     asm volatile("griddepcontrol.wait;" ::: "memory");
     const int row = blockIdx.x;                   // b * Hq + h
     const int b = row / Hq;
@@ -318,36 +317,29 @@ decode_merge_kernel(const float *__restrict__ ws_ml, const float *__restrict__ w
     }
     const int ns = (len + kDecCH - 1) / kDecCH;
     const float *ml = ws_ml + (size_t)row * n_splits * 2;
-    const float *po = ws_o + (size_t)row * n_splits * D;
-    const bool stored = ns <= kCombMaxStored;
-    if (tid < 32) {
-        float M = -INFINITY;
-        for (int i = lane; i < ns; i += 32) M = fmaxf(M, ml[2 * i]);
-        M = warp_max(M);
-        float L = 0.f;
-        for (int i = lane; i < ns; i += 32) {
-            const float w = ex2(ml[2 * i] - M);
-            if (stored) wsplit[i] = w;
-            L = fmaf(w, ml[2 * i + 1], L);
+    const float *po = ws_o + (size_t)row * n_splits * D + tid;
+    const bool live = tid < D;
+    float M = -INFINITY;
+    for (int i = lane; i < ns; i += 32) M = fmaxf(M, ml[2 * i]);
+    M = warp_max(M);
+    float acc = 0.f, L = 0.f;
+    for (int base = 0; base < ns; base += 32) {
+        const int n = min(32, ns - base);
+        float pv[32];
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj)
+            pv[jj] = (live && jj < n) ? po[(size_t)(base + jj) * D] : 0.f;
+        float w = 0.f;
+        if (lane < n) {
+            const float2 mi = *reinterpret_cast<const float2 *>(ml + 2 * (base + lane));
+            w = ex2(mi.x - M);
+            L = fmaf(w, mi.y, L);
         }
-        L = warp_sum(L);
-        if (lane == 0) {
-            stats[0] = M;
-            stats[1] = L;
-        }
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj) acc = fmaf(__shfl_sync(0xffffffffu, w, jj), pv[jj], acc);
     }
-    __syncthreads();
-    const float M = stats[0], inv = 1.f / stats[1];
-    for (int d = tid; d < D; d += blockDim.x) {
-        float acc = 0.f;
-        if (stored) {
-#pragma unroll 8
-            for (int i = 0; i < ns; ++i) acc = fmaf(wsplit[i], po[(size_t)i * D + d], acc);
-        } else {
-            for (int i = 0; i < ns; ++i) acc = fmaf(ex2(ml[2 * i] - M), po[(size_t)i * D + d], acc);
-        }
-        o[d] = (uint16_t)(pack_bf16x2(acc * inv, 0.f) & 0xffffu);
-    }
+    L = warp_sum(L);
+    if (live) o[tid] = (uint16_t)(pack_bf16x2(acc / L, 0.f) & 0xffffu);
 }
 
 template <int D, int G>
