@@ -15,15 +15,21 @@
 // Three launches:
 //   delta_kernel   Delta[b, h, t] = sum_d dO * O (HBM-bound, 16-byte loads);
 //   bwd_kv_kernel  per (b, KV head, 128-key tile j), persistent: for every query
-//                  head of the group and every query tile i >= j,
-//                    S^T = K_j Q_i^T, dP^T = V_j dO_i^T       (two SS MMAs)
-//                    P^T, dS^T in bf16 over S^T, dP^T in TMEM  (4 warps, thread = key)
-//                    dV_j += P^T dO_i, dK_j += dS^T Q_i         (two TS MMAs)
+//                  head of the group and every query tile i >= j, in halves of 64
+//                  queries,
+//                    S^T = K_j Q^T, dP^T = V_j dO^T            (two SS MMAs)
+//                    P^T, dS^T in bf16 over S^T, dP^T in TMEM  (thread = key)
+//                    dV_j += P^T dO, dK_j += dS^T Q             (two TS MMAs)
 //                  dK_j and dV_j stay in tensor memory until the tile is done, so
 //                  the group's sum needs no atomics;
 //   bwd_q_kernel   per (b, query head, 128-query tile i), persistent: for every
 //                  key tile j <= i,  S = Q_i K_j^T, dP = dO_i V_j^T, dS in bf16 over
 //                  dP, dQ_i += dS K_j.
+// The dK/dV kernel keeps two halves in flight (S^T / dP^T double-buffered in
+// tensor memory), so the tensor core works on one while the elementwise warps
+// work on the other.  The dQ kernel has no room for a second buffer next to dQ
+// and runs tile by tile (with 64-key halves its N = 64 MMAs re-read the whole
+// Q / dO operand per half and are bound by shared-memory bandwidth: slower).
 // The same shared-memory tile serves as a K-major operand (the contraction over
 // D) and as an MN-major one (the contraction over its rows), as in the forward
 // kernel.  Warp roles (384 threads, three warpgroups): warps 0-7 elementwise +
@@ -78,7 +84,8 @@ struct BwMaps {
 struct BwSync {
     uint64_t fixed_full, fixed_empty;          // K_j/V_j (dK/dV kernel) or Q_i/dO_i (dQ kernel)
     uint64_t st_full[2], st_empty[2];          // the ring
-    uint64_t s_full, p_full, acc_full, acc_empty;
+    uint64_t s_full, p_full, acc_full, acc_empty;   // dQ kernel: one tile at a time
+    uint64_t h_full[2], h_done[2];                  // dK/dV kernel: two 64-query halves
     uint64_t mma_done;
     uint32_t tmem_base;
 };
@@ -115,6 +122,30 @@ struct BwMma {
         constexpr uint32_t id = ptx::idesc_bf16_f32(128, D, true);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
+            ptx::mma_ts(d, a_tmem + ks * 8, ptx::smem_desc_sw128(b + ks * 2048, S::kBlockBytes, 1024),
+                        id, (acc || ks > 0) ? 1u : 0u);
+    }
+};
+
+// MMAs on halves of a 128-row tile (64 rows at a time), for the dK/dV pipeline.
+template <int D>
+struct BwMmaHalf {
+    using S = BwShape<D>;
+    // D(tmem, 128 x 64) = A(smem, K-major 128 x D) . B(smem, 64 rows of a K-major tile)^T
+    static __device__ __forceinline__ void ss(uint32_t d, uint32_t a, uint32_t b) {
+        constexpr uint32_t id = ptx::idesc_bf16_f32(128, 64, false);
+#pragma unroll
+        for (int ks = 0; ks < S::kKSteps; ++ks) {
+            const uint32_t off = (ks >> 2) * S::kBlockBytes + (ks & 3) * 32;
+            ptx::mma_ss(d, ptx::smem_desc_sw128(a + off, 16, 1024),
+                        ptx::smem_desc_sw128(b + off, 16, 1024), id, ks > 0);
+        }
+    }
+    // D(tmem, 128 x D) (+)= A(tmem, bf16 128 x 64) . B(smem, 64 rows x D, MN-major)
+    static __device__ __forceinline__ void ts(uint32_t d, uint32_t a_tmem, uint32_t b, bool acc) {
+        constexpr uint32_t id = ptx::idesc_bf16_f32(128, D, true);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
             ptx::mma_ts(d, a_tmem + ks * 8, ptx::smem_desc_sw128(b + ks * 2048, S::kBlockBytes, 1024),
                         id, (acc || ks > 0) ? 1u : 0u);
     }
@@ -217,14 +248,29 @@ __device__ void kv_producer(const BwMaps &maps, BwSync &sy, uint8_t *smem, const
     }
 }
 
+// The tile's queries are taken in two halves of 64 with S^T / dP^T of half u in
+// tensor-memory buffer u % 2 (columns [128 (u % 2), 128 (u % 2) + 128): S^T then
+// dP^T, 64 columns each), so the tensor core computes dV/dK of one half and
+// S^T/dP^T of the next while the elementwise warps work on the other half.
 template <int D>
 __device__ void kv_mma(BwSync &sy, uint8_t *smem, uint32_t tmem, const BwGrid &g, int32_t *status) {
     using S = BwShape<D>;
-    using M = BwMma<D>;
+    using M = BwMmaHalf<D>;
     const int grp = g.Hq / g.Hkv;
     const uint32_t k_base = ptx::smem_addr(smem), v_base = k_base + S::kTileBytes;
-    int ic = 0, sc = 0, pc = 0, ac = 0;
+    int ic = 0, sc = 0, hc = 0, ac = 0;    // items, stages and halves consumed, accumulators
     bool ok = true;
+    auto stage_base = [&](int st) {
+        return ptx::smem_addr(smem + S::kOffStage + st * S::kStageBytes);
+    };
+    // S^T / dP^T of half u (stage st, 64-row half h) into buffer u % 2
+    auto issue_scores = [&](int u, int st, int h) {
+        const uint32_t buf = tmem + 128 * (u & 1);
+        const uint32_t qb = stage_base(st) + h * 64 * 128;
+        M::ss(buf, k_base, qb);                          // S^T  = K_j Q_half^T
+        M::ss(buf + 64, v_base, qb + S::kTileBytes);     // dP^T = V_j dO_half^T
+        ptx::mma_commit(A(sy.h_full[u & 1]));
+    };
     for (int w = blockIdx.x; w < g.n_items && ok; w += gridDim.x) {
         int b, kvh, j;
         kv_item(w, g, b, kvh, j);
@@ -232,33 +278,43 @@ __device__ void kv_mma(BwSync &sy, uint8_t *smem, uint32_t tmem, const BwGrid &g
         if (!ok) break;
         ++ic;
         ptx::tc_fence_after();
-        bool first = true;
-        const int steps = grp * (g.nT - j);
-        for (int s = 0; s < steps && ok; ++s) {
-            const int st = sc % S::kStages;
-            ok = ptx::mbar_wait(A(sy.st_full[st]), (sc / S::kStages) & 1);
+        const int n_half = 2 * grp * (g.nT - j);        // halves of this item
+        const int sc0 = sc;
+        // prologue: the scores of the first two halves (one stage)
+        ok = ptx::mbar_wait(A(sy.st_full[sc0 % S::kStages]), (sc0 / S::kStages) & 1);
+        if (!ok) break;
+        ptx::tc_fence_after();
+        issue_scores(hc, sc0 % S::kStages, 0);
+        issue_scores(hc + 1, sc0 % S::kStages, 1);
+        for (int x = 0; x < n_half && ok; ++x) {
+            const int u = hc + x;
+            const int st = (sc0 + x / 2) % S::kStages;
+            ok = ptx::mbar_wait(A(sy.h_done[u & 1]), (u >> 1) & 1);   // P^T, dS^T of half u
             if (!ok) break;
-            ptx::tc_fence_after();
-            const uint32_t q_base = ptx::smem_addr(smem + S::kOffStage + st * S::kStageBytes);
-            const uint32_t do_base = q_base + S::kTileBytes;
-            M::ss(tmem + S::kColS, k_base, q_base);      // S^T  = K_j Q_i^T
-            M::ss(tmem + S::kColDP, v_base, do_base);    // dP^T = V_j dO_i^T
-            ptx::mma_commit(A(sy.s_full));
-            ok = ptx::mbar_wait(A(sy.p_full), pc & 1);
-            if (!ok) break;
-            ++pc;
-            if (first) {        // the previous item's epilogue has read dK, dV
+            if (x == 0) {       // the previous item's epilogue has read dK, dV
                 ok = ptx::mbar_wait(A(sy.acc_empty), (ac & 1) ^ 1);
                 if (!ok) break;
             }
             ptx::tc_fence_after();
-            M::ts(tmem + S::kColAcc0, tmem + S::kColS, do_base, !first);   // dV += P^T dO_i
-            M::ts(tmem + S::kColAcc1, tmem + S::kColDP, q_base, !first);   // dK += dS^T Q_i
-            ptx::mma_commit(A(sy.st_empty[st]));
-            first = false;
-            ++sc;
+            const uint32_t buf = tmem + 128 * (u & 1);
+            const uint32_t qb = stage_base(st) + (x & 1) * 64 * 128;
+            M::ts(tmem + S::kColAcc0, buf, qb + S::kTileBytes, x > 0);   // dV += P^T dO_half
+            M::ts(tmem + S::kColAcc1, buf + 64, qb, x > 0);              // dK += dS^T Q_half
+            if (x & 1) ptx::mma_commit(A(sy.st_empty[st]));              // both halves done
+            // the scores of half u + 2 go into the buffer just consumed
+            if (x + 2 < n_half) {
+                const int st2 = (sc0 + (x + 2) / 2) % S::kStages;
+                if (!(x & 1)) {
+                    ok = ptx::mbar_wait(A(sy.st_full[st2]), ((sc0 + (x + 2) / 2) / S::kStages) & 1);
+                    if (!ok) break;
+                    ptx::tc_fence_after();
+                }
+                issue_scores(u + 2, st2, x & 1);
+            }
         }
         if (!ok) break;
+        hc += n_half;
+        sc += n_half / 2;
         ptx::mma_commit(A(sy.acc_full));
         ptx::mma_commit(A(sy.fixed_empty));
         ++ac;
@@ -268,20 +324,20 @@ __device__ void kv_mma(BwSync &sy, uint8_t *smem, uint32_t tmem, const BwGrid &g
     ptx::mbar_wait(A(sy.mma_done), 0);
 }
 
-// Elementwise step of the dK/dV kernel: thread = key row r of tile j, columns =
-// the queries of tile i; warp w takes lane quadrant w % 4 and columns
-// [64 (w / 4), 64 (w / 4) + 64).  Both warps of a quadrant load their S^T and dP^T
-// columns before either writes P^T / dS^T over them (the packed bf16 halves land
-// on the lower columns), hence the barrier between loads and stores.
+// Elementwise work of the dK/dV kernel on one 64-query half: thread = key row r
+// of tile j; warp w takes lane quadrant w % 4 and the half's columns
+// [32 (w / 4), 32 (w / 4) + 32).  Both warps of a quadrant load their S^T and
+// dP^T columns before either stores P^T / dS^T (packed bf16, on the lower
+// columns) over them, hence the barrier between loads and stores.
 template <int D, bool kEdge>
-__device__ __forceinline__ void kv_block(const uint32_t (&sv)[64], const uint32_t (&dv)[64],
-                                         const float *lse_v, const float *del_v, int col0,
-                                         int qbase, int key, int T, float sl2,
-                                         uint32_t (&pp)[32], uint32_t (&dd)[32]) {
+__device__ __forceinline__ void kv_block(const uint32_t (&sv)[32], const uint32_t (&dv)[32],
+                                         const float *lse_v, const float *del_v, int qbase,
+                                         int key, int T, float sl2, uint32_t (&pp)[16],
+                                         uint32_t (&dd)[16]) {
 #pragma unroll
-    for (int c4 = 0; c4 < 16; ++c4) {
-        const float4 l4 = *reinterpret_cast<const float4 *>(lse_v + col0 + 4 * c4);
-        const float4 d4 = *reinterpret_cast<const float4 *>(del_v + col0 + 4 * c4);
+    for (int c4 = 0; c4 < 8; ++c4) {
+        const float4 l4 = *reinterpret_cast<const float4 *>(lse_v + 4 * c4);
+        const float4 d4 = *reinterpret_cast<const float4 *>(del_v + 4 * c4);
         const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
         const float dl[4] = {d4.x, d4.y, d4.z, d4.w};
         float p[4], ds[4];
@@ -290,7 +346,7 @@ __device__ __forceinline__ void kv_block(const uint32_t (&sv)[64], const uint32_
             const int e = 4 * c4 + u;
             float pv = ex2(fmaf(__uint_as_float(sv[e]), sl2, -lv[u] * kLog2e));
             if (kEdge) {
-                const int query = qbase + col0 + e;
+                const int query = qbase + e;
                 if (query < key || query >= T) pv = 0.f;
             }
             p[u] = pv;
@@ -308,57 +364,56 @@ __device__ void kv_elementwise(BwSync &sy, uint8_t *smem, uint32_t tmem, const B
                                int32_t *status) {
     using S = BwShape<D>;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int quad = warp & 3, half = warp >> 2;
+    const int quad = warp & 3, part = warp >> 2;
     const int r = quad * 32 + lane;
     const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
-    const int col0 = 64 * half;                  // this warp's 64 query columns
     const int grp = g.Hq / g.Hkv;
-    int sc = 0, ac = 0;
+    int hc = 0, sc = 0, ac = 0;
     bool ok = true;
     for (int w = blockIdx.x; w < g.n_items && ok; w += gridDim.x) {
         int b, kvh, j;
         kv_item(w, g, b, kvh, j);
         const int key = j * 128 + r;
-        const int steps = grp * (g.nT - j);
-        for (int s = 0; s < steps && ok; ++s) {
-            const int i = j + s % (g.nT - j);
-            ok = __all_sync(0xffffffffu, ptx::mbar_wait(A(sy.s_full), sc & 1));
+        const int n_half = 2 * grp * (g.nT - j);
+        for (int x = 0; x < n_half && ok; ++x) {
+            const int u = hc + x;
+            const int i = j + (x / 2) % (g.nT - j);
+            const int st = (sc + x / 2) % S::kStages;
+            ok = __all_sync(0xffffffffu, ptx::mbar_wait(A(sy.h_full[u & 1]), (u >> 1) & 1));
             if (!ok) break;
-            const int st = sc % S::kStages;
-            ++sc;
             ptx::tc_fence_after();
+            const int col = 64 * (x & 1) + 32 * part;          // first query column of this warp
             const float *lse_v = reinterpret_cast<const float *>(
-                smem + S::kOffStage + st * S::kStageBytes + 2 * S::kTileBytes);
+                smem + S::kOffStage + st * S::kStageBytes + 2 * S::kTileBytes) + col;
             const float *del_v = lse_v + 128;
-            uint32_t sv[64], dv[64];
-            ptx::tmem_ld32(lane_addr + S::kColS + col0, *reinterpret_cast<uint32_t(*)[32]>(sv));
-            ptx::tmem_ld32(lane_addr + S::kColS + col0 + 32, *reinterpret_cast<uint32_t(*)[32]>(sv + 32));
-            ptx::tmem_ld32(lane_addr + S::kColDP + col0, *reinterpret_cast<uint32_t(*)[32]>(dv));
-            ptx::tmem_ld32(lane_addr + S::kColDP + col0 + 32, *reinterpret_cast<uint32_t(*)[32]>(dv + 32));
+            const uint32_t buf = lane_addr + 128 * (u & 1);
+            uint32_t sv[32], dv[32];
+            ptx::tmem_ld32(buf + 32 * part, sv);
+            ptx::tmem_ld32(buf + 64 + 32 * part, dv);
             ptx::tmem_wait_ld();
-            ew_sync();            // every S^T / dP^T column is in registers before any store
-            uint32_t pp[32], dd[32];
+            ew_sync();
+            uint32_t pp[16], dd[16];
             if (i == j || (i + 1) * 128 > g.T)                   // some (query, key) masked
-                kv_block<D, true>(sv, dv, lse_v, del_v, col0, i * 128, key, g.T, g.scale_log2, pp, dd);
+                kv_block<D, true>(sv, dv, lse_v, del_v, i * 128 + col, key, g.T, g.scale_log2, pp, dd);
             else
-                kv_block<D, false>(sv, dv, lse_v, del_v, col0, i * 128, key, g.T, g.scale_log2, pp, dd);
-            ptx::tmem_st16(lane_addr + S::kColS + col0 / 2, *reinterpret_cast<uint32_t(*)[16]>(pp));
-            ptx::tmem_st16(lane_addr + S::kColS + col0 / 2 + 16, *reinterpret_cast<uint32_t(*)[16]>(pp + 16));
-            ptx::tmem_st16(lane_addr + S::kColDP + col0 / 2, *reinterpret_cast<uint32_t(*)[16]>(dd));
-            ptx::tmem_st16(lane_addr + S::kColDP + col0 / 2 + 16, *reinterpret_cast<uint32_t(*)[16]>(dd + 16));
+                kv_block<D, false>(sv, dv, lse_v, del_v, i * 128 + col, key, g.T, g.scale_log2, pp, dd);
+            ptx::tmem_st16(buf + 16 * part, pp);
+            ptx::tmem_st16(buf + 64 + 16 * part, dd);
             ptx::tmem_wait_st();
             ptx::tc_fence_before();
             __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(A(sy.p_full));
+            if (lane == 0) ptx::mbar_arrive(A(sy.h_done[u & 1]));
         }
         if (!ok) break;
+        hc += n_half;
+        sc += n_half / 2;
         // epilogue: dV_j and c dK_j rows to global memory, half of D per warp
         ok = __all_sync(0xffffffffu, ptx::mbar_wait(A(sy.acc_full), ac & 1));
         if (!ok) break;
         ++ac;
         ptx::tc_fence_after();
         const size_t row = ((size_t)b * g.Hkv + kvh) * g.Lmax + key;
-        for (int c = half; c < D / 32; c += 2) {
+        for (int c = part; c < D / 32; c += 2) {
             uint32_t va[32], ka[32];
             ptx::tmem_ld32(lane_addr + S::kColAcc0 + 32 * c, va);
             ptx::tmem_ld32(lane_addr + S::kColAcc1 + 32 * c, ka);
@@ -374,9 +429,9 @@ __device__ void kv_elementwise(BwSync &sy, uint8_t *smem, uint32_t tmem, const B
                 uint4 *dvp = reinterpret_cast<uint4 *>(g.d1 + row * D + 32 * c);
                 uint4 *dkp = reinterpret_cast<uint4 *>(g.d0 + row * D + 32 * c);
 #pragma unroll
-                for (int x = 0; x < 4; ++x) {
-                    dvp[x] = make_uint4(wv[4 * x], wv[4 * x + 1], wv[4 * x + 2], wv[4 * x + 3]);
-                    dkp[x] = make_uint4(wk[4 * x], wk[4 * x + 1], wk[4 * x + 2], wk[4 * x + 3]);
+                for (int y = 0; y < 4; ++y) {
+                    dvp[y] = make_uint4(wv[4 * y], wv[4 * y + 1], wv[4 * y + 2], wv[4 * y + 3]);
+                    dkp[y] = make_uint4(wk[4 * y], wk[4 * y + 1], wk[4 * y + 2], wk[4 * y + 3]);
                 }
             }
         }
@@ -603,6 +658,10 @@ __device__ __forceinline__ void bw_setup(BwSync &sy) {
         ptx::mbar_init(A(sy.p_full), kEwWarps);     // one elected lane per elementwise warp
         ptx::mbar_init(A(sy.acc_full), 1);
         ptx::mbar_init(A(sy.acc_empty), kEwWarps);
+        for (int h = 0; h < 2; ++h) {
+            ptx::mbar_init(A(sy.h_full[h]), 1);
+            ptx::mbar_init(A(sy.h_done[h]), kEwWarps);
+        }
         ptx::mbar_init(A(sy.mma_done), 1);
         ptx::fence_barrier_init();
     }

@@ -104,8 +104,9 @@ __device__ __forceinline__ uint32_t A(const uint64_t &b) { return ptx::smem_addr
 // covers.  Items are numbered longest first (pairs nearer the end of the
 // chunk see more keys), with the heads of one KV group side by side.
 // Kernel modes: a prompt from position 0, a continuation chunk after a cached
-// prefix, or a prompt of packed documents.
-constexpr int kPrompt = 0, kChunkMode = 1, kDocs = 2;
+// prefix, a prompt of packed documents, or a prompt that also stores each row's
+// log-sum-exp for the backward.
+constexpr int kPrompt = 0, kChunkMode = 1, kDocs = 2, kPromptLse = 3;
 
 struct PfItem {
     int b, h, kvh, q0, n0, n1, n_kv;
@@ -516,7 +517,7 @@ __device__ void softmax_tile(PfSync &sy, uint8_t *smem, uint32_t tmem, int t, co
         ptx::tc_fence_after();
         const float inv_l = 1.f / l;
         uint16_t *dst = out + (((size_t)I.b * T + qrow) * g.Hq + I.h) * D;
-        if (kMode == kPrompt && g.lse && qrow < T)   // natural-log LSE of the scaled scores
+        if (kMode == kPromptLse && qrow < T)   // natural-log LSE of the scaled scores
             g.lse[((size_t)I.b * g.Hq + I.h) * g.lse_stride + qrow] =
                 (m + log2f(l)) * 0.69314718055994531f;
 #pragma unroll
@@ -654,7 +655,8 @@ gqa_status launch_prefill(const void *q, const void *kc, const void *vc, void *o
         if (!encode(&maps.v, vc, 3, dims, str, box)) return GQA_ERR_CUDA;
     }
     auto kern = pos0 ? prefill_kernel<D, kChunkMode>
-                     : (doc_start ? prefill_kernel<D, kDocs> : prefill_kernel<D, kPrompt>);
+                     : doc_start ? prefill_kernel<D, kDocs>
+                     : lse ? prefill_kernel<D, kPromptLse> : prefill_kernel<D, kPrompt>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kSmem) !=
         cudaSuccess)
         return GQA_ERR_CUDA;
