@@ -291,6 +291,15 @@ gqa_status gqa_decode_noalloc(const void *q, const void *k_cache, const void *v_
                               int Hkv, int D, int Lmax, float scale, int32_t *status_dev,
                               void *stream);
 
+/*
+ * gqa_selftest_bounded_wait -- checks the failure path of the bounded waits
+ * without a fault: one thread waits, for limit_ms (1 .. 10000), on an mbarrier
+ * that nothing arrives on, gives up and ORs GQA_DEV_TIMEOUT into *status_dev
+ * (required).  The context stays usable.  The paper has no counterpart of this
+ * call; it is a property of this library.
+ */
+gqa_status gqa_selftest_bounded_wait(int32_t *status_dev, int limit_ms, void *stream);
+
 /* Static, human-readable text for a status code. */
 const char *gqa_status_string(gqa_status s);
 

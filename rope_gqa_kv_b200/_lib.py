@@ -68,6 +68,7 @@ SIGNATURES = {
                         _vp, _vp]),
     "gqa_decode_workspace_bytes": (_sz, [_i, _i, _i, _i]),
     "gqa_decode_noalloc": (_i, [_vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _f, _vp, _vp]),
+    "gqa_selftest_bounded_wait": (_i, [_vp, _i, _vp]),
     "gqa_status_string": (ctypes.c_char_p, [_i]),
     "gqa_version": (_i, []),
 }

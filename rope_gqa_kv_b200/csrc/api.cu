@@ -1,5 +1,6 @@
-// api.cu -- status strings and version of the libgqa C ABI.
+// api.cu -- status strings, version, and the bounded-wait self-test of the libgqa C ABI.
 #include "common.cuh"
+#include "ptx.cuh"
 
 extern "C" const char *gqa_status_string(gqa_status s) {
     switch (s) {
@@ -15,3 +16,24 @@ extern "C" const char *gqa_status_string(gqa_status s) {
 }
 
 extern "C" int gqa_version(void) { return 200; }
+
+// One thread waits on an mbarrier that nothing arrives on.  The wait is the one
+// every kernel of the library uses, with its limit shortened to limit_ns: it
+// gives up, and the thread raises GQA_DEV_TIMEOUT instead of hanging.
+__global__ void selftest_wait_kernel(int32_t *status, unsigned long long limit_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    const uint32_t b = gqa::ptx::smem_addr(&bar);
+    gqa::ptx::mbar_init(b, 1);
+    gqa::ptx::fence_barrier_init();
+    const uint64_t t0 = gqa::ptx::globaltimer();
+    bool done = gqa::ptx::mbar_try_wait(b, 0);
+    while (!done && gqa::ptx::globaltimer() - t0 < limit_ns) done = gqa::ptx::mbar_try_wait(b, 0);
+    if (!done) gqa::report(status, GQA_DEV_TIMEOUT);
+}
+
+extern "C" gqa_status gqa_selftest_bounded_wait(int32_t *status_dev, int limit_ms, void *stream) {
+    if (!status_dev || limit_ms < 1 || limit_ms > 10000) return GQA_ERR_INVALID_ARG;
+    selftest_wait_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(
+        status_dev, (unsigned long long)limit_ms * 1000000ull);
+    return gqa_host::launch_status();
+}

@@ -159,6 +159,12 @@ def test_backward_validation(lib):
     assert lib.gqa_prefill_lse(f, f, f, f, None, 1, 10, 4, 2, 64, 128, 0.0, None, None) == 1
 
 
+def test_selftest_validation(lib):
+    assert lib.gqa_selftest_bounded_wait(None, 10, None) == 1
+    assert lib.gqa_selftest_bounded_wait(FAKE, 0, None) == 1
+    assert lib.gqa_selftest_bounded_wait(FAKE, 20000, None) == 1
+
+
 def test_decode_validation(lib):
     f = FAKE
     ws = ctypes.c_size_t(1 << 20)
