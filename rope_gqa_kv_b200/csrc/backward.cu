@@ -100,6 +100,13 @@ struct BwGrid {
 
 __device__ __forceinline__ uint32_t A(const uint64_t &b) { return ptx::smem_addr(&b); }
 
+// The k-th item of this CTA: items are numbered longest first and dealt out in
+// rounds of gridDim.x in snake order (every other round backwards).
+__device__ __forceinline__ int bw_w(int k) {
+    const int G = gridDim.x, c = blockIdx.x;
+    return k * G + ((k & 1) ? G - 1 - c : c);
+}
+
 __device__ __forceinline__ void ew_sync() {
     asm volatile("bar.sync %0, %1;" ::"n"(kEwBarrier), "n"(kEwWarps * 32) : "memory");
 }
@@ -204,7 +211,7 @@ __device__ void kv_producer(const BwMaps &maps, BwSync &sy, uint8_t *smem, const
     const int grp = g.Hq / g.Hkv;
     int ic = 0, sc = 0;
     bool ok = true;
-    for (int w = blockIdx.x; w < g.n_items && ok; w += gridDim.x) {
+    for (int kk = 0, w = bw_w(0); w < g.n_items && ok; w = bw_w(++kk)) {
         int b, kvh, j;
         kv_item(w, g, b, kvh, j);
         ok = ptx::mbar_wait(A(sy.fixed_empty), (ic & 1) ^ 1);
@@ -271,7 +278,7 @@ __device__ void kv_mma(BwSync &sy, uint8_t *smem, uint32_t tmem, const BwGrid &g
         M::ss(buf + 64, v_base, qb + S::kTileBytes);     // dP^T = V_j dO_half^T
         ptx::mma_commit(A(sy.h_full[u & 1]));
     };
-    for (int w = blockIdx.x; w < g.n_items && ok; w += gridDim.x) {
+    for (int kk = 0, w = bw_w(0); w < g.n_items && ok; w = bw_w(++kk)) {
         int b, kvh, j;
         kv_item(w, g, b, kvh, j);
         ok = ptx::mbar_wait(A(sy.fixed_full), ic & 1);
@@ -370,7 +377,7 @@ __device__ void kv_elementwise(BwSync &sy, uint8_t *smem, uint32_t tmem, const B
     const int grp = g.Hq / g.Hkv;
     int hc = 0, sc = 0, ac = 0;
     bool ok = true;
-    for (int w = blockIdx.x; w < g.n_items && ok; w += gridDim.x) {
+    for (int kk = 0, w = bw_w(0); w < g.n_items && ok; w = bw_w(++kk)) {
         int b, kvh, j;
         kv_item(w, g, b, kvh, j);
         const int key = j * 128 + r;
@@ -461,7 +468,7 @@ __device__ void q_producer(const BwMaps &maps, BwSync &sy, uint8_t *smem, const 
     const int grp = g.Hq / g.Hkv;
     int ic = 0, sc = 0;
     bool ok = true;
-    for (int w = blockIdx.x; w < g.n_items && ok; w += gridDim.x) {
+    for (int kk = 0, w = bw_w(0); w < g.n_items && ok; w = bw_w(++kk)) {
         int b, h, i;
         q_item(w, g, b, h, i);
         const int kvh = h / grp;
@@ -506,7 +513,7 @@ __device__ void q_mma(BwSync &sy, uint8_t *smem, uint32_t tmem, const BwGrid &g,
     const uint32_t q_base = ptx::smem_addr(smem), do_base = q_base + S::kTileBytes;
     int ic = 0, sc = 0, pc = 0, ac = 0;
     bool ok = true;
-    for (int w = blockIdx.x; w < g.n_items && ok; w += gridDim.x) {
+    for (int kk = 0, w = bw_w(0); w < g.n_items && ok; w = bw_w(++kk)) {
         int b, h, i;
         q_item(w, g, b, h, i);
         ok = ptx::mbar_wait(A(sy.fixed_full), ic & 1);
@@ -583,12 +590,12 @@ __device__ void q_elementwise(BwSync &sy, uint32_t tmem, const BwGrid &g, int32_
         dl = qrow < g.T ? g.delta[off] : 0.f;
     };
     float nl2 = 0.f, ndl = 0.f;
-    if ((int)blockIdx.x < g.n_items) fetch(blockIdx.x, nl2, ndl);
-    for (int w = blockIdx.x; w < g.n_items && ok; w += gridDim.x) {
+    if (bw_w(0) < g.n_items) fetch(bw_w(0), nl2, ndl);
+    for (int kk = 0, w = bw_w(0); w < g.n_items && ok; w = bw_w(++kk)) {
         int b, h, i;
         q_item(w, g, b, h, i);
         const float lse2 = nl2, dlt = ndl;
-        if (w + (int)gridDim.x < g.n_items) fetch(w + gridDim.x, nl2, ndl);
+        if (bw_w(kk + 1) < g.n_items) fetch(bw_w(kk + 1), nl2, ndl);
         const int qrow = i * 128 + r;
         for (int j = 0; j <= i && ok; ++j) {
             ok = __all_sync(0xffffffffu, ptx::mbar_wait(A(sy.s_full), sc & 1));
