@@ -51,6 +51,23 @@ __device__ __forceinline__ float group_sum(float v) {
     return v;
 }
 
+// Two fp32 lanes at once (one issue slot each): d = a * b, d = a * b + c.
+__device__ __forceinline__ void mul2(float &d0, float &d1, float a0, float a1, float b0, float b1) {
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d0), "=f"(d1)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+__device__ __forceinline__ void fma2(float &d0, float &d1, float a0, float a1, float b0, float b1,
+                                     float c0, float c1) {
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d0), "=f"(d1)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+
 template <int D>
 __device__ __forceinline__ void rotate_vector(const uint4 a_in, const uint4 b_in, uint4 &a_out,
                                               uint4 &b_out, const float *cs, const float *sn,
@@ -67,34 +84,43 @@ __device__ __forceinline__ void rotate_vector(const uint4 a_in, const uint4 b_in
         xb[2 * e + 1] = bf16hi(wb[e]);
     }
     if (qk_norm) {
-        float ss = 0.f;
+        // sum of squares and the scaling on coordinate pairs (packed f32x2)
+        float s0 = 0.f, s1 = 0.f;
         if (active) {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) ss += xa[e] * xa[e] + xb[e] * xb[e];
+            for (int e = 0; e < 8; e += 2) {
+                fma2(s0, s1, xa[e], xa[e + 1], xa[e], xa[e + 1], s0, s1);
+                fma2(s0, s1, xb[e], xb[e + 1], xb[e], xb[e + 1], s0, s1);
+            }
         }
-        ss = group_sum<S::kTPV>(ss);
+        const float ss = group_sum<S::kTPV>(s0 + s1);
         const float inv = rsqrtf(ss * (1.0f / D) + eps);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            xa[e] *= inv;
-            xb[e] *= inv;
+        for (int e = 0; e < 8; e += 2) {
+            mul2(xa[e], xa[e + 1], xa[e], xa[e + 1], inv, inv);
+            mul2(xb[e], xb[e + 1], xb[e], xb[e + 1], inv, inv);
         }
     }
+    // rotation of pairs (8j + 2e, 8j + 2e + 1) two at a time:
+    //   ya = a c - b s,  yb = a s + b c
     uint32_t oa[4], ob[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-        float ya[2], yb[2];
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const int i = 8 * j + 2 * e + u;       // pair index
-            const float c = active ? cs[i] : 0.f;
-            const float s = active ? sn[i] : 0.f;
-            const float a = xa[2 * e + u], b = xb[2 * e + u];
-            ya[u] = a * c - b * s;
-            yb[u] = a * s + b * c;
+        const int i = 8 * j + 2 * e;               // first of the two pair indices
+        float c0 = 0.f, c1 = 0.f, s0 = 0.f, s1 = 0.f;
+        if (active) {
+            const float2 c2 = *reinterpret_cast<const float2 *>(cs + i);
+            const float2 s2 = *reinterpret_cast<const float2 *>(sn + i);
+            c0 = c2.x; c1 = c2.y; s0 = s2.x; s1 = s2.y;
         }
-        oa[e] = pack_bf16x2(ya[0], ya[1]);
-        ob[e] = pack_bf16x2(yb[0], yb[1]);
+        const float a0 = xa[2 * e], a1 = xa[2 * e + 1], b0 = xb[2 * e], b1 = xb[2 * e + 1];
+        float ya0, ya1, yb0, yb1;
+        mul2(ya0, ya1, b0, b1, -s0, -s1);
+        fma2(ya0, ya1, a0, a1, c0, c1, ya0, ya1);
+        mul2(yb0, yb1, b0, b1, c0, c1);
+        fma2(yb0, yb1, a0, a1, s0, s1, yb0, yb1);
+        oa[e] = pack_bf16x2(ya0, ya1);
+        ob[e] = pack_bf16x2(yb0, yb1);
     }
     a_out = make_uint4(oa[0], oa[1], oa[2], oa[3]);
     b_out = make_uint4(ob[0], ob[1], ob[2], ob[3]);
@@ -117,8 +143,8 @@ rope_append_kernel(uint16_t *__restrict__ q, const uint16_t *__restrict__ k,
                    int qk_norm, float eps, const __grid_constant__ RopeTable tab,
                    int32_t *status) {
     using S = RopeShape<D>;
-    __shared__ float cs[TB][S::kHalf];
-    __shared__ float sn[TB][S::kHalf];
+    __shared__ __align__(16) float cs[TB][S::kHalf];
+    __shared__ __align__(16) float sn[TB][S::kHalf];
     // A kernel launched after this one as a programmatic dependent (the prefill
     // or the decode) may start its prologue now; it waits for this grid to
     // complete before it reads anything written here.
