@@ -68,10 +68,29 @@ __device__ __forceinline__ void fma2(float &d0, float &d1, float a0, float a1, f
         : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
 }
 
+// cos / sin (times the YaRN factor) of the 8 rotation pairs 8j .. 8j+7 that
+// lane j of a vector group owns, read from a row of D/2 angles in shared memory;
+// zero on lanes that own no pair.
+template <int D>
+__device__ __forceinline__ void lane_angles(const float *cs_row, const float *sn_row, int j,
+                                            bool active, float (&c)[8], float (&sv)[8]) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        float4 cv = make_float4(0.f, 0.f, 0.f, 0.f), sq = cv;
+        if (active) {
+            cv = *reinterpret_cast<const float4 *>(cs_row + 8 * j + 4 * h);
+            sq = *reinterpret_cast<const float4 *>(sn_row + 8 * j + 4 * h);
+        }
+        c[4 * h] = cv.x; c[4 * h + 1] = cv.y; c[4 * h + 2] = cv.z; c[4 * h + 3] = cv.w;
+        sv[4 * h] = sq.x; sv[4 * h + 1] = sq.y; sv[4 * h + 2] = sq.z; sv[4 * h + 3] = sq.w;
+    }
+}
+
 template <int D>
 __device__ __forceinline__ void rotate_vector(const uint4 a_in, const uint4 b_in, uint4 &a_out,
-                                              uint4 &b_out, const float *cs, const float *sn,
-                                              int j, bool active, bool qk_norm, float eps) {
+                                              uint4 &b_out, const float (&c)[8],
+                                              const float (&sv)[8], bool active, bool qk_norm,
+                                              float eps) {
     using S = RopeShape<D>;
     float xa[8], xb[8];
     const uint32_t wa[4] = {a_in.x, a_in.y, a_in.z, a_in.w};
@@ -106,13 +125,7 @@ __device__ __forceinline__ void rotate_vector(const uint4 a_in, const uint4 b_in
     uint32_t oa[4], ob[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-        const int i = 8 * j + 2 * e;               // first of the two pair indices
-        float c0 = 0.f, c1 = 0.f, s0 = 0.f, s1 = 0.f;
-        if (active) {
-            const float2 c2 = *reinterpret_cast<const float2 *>(cs + i);
-            const float2 s2 = *reinterpret_cast<const float2 *>(sn + i);
-            c0 = c2.x; c1 = c2.y; s0 = s2.x; s1 = s2.y;
-        }
+        const float c0 = c[2 * e], c1 = c[2 * e + 1], s0 = sv[2 * e], s1 = sv[2 * e + 1];
         const float a0 = xa[2 * e], a1 = xa[2 * e + 1], b0 = xb[2 * e], b1 = xb[2 * e + 1];
         float ya0, ya1, yb0, yb1;
         mul2(ya0, ya1, b0, b1, -s0, -s1);
@@ -251,12 +264,141 @@ rope_append_kernel(uint16_t *__restrict__ q, const uint16_t *__restrict__ k,
             // Every lane computes the rotation (the norm's shuffle spans the
             // whole warp); value vectors keep their loaded bits.
             uint4 a = ra[u], bb = rb[u], oa, ob;
-            rotate_vector<D>(a, bb, oa, ob, cs[tl], sn[tl], j, mem, qk_norm != 0, eps);
+            float c[8], sv[8];
+            lane_angles<D>(cs[tl], sn[tl], j, mem, c, sv);
+            rotate_vector<D>(a, bb, oa, ob, c, sv, mem, qk_norm != 0, eps);
             if (rotate) {
                 a = oa;
                 bb = ob;
             }
             if (mem) {
+                *reinterpret_cast<uint4 *>(dst + 8 * j) = a;
+                *reinterpret_cast<uint4 *>(dst + S::kHalf + 8 * j) = bb;
+            }
+        }
+    }
+}
+
+// Prompts and chunks (T >= kTokWarps): one warp per token, kTokWarps tokens per
+// CTA.  The warp walks its token's vectors -- Hq query heads, Hkv key heads, Hkv
+// value heads -- kVecPerWarp at a time (one pass), loads kTokBatch passes ahead,
+// and keeps the cos/sin of each lane's 8 pairs in registers for the whole token.
+// A pass that holds value heads only skips the arithmetic.  Sources and
+// destinations follow from the head index by adds alone.
+constexpr int kTokWarps = 4;
+constexpr int kTokBatch = 5;
+
+template <int D>
+__global__ void __launch_bounds__(kTokWarps * 32)
+rope_append_tok_kernel(uint16_t *__restrict__ q, const uint16_t *__restrict__ k,
+                       const uint16_t *__restrict__ v, uint16_t *__restrict__ kc,
+                       uint16_t *__restrict__ vc, const int32_t *__restrict__ pos0,
+                       int32_t *__restrict__ new_len, int T, int Hq, int Hkv, int Lmax,
+                       int qk_norm, float eps, const __grid_constant__ RopeTable tab,
+                       int32_t *status) {
+    using S = RopeShape<D>;
+    __shared__ __align__(16) float cs[kTokWarps][S::kHalf];
+    __shared__ __align__(16) float sn[kTokWarps][S::kHalf];
+    asm volatile("griddepcontrol.launch_dependents;");
+
+    const int nblk = (T + kTokWarps - 1) / kTokWarps;
+    const int b = blockIdx.x / nblk;
+    const int t0 = (blockIdx.x - b * nblk) * kTokWarps;
+    const int p0 = pos0 ? pos0[b] : 0;
+
+    bool write_cache = (k != nullptr);
+    if (threadIdx.x == 0) {
+        if (p0 < 0) {
+            report(status, GQA_DEV_BAD_LEN);
+        } else if (write_cache && p0 + T > Lmax) {
+            report(status, GQA_DEV_CAPACITY);
+        }
+        if (new_len && t0 == 0) new_len[b] = p0 + T;
+    }
+    if (p0 < 0) return;
+    if (write_cache && p0 + T > Lmax) write_cache = false;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int t = t0 + warp;
+    if (t >= T) return;                        // only warp-level sync follows
+    const int p = p0 + t;
+    const int j = lane % S::kTPV;
+    const int slot = lane / S::kTPV;
+    const bool active = j < S::kChunks;
+    const int nq = q ? Hq : 0;
+    const int nk = write_cache ? Hkv : 0;
+    const int nrot = nq + nk;
+    const int nvec = nrot + nk;
+    const int npass = (nvec + S::kVecPerWarp - 1) / S::kVecPerWarp;
+    const size_t token = (size_t)b * T + t;
+
+    auto locate = [&](int r, const uint16_t *&src, uint16_t *&dst) {
+        if (r < nq) {
+            dst = q + (token * Hq + r) * D;
+            src = dst;
+        } else if (r < nrot) {
+            const int h = r - nq;
+            src = k + (token * Hkv + h) * D;
+            dst = kc + (((size_t)b * Hkv + h) * Lmax + p) * D;
+        } else {
+            const int h = r - nrot;
+            src = v + (token * Hkv + h) * D;
+            dst = vc + (((size_t)b * Hkv + h) * Lmax + p) * D;
+        }
+    };
+
+    float c[8], sv[8];
+    for (int pb = 0; pb < npass; pb += kTokBatch) {
+        uint4 ra[kTokBatch], rb[kTokBatch];
+#pragma unroll
+        for (int u = 0; u < kTokBatch; ++u) {
+            const int r = (pb + u) * S::kVecPerWarp + slot;
+            ra[u] = make_uint4(0, 0, 0, 0);
+            rb[u] = make_uint4(0, 0, 0, 0);
+            if (r < nvec && active) {
+                const uint16_t *src;
+                uint16_t *dst;
+                locate(r, src, dst);
+                ra[u] = *reinterpret_cast<const uint4 *>(src + 8 * j);
+                rb[u] = *reinterpret_cast<const uint4 *>(src + S::kHalf + 8 * j);
+            }
+        }
+        if (pb == 0) {
+            // Angle p * theta_i in float64, reduced to [-pi, pi] in float64, then
+            // sin/cos in fp32; the warp's row of D/2 angles goes through shared
+            // memory to the lanes that own each pair.
+            for (int i = lane; i < S::kHalf; i += 32) {
+                const double a = (double)p * tab.theta[i];
+                const double two_pi = 6.283185307179586476925286766559;
+                const double r = a - rint(a * (1.0 / two_pi)) * two_pi;
+                float sf, cf;
+                sincosf((float)r, &sf, &cf);
+                cs[warp][i] = cf * tab.mscale;
+                sn[warp][i] = sf * tab.mscale;
+            }
+            __syncwarp();
+            lane_angles<D>(cs[warp], sn[warp], j, active, c, sv);
+        }
+#pragma unroll
+        for (int u = 0; u < kTokBatch; ++u) {
+            if (pb + u >= npass) break;                    // uniform across the warp
+            const int r0 = (pb + u) * S::kVecPerWarp;      // first vector of the pass
+            const int r = r0 + slot;
+            const bool mem = r < nvec && active;
+            uint4 a = ra[u], bb = rb[u];
+            if (r0 < nrot) {                               // uniform across the warp
+                uint4 oa, ob;
+                rotate_vector<D>(a, bb, oa, ob, c, sv, mem, qk_norm != 0, eps);
+                if (r < nrot) {
+                    a = oa;
+                    bb = ob;
+                }
+            }
+            if (mem) {
+                const uint16_t *src;
+                uint16_t *dst;
+                locate(r, src, dst);
                 *reinterpret_cast<uint4 *>(dst + 8 * j) = a;
                 *reinterpret_cast<uint4 *>(dst + S::kHalf + 8 * j) = bb;
             }
@@ -307,10 +449,18 @@ template <int D>
 cudaError_t launch_tb(void *q, const void *k, const void *v, void *kc, void *vc,
                       const int32_t *pos0, int32_t *new_len, int B, int T, int Hq, int Hkv,
                       int Lmax, const gqa_rope_params &p, int32_t *status, cudaStream_t s) {
-    // Blocks of 4 tokens once a sequence has that many; one token otherwise
-    // (decode), so that the grid still covers the batch.
-    if (T >= 4)
-        return launch<D, 4>(q, k, v, kc, vc, pos0, new_len, B, T, Hq, Hkv, Lmax, p, status, s);
+    // A warp per token once a sequence has kTokWarps tokens; otherwise (decode)
+    // a whole CTA per token, so that the grid still spreads the batch's few
+    // tokens over enough warps.
+    if (T >= kTokWarps) {
+        const unsigned grid = (unsigned)B * (unsigned)((T + kTokWarps - 1) / kTokWarps);
+        rope_append_tok_kernel<D><<<grid, kTokWarps * 32, 0, s>>>(
+            static_cast<uint16_t *>(q), static_cast<const uint16_t *>(k),
+            static_cast<const uint16_t *>(v), static_cast<uint16_t *>(kc),
+            static_cast<uint16_t *>(vc), pos0, new_len, T, Hq, Hkv, Lmax, p.qk_norm, p.eps,
+            make_table(D, p), status);
+        return cudaGetLastError();
+    }
     return launch<D, 1>(q, k, v, kc, vc, pos0, new_len, B, T, Hq, Hkv, Lmax, p, status, s);
 }
 
