@@ -152,10 +152,15 @@ class ClockSampler:
 
 
 def kernel_source_hash() -> str:
+    """Hash of the prefill kernel's code (its sources with // comments and
+    blank lines dropped, so that a comment edit keeps a profile valid)."""
     h = hashlib.sha256()
     for f in ("prefill.cu", "ptx.cuh", "common.cuh"):
-        with open(os.path.join(ROOT, "rope_gqa_kv_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "rope_gqa_kv_b200", "csrc", f), encoding="utf-8") as fh:
+            for ln in fh:
+                code = ln.split("//", 1)[0].rstrip()
+                if code:
+                    h.update(code.encode() + b"\n")
     return h.hexdigest()[:16]
 
 

@@ -25,7 +25,9 @@
 // O1 [384, 384+D) fp32 accumulators.
 // The tensor core alternates between the tiles -- PV0(j), S0(j+1), PV1(j),
 // S1(j+1) -- so the softmax of one tile runs while the other tile's two MMAs
-// execute.  A commit after S_t(j+1) also covers PV_t(j), so the softmax may
+// execute.  In a prompt the softmax hands P over in two halves (key columns
+// 0-63, then 64-127) and the first half's P V product runs while it computes
+// the second half.  A commit after S_t(j+1) also covers PV_t(j), so the softmax may
 // rescale O_t in TMEM as soon as its next scores are ready.  O_t is only
 // rescaled when the running maximum grows by more than 2^8 (the stale maximum
 // otherwise keeps p <= 256, exact in the final normalisation).
@@ -93,7 +95,7 @@ struct PfMaps {
 struct PfSync {
     uint64_t q_full, q_empty;
     uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
-    uint64_t s_full[2], p_full[2], o_final[2];
+    uint64_t s_full[2], p_half[2], p_full[2], o_final[2];
     uint64_t mma_done;
     uint32_t tmem_base;
 };
@@ -107,6 +109,9 @@ __device__ __forceinline__ uint32_t A(const uint64_t &b) { return ptx::smem_addr
 // prefix, a prompt of packed documents, or a prompt that also stores each row's
 // log-sum-exp for the backward.
 constexpr int kPrompt = 0, kChunkMode = 1, kDocs = 2, kPromptLse = 3;
+// whether the softmax hands P to the MMA issuer in two halves (prompts)
+template <int kMode>
+constexpr bool kPHalvesOf = kMode == kPrompt || kMode == kPromptLse;
 
 struct PfItem {
     int b, h, kvh, q0, n0, n1, n_kv;
@@ -275,6 +280,7 @@ template <int D, int kMode>
 __device__ void mma_issuer(PfSync &sy, uint8_t *smem, uint32_t tmem, const PfGrid &g,
                            int32_t *status) {
     using S = PfShape<D>;
+    constexpr bool kPHalves = kPHalvesOf<kMode>;
     constexpr uint32_t idS = ptx::idesc_bf16_f32(128, 128, false);
     constexpr uint32_t idO = ptx::idesc_bf16_f32(128, D, true);
     const uint32_t q_base = ptx::smem_addr(smem + S::kOffQ);
@@ -292,13 +298,33 @@ __device__ void mma_issuer(PfSync &sy, uint8_t *smem, uint32_t tmem, const PfGri
         }
         ptx::mma_commit(A(sy.s_full[t]));
     };
-    auto issue_pv = [&](int t, int vst, bool acc) {
+    // O_t (+)= P_t V over key rows [16 k0, 16 k1) of the tile.
+    auto issue_pv = [&](int t, int vst, bool acc, int k0, int k1) {
         const uint32_t va = v_base + vst * S::kTileBytes;
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks)
+        for (int ks = k0; ks < k1; ++ks)
             ptx::mma_ts(tmem + 256 + t * 128, tmem + t * 128 + ks * 8,
                         ptx::smem_desc_sw128(va + ks * 2048, S::kBlockBytes, 1024), idO,
                         (acc || ks > 0) ? 1u : 0u);
+    };
+    // Prompts: P_t arrives in two halves (key columns 0-63, then 64-127), and
+    // the product with the first half runs while the softmax computes the
+    // second (2 % faster on the 8 x 2048 prompt; chunks and documents, with
+    // their extra masking state, measured slower and hand P over whole).
+    auto issue_pv_halves = [&](int t, int vst, bool acc, int pc) {
+        if (!kPHalves) {
+            if (!ptx::mbar_wait(A(sy.p_full[t]), pc & 1)) return false;
+            ptx::tc_fence_after();
+            issue_pv(t, vst, acc, 0, 8);
+            return true;
+        }
+        if (!ptx::mbar_wait(A(sy.p_half[t]), pc & 1)) return false;
+        ptx::tc_fence_after();
+        issue_pv(t, vst, acc, 0, 4);
+        if (!ptx::mbar_wait(A(sy.p_full[t]), pc & 1)) return false;
+        ptx::tc_fence_after();
+        issue_pv(t, vst, true, 4, 8);
+        return true;
     };
 
     int kc = 0, vc = 0, qc = 0;     // K, V tiles and Q pairs consumed
@@ -331,11 +357,9 @@ __device__ void mma_issuer(PfSync &sy, uint8_t *smem, uint32_t tmem, const PfGri
             const int kst = kidx % S::kStagesK;
             bool k_next = false;
             if (j < I.n0) {
-                ok = ptx::mbar_wait(A(sy.p_full[0]), pc0 & 1);
+                ok = issue_pv_halves(0, vst, j > I.lo0, pc0);
                 if (!ok) break;
                 ++pc0;
-                ptx::tc_fence_after();
-                issue_pv(0, vst, j > I.lo0);
                 if (jn < I.n0) {
                     ok = ptx::mbar_wait(A(sy.k_full[kst]), (kidx / S::kStagesK) & 1);
                     if (!ok) break;
@@ -346,11 +370,9 @@ __device__ void mma_issuer(PfSync &sy, uint8_t *smem, uint32_t tmem, const PfGri
                 }
             }
             if (I.has1 && j >= I.lo1 && j < I.n1) {
-                ok = ptx::mbar_wait(A(sy.p_full[1]), pc1 & 1);
+                ok = issue_pv_halves(1, vst, j > I.lo1, pc1);
                 if (!ok) break;
                 ++pc1;
-                ptx::tc_fence_after();
-                issue_pv(1, vst, j > I.lo1);
                 if (jn < I.n1) {
                     if (!k_next) {
                         ok = ptx::mbar_wait(A(sy.k_full[kst]), (kidx / S::kStagesK) & 1);
@@ -388,6 +410,7 @@ __device__ void mma_issuer(PfSync &sy, uint8_t *smem, uint32_t tmem, const PfGri
 template <int D, int kMode>
 __device__ void softmax_tile(PfSync &sy, uint8_t *smem, uint32_t tmem, int t, const PfGrid &g,
                              float scale_log2, uint16_t *__restrict__ out, int32_t *status) {
+    constexpr bool kPHalves = kPHalvesOf<kMode>;
     using S = PfShape<D>;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int row = (warp & 3) * 32 + lane;
@@ -481,6 +504,26 @@ __device__ void softmax_tile(PfSync &sy, uint8_t *smem, uint32_t tmem, int t, co
             // special-function unit for 2^x, four independent partial row sums.
             // (with documents a row may see no key yet: m is -inf, its p must be 0)
             const float neg_m = (kMode == kDocs && m == -INFINITY) ? 0.f : -m;
+            // The last V tile has landed once its barrier's phase completes; zero
+            // its rows past the last valid key, then publish the stores to the
+            // tensor core (async proxy) before P is handed over.
+            auto clear_v_tail = [&]() {
+                if (clears && j == nt - 1) {
+                    const int vidx = vc0 + I.n_kv - 1;
+                    ok = __all_sync(0xffffffffu, ptx::mbar_wait(A(sy.v_full[vidx % S::kStagesV]),
+                                                                 (vidx / S::kStagesV) & 1));
+                    if (ok) {
+                        uint8_t *vt = smem + S::kOffV + (vidx % S::kStagesV) * S::kTileBytes;
+                        const int n16 = (128 - I.r_valid) * 8;   // 16-byte pieces per column block
+                        for (int x = row; x < n16 * S::kBlocks; x += 128) {
+                            const int kb = x / n16, y = x - kb * n16;
+                            *reinterpret_cast<uint4 *>(vt + kb * S::kBlockBytes + I.r_valid * 128 + y * 16) =
+                                make_uint4(0, 0, 0, 0);
+                        }
+                        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    }
+                }
+            };
             float la0 = 0.f, la1 = 0.f, lb0 = 0.f, lb1 = 0.f;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
@@ -498,27 +541,18 @@ __device__ void softmax_tile(PfSync &sy, uint8_t *smem, uint32_t tmem, int t, co
                         ptx::fadd2(lb0, lb1, lb0, lb1, p0, p1);
                 }
                 ptx::tmem_st16(lane_addr + s_col + 16 * c, p);
+                if (kPHalves && c == 1) {
+                    clear_v_tail();
+                    // first half of P (key columns 0-63) to the tensor core
+                    ptx::tmem_wait_st();
+                    ptx::tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(A(sy.p_half[t]));
+                }
             }
 #undef SV
             l += (la0 + la1) + (lb0 + lb1);
-            if (clears && j == nt - 1) {
-                // The last V tile has landed once its barrier's phase completes;
-                // zero its rows past the last valid key, then publish the stores to
-                // the tensor core (async proxy) before P is handed over.
-                const int vidx = vc0 + I.n_kv - 1;
-                ok = __all_sync(0xffffffffu, ptx::mbar_wait(A(sy.v_full[vidx % S::kStagesV]),
-                                                             (vidx / S::kStagesV) & 1));
-                if (ok) {
-                    uint8_t *vt = smem + S::kOffV + (vidx % S::kStagesV) * S::kTileBytes;
-                    const int n16 = (128 - I.r_valid) * 8;   // 16-byte pieces per column block
-                    for (int x = row; x < n16 * S::kBlocks; x += 128) {
-                        const int kb = x / n16, y = x - kb * n16;
-                        *reinterpret_cast<uint4 *>(vt + kb * S::kBlockBytes + I.r_valid * 128 + y * 16) =
-                            make_uint4(0, 0, 0, 0);
-                    }
-                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                }
-            }
+            if (!kPHalves) clear_v_tail();
             ptx::tmem_wait_st();
             ptx::tc_fence_before();
             __syncwarp();
@@ -597,7 +631,8 @@ prefill_kernel(const __grid_constant__ PfMaps maps, uint16_t *__restrict__ out, 
         }
         for (int t = 0; t < 2; ++t) {
             ptx::mbar_init(A(sy.s_full[t]), 1);
-            ptx::mbar_init(A(sy.p_full[t]), 4);   // one elected lane per softmax warp
+            ptx::mbar_init(A(sy.p_half[t]), 4);   // one elected lane per softmax warp
+            ptx::mbar_init(A(sy.p_full[t]), 4);
             ptx::mbar_init(A(sy.o_final[t]), 1);
         }
         ptx::mbar_init(A(sy.mma_done), 1);
