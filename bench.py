@@ -385,6 +385,10 @@ def run_ours(args, rank, world, dev, dist_on):
                          "rope_scaling": measure_scaled_append(layer, peaks, tag),
                          "doc_masked_prefill": measure_docs(layer, peaks, tag),
                          "attention_backward": measure_backward(layer, peaks, tag)}
+    try:
+        line["decode_loop"] = measure_decode_loop(dev)
+    except Exception as e:  # a side measurement: report it, keep the line
+        line["decode_loop"] = {"error": ("%s: %s" % (type(e).__name__, e))[:200]}
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
     return line
@@ -489,6 +493,53 @@ def measure_docs(layer, peaks, tag, reps: int = 30):
             "algorithmic_per_launch": fl,
             "causal_fraction_kept": round(fl / prefill_flops(), 4),
             "l2": "flushed (256 MB write) before each launch"}
+
+
+def measure_decode_loop(dev, steps: int = 100):
+    """The generation loop (512-token prompt, then 100 generated tokens; B=1,
+    16q/4kv, D=64), outside the timed step, per generated token: eager (the
+    append and the decode's two kernels launched from the host each token) and
+    replayed from CUDA graphs (DecodeGraph).  Device time of the whole loop
+    between two CUDA events, so the gaps the host's launches leave count."""
+    import rope_gqa_kv_b200 as gqa
+    w = inputs.BY_NAME["generation"]
+    x = inputs.make_inputs(w, decode_steps=1)
+    d = lambda t: t.to(dev)  # noqa: E731
+    q0, k0, v0 = (d(t) for t in x["steps"][0])
+    per_token = {}
+    for mode in ("eager", "graph"):
+        kc, vc = d(x["k_cache"]), d(x["v_cache"])
+        gqa.gqa_rope_append(d(x["q"]), d(x["k"]), d(x["v"]), kc, vc, qk_norm=w.qk_norm)
+        pos = torch.full((w.B,), w.T, dtype=torch.int32, device=dev)
+        if mode == "graph":
+            dg = gqa.DecodeGraph(kc, vc, pos, w.Hq, qk_norm=w.qk_norm)
+            dg.q.copy_(q0)
+            dg.k.copy_(k0)
+            dg.v.copy_(v0)
+            run = dg.step
+        else:
+            ws = gqa.decode_workspace(w.B, w.Hq, w.D, w.Lmax, dev)
+            out = torch.empty_like(q0)
+            lens = [pos.clone(), pos.clone()]
+            cur = [0]
+
+            def run():
+                a, b = cur[0], cur[0] ^ 1
+                gqa.gqa_rope_append(q0, k0, v0, kc, vc, pos0=lens[a], new_len=lens[b],
+                                    qk_norm=w.qk_norm)
+                gqa.gqa_decode(q0, kc, vc, lens[b], w.Lmax, out=out, workspace=ws)
+                cur[0] = b
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(steps):
+            run()
+        e1.record()
+        torch.cuda.synchronize()
+        per_token[mode] = e0.elapsed_time(e1) * 1e3 / steps
+    return {"workload": "B=1 16q/4kv D=64: 512-token prompt, then %d generated tokens" % steps,
+            "kernels_per_token": 3, "eager_us_per_token": round(per_token["eager"], 2),
+            "graph_us_per_token": round(per_token["graph"], 2)}
 
 
 def measure_chunk(dev, peaks, tag, reps: int = 30):

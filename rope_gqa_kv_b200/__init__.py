@@ -5,6 +5,7 @@ include/gqa.h); this package is its thin Python binding plus the seeded
 workload generator used by the tests and the benchmark.
 """
 from . import inputs  # noqa: F401
+from .decode_graph import DecodeGraph  # noqa: F401
 from ._lib import (GQA_DEV_BAD_LEN, GQA_DEV_CAPACITY, GQA_DEV_TIMEOUT,  # noqa: F401
                    LIB_PATH, SIGNATURES, GqaError, RopeScaling, decode_workspace,
                    gqa_attention_backward, gqa_backward_workspace_bytes, gqa_decode,

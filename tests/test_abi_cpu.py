@@ -182,3 +182,11 @@ def test_binding_refuses_cpu_tensors(lib):
     q = torch.zeros(1, 4, 2, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError, match="CUDA"):
         gqa.gqa_rope_apply(q)
+
+
+def test_decode_graph_refuses_host_tensors():
+    """DecodeGraph captures device work only: host tensors are refused up front."""
+    import torch
+    kc = torch.zeros(1, 1, 128, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        gqa.DecodeGraph(kc, kc.clone(), torch.zeros(1, dtype=torch.int32), 1)

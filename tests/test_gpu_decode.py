@@ -74,6 +74,38 @@ def test_generation_loop(cuda_lib, name):
         pos = pos + 1
 
 
+def test_decode_graph_replays_the_eager_loop(cuda_lib):
+    """The 512-token prompt + 100 generated tokens through DecodeGraph (the step
+    captured in CUDA graphs): every step's output bit-identical to the eager
+    calls (which test_generation_loop holds against the oracle), the same
+    caches at the end, and the lengths advanced by one per step."""
+    w = inputs.BY_NAME["generation"]
+    x = inputs.make_inputs(w)
+    B, T = w.B, w.T
+    caches = []
+    for _ in range(2):
+        kc, vc = x["k_cache"].to(DEV), x["v_cache"].to(DEV)
+        gqa.gqa_rope_append(x["q"].to(DEV), x["k"].to(DEV), x["v"].to(DEV), kc, vc,
+                            qk_norm=w.qk_norm)
+        caches.append((kc, vc))
+    pos = torch.full((B,), T, dtype=torch.int32, device=DEV)
+    dg = gqa.DecodeGraph(caches[1][0], caches[1][1], pos, w.Hq, qk_norm=w.qk_norm)
+    for s, (q, k, v) in enumerate(x["steps"]):
+        eager = _decode_step(q.to(DEV), k.to(DEV), v.to(DEV), caches[0][0], caches[0][1], pos,
+                             w.qk_norm, w.Lmax)
+        dg.q.copy_(q)
+        dg.k.copy_(k)
+        dg.v.copy_(v)
+        got = dg.step()
+        assert torch.equal(got.view(torch.int16), eager.view(torch.int16)), "step %d" % s
+        pos = pos + 1
+    torch.cuda.synchronize()
+    assert dg.status.item() == 0
+    assert torch.equal(dg.lens, pos)
+    for a, b in zip(caches[0], caches[1]):
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
 @pytest.mark.parametrize("Hq,Hkv,D", [(8, 8, 64), (8, 1, 64), (12, 4, 96), (16, 2, 128),
                                       (4, 4, 128), (6, 2, 96)])
 def test_groupings_and_head_dims(cuda_lib, Hq, Hkv, D):
