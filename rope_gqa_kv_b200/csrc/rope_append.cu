@@ -5,11 +5,13 @@
 // QK-norm: page "训练3.8B LLM至0.384 CORE，成本998美元 – Hugo Vergnes", section "设置";
 // KV-cache append: first page, section "V3：扩容与推理优化".
 //
-// One CTA per block of 4 consecutive tokens of a sequence (1 token in decode).
-// The CTA issues the loads of its first head vectors, then turns each token's
-// position into the D/2 rotation angles (float64 angle p * theta_i reduced to
-// [-pi, pi] in float64, cos/sin in fp32) in shared memory, shared by all of the
-// token's heads.  The float64 table theta_i -- base^(-2i/D), or one of the
+// Prompts and chunks: one warp per token (rope_append_tok_kernel); decode, with
+// its one token per sequence: one CTA per token (rope_append_kernel), so the
+// batch's few tokens still spread over enough warps.  Either issues the loads
+// of its first head vectors, then turns each token's position into the D/2
+// rotation angles (float64 angle p * theta_i reduced to [-pi, pi] in float64,
+// cos/sin in fp32) through shared memory, shared by all of the token's heads.
+// The float64 table theta_i -- base^(-2i/D), or one of the
 // context-extension variants (linear interpolation, NTK-aware, YaRN, see
 // gqa.h) -- is computed once per call on the host and passed as a kernel
 // parameter, together with YaRN's scale of the rotated vectors.  Each head vector
@@ -141,10 +143,11 @@ __device__ __forceinline__ void rotate_vector(const uint4 a_in, const uint4 b_in
 
 // Vectors of one token, in order: Hq query heads (if q), Hkv key heads and Hkv
 // value heads (if k).  Query heads are rotated in place; key heads are rotated
-// into the cache; value heads are copied into the cache bit for bit.  A CTA
-// takes TB consecutive tokens of one sequence: its global loads go out in
-// batches of kBatch passes (the first batch before the angles are computed),
-// so every lane has several 32-byte loads in flight.
+// into the cache; value heads are copied into the cache bit for bit.  This
+// kernel's CTA takes TB consecutive tokens of one sequence (TB = 1: the decode
+// step): its global loads go out in batches of kBatch passes (the first batch
+// before the angles are computed), so every lane has several 32-byte loads in
+// flight.
 constexpr int kBatch = 4;
 
 template <int D, int TB>
