@@ -62,6 +62,39 @@ def test_rope_append_matches_oracle(cuda_lib, D, qk_norm):
         assert torch.equal(got_vc[b][:, keep].view(torch.int16), vc[b][:, keep].view(torch.int16))
 
 
+@pytest.mark.parametrize("Hq,Hkv,D,T", [(2, 1, 128, 5), (4, 2, 64, 6), (3, 1, 96, 4),
+                                        (1, 1, 128, 9), (8, 8, 64, 3), (2, 2, 128, 2),
+                                        (12, 4, 128, 7)])
+def test_rope_append_head_mixes_and_short_chunks(cuda_lib, Hq, Hkv, D, T):
+    """Head counts whose query, key and value vectors share a warp's pass (the
+    prompt kernel walks a token's Hq + 2 Hkv vectors 4 (D = 64: 8) at a time),
+    chunks of 4 to 9 tokens with a ragged last block, and 2 or 3 tokens (the
+    per-token kernel)."""
+    B, L = 2, 128
+    q, k, v, kc, vc = _case(B, T, Hq, Hkv, D, L, seed=100 + Hq + D + T)
+    pos0 = torch.tensor([0, 117 - T], dtype=torch.int32)
+    dq, dk, dv = q.to(DEV), k.to(DEV), v.to(DEV)
+    dkc, dvc = kc.to(DEV), vc.to(DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    gqa.gqa_rope_append(dq, dk, dv, dkc, dvc, pos0=pos0.to(DEV), max_pos0=int(pos0.max()),
+                        qk_norm=True, status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    assert_within_one_ulp(dq, oracle.rope_apply(bits(q), pos0.numpy(), True), "q")
+    want_k = oracle.rope_apply(bits(k), pos0.numpy(), True)
+    got_kc, got_vc = dkc.cpu(), dvc.cpu()
+    for b in range(B):
+        p = int(pos0[b])
+        sl = slice(p, p + T)
+        assert_within_one_ulp(got_kc[b, :, sl].transpose(0, 1), want_k[b], "k_cache[%d]" % b)
+        assert torch.equal(got_vc[b, :, sl].transpose(0, 1).view(torch.int16),
+                           v[b].view(torch.int16))
+        keep = torch.ones(L, dtype=torch.bool)
+        keep[sl] = False
+        assert torch.equal(got_kc[b][:, keep].view(torch.int16), kc[b][:, keep].view(torch.int16))
+        assert torch.equal(got_vc[b][:, keep].view(torch.int16), vc[b][:, keep].view(torch.int16))
+
+
 def test_fused_equals_separate_calls(cuda_lib):
     B, T, Hq, Hkv, D, L = 2, 129, 8, 2, 128, 384
     q, k, v, kc, vc = _case(B, T, Hq, Hkv, D, L, seed=11)
