@@ -5,6 +5,7 @@ sign, a wrong index or head map, a transposed operand), builds that copy into a
 scratch directory and runs the pin suite against it in a child process.  The
 pin suite has to fail for every mutant.  The real oracle is never modified.
 """
+import concurrent.futures
 import os
 import subprocess
 import sys
@@ -35,32 +36,51 @@ MUTANTS = {
 }
 
 
+def _run(name, scratch):
+    """Build the copy of oracle.c (mutated unless name is None) and run the pins
+    against it; returns the child's (returncode, stdout tail)."""
+    src = open(SRC).read()
+    if name is not None:
+        old, new = MUTANTS[name]
+        if src.count(old) != 1:
+            return None, "mutation anchor not found exactly once: %r" % old
+        src = src.replace(old, new)
+    d = os.path.join(scratch, name or "control")
+    os.makedirs(d)
+    mut_src = os.path.join(d, "oracle_mut.c")
+    with open(mut_src, "w") as f:
+        f.write(src)
+    lib = os.path.join(d, "liboracle_mut.so")
+    subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", mut_src, "-o", lib,
+                           "-lm"])
+    env = dict(os.environ, GQA_ORACLE_LIB=lib, OMP_NUM_THREADS="2")
+    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+                        os.path.join(HERE, "test_oracle_pins.py")],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=900)
+    return r.returncode, r.stdout[-2000:]
+
+
+@pytest.fixture(scope="module")
+def results(tmp_path_factory):
+    """Every mutant and the control, run side by side (one child per case)."""
+    scratch = str(tmp_path_factory.mktemp("oracle_mutants"))
+    names = sorted(MUTANTS) + [None]
+    workers = max(2, min(len(names), (os.cpu_count() or 2) // 2))
+    with concurrent.futures.ThreadPoolExecutor(max_workers=workers) as ex:
+        return dict(zip(names, ex.map(lambda n: _run(n, scratch), names)))
+
+
 @pytest.mark.slow
 @pytest.mark.parametrize("name", sorted(MUTANTS))
-def test_pins_reject_mutant(name, tmp_path):
-    old, new = MUTANTS[name]
-    src = open(SRC).read()
-    assert src.count(old) == 1, "mutation anchor not found exactly once: %r" % old
-    mut_src = tmp_path / "oracle_mut.c"
-    mut_src.write_text(src.replace(old, new))
-    lib = tmp_path / "liboracle_mut.so"
-    subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", str(mut_src),
-                           "-o", str(lib), "-lm"])
-    env = dict(os.environ, GQA_ORACLE_LIB=str(lib))
-    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
-                        os.path.join(HERE, "test_oracle_pins.py")],
-                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
-    assert r.returncode != 0, "pins did not catch mutant %s:\n%s" % (name, r.stdout[-2000:])
+def test_pins_reject_mutant(name, results):
+    rc, out = results[name]
+    assert rc is not None, out
+    assert "passed" in out or "failed" in out, out
+    assert rc != 0, "pins did not catch mutant %s:\n%s" % (name, out)
 
 
 @pytest.mark.slow
-def test_unmutated_copy_passes(tmp_path):
+def test_unmutated_copy_passes(results):
     """Control: the same harness on an unchanged copy must pass."""
-    lib = tmp_path / "liboracle_copy.so"
-    subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", SRC,
-                           "-o", str(lib), "-lm"])
-    env = dict(os.environ, GQA_ORACLE_LIB=str(lib))
-    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
-                        os.path.join(HERE, "test_oracle_pins.py")],
-                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
-    assert r.returncode == 0, r.stdout[-2000:]
+    rc, out = results[None]
+    assert rc == 0, out

@@ -536,6 +536,11 @@ def test_backward_matches_torch_autograd_sdpa():
     # log-sum-exp of the first row: one key
     s00 = float(q[0, 0, 0] @ k[0, 0, 0]) / math.sqrt(D)
     assert abs(lse[0, 0, 0] - s00) < 1e-12
+    # every row: torch's logsumexp over the row's visible keys
+    sc = (tq.detach().transpose(1, 2) @ tk.detach().repeat_interleave(g, dim=2)
+          .transpose(1, 2).transpose(-1, -2)) / math.sqrt(D)
+    sc = sc.masked_fill(torch.ones(T, T, dtype=torch.bool).triu(1), float("-inf"))
+    np.testing.assert_allclose(lse, torch.logsumexp(sc, dim=-1).numpy(), rtol=0, atol=1e-12)
 
 
 def test_backward_sums():
