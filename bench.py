@@ -220,41 +220,82 @@ class Layer:
         self.pin_out_p = torch.empty(self.pout.shape, dtype=torch.bfloat16).pin_memory()
         self.pin_out_d = torch.empty(self.dout.shape, dtype=torch.bfloat16).pin_memory()
 
-    def step(self, ev=None):
+    def io_set(self, other=False):
+        """The step's inputs and outputs on the device: the layer's own tensors,
+        or (other=True) a second set of the same shapes for the pipelined
+        end-to-end leg."""
+        names = ("pq", "pk", "pv", "dq", "dk", "dv", "pos", "pout", "dout")
+        if not other:
+            return {k: getattr(self, k) for k in names}
+        return {k: torch.empty_like(getattr(self, k)) for k in names}
+
+    def step(self, ev=None, io=None):
         """The device-resident step.  ev: optional list of 5 events recorded
-        around the four phases (prefill append, prefill, decode append, decode)."""
+        around the four phases (prefill append, prefill, decode append, decode);
+        io: the input / output tensors (default: the layer's own)."""
         g = self.gqa
+        x = io if io is not None else self.io_set()
         if ev is not None:
             ev[0].record()
-        g.gqa_rope_append(self.pq, self.pk, self.pv, self.pkc, self.pvc, qk_norm=True,
+        g.gqa_rope_append(x["pq"], x["pk"], x["pv"], self.pkc, self.pvc, qk_norm=True,
                           max_pos0=0, status=self.status)
         if ev is not None:
             ev[1].record()
-        g.gqa_prefill(self.pq, self.pkc, self.pvc, out=self.pout, status=self.status)
+        g.gqa_prefill(x["pq"], self.pkc, self.pvc, out=x["pout"], status=self.status)
         if ev is not None:
             ev[2].record()
-        g.gqa_rope_append(self.dq, self.dk, self.dv, self.dkc, self.dvc, pos0=self.pos,
+        g.gqa_rope_append(x["dq"], x["dk"], x["dv"], self.dkc, self.dvc, pos0=x["pos"],
                           max_pos0=self.max_len - 1, new_len=self.lens_new, qk_norm=True,
                           status=self.status)
         if ev is not None:
             ev[3].record()
-        g.gqa_decode(self.dq, self.dkc, self.dvc, self.lens_new, self.max_len, out=self.dout,
+        g.gqa_decode(x["dq"], self.dkc, self.dvc, self.lens_new, self.max_len, out=x["dout"],
                      workspace=self.ws, status=self.status)
         if ev is not None:
             ev[4].record()
 
-    def step_e2e(self):
-        """Same step from pinned host buffers: H2D inputs, compute, D2H outputs."""
-        self.pq.copy_(self.pin["pq"], non_blocking=True)
-        self.pk.copy_(self.pin["pk"], non_blocking=True)
-        self.pv.copy_(self.pin["pv"], non_blocking=True)
-        self.dq.copy_(self.pin["dq"], non_blocking=True)
-        self.dk.copy_(self.pin["dk"], non_blocking=True)
-        self.dv.copy_(self.pin["dv"], non_blocking=True)
-        self.pos.copy_(self.pin["pos"], non_blocking=True)
-        self.step()
-        self.pin_out_p.copy_(self.pout, non_blocking=True)
-        self.pin_out_d.copy_(self.dout, non_blocking=True)
+    def run_e2e(self, steps):
+        """`steps` steps from pinned host buffers: every step copies its inputs
+        host -> device and reads both outputs back device -> host.  Pipelined
+        over two device input / output sets and three streams: the upload of
+        step i + 1 and the download of step i - 1 run while step i computes
+        (and the two copy directions share the PCIe link's two halves).  The
+        kernels still run one step after another on the compute stream, which
+        is the stream the returned events are recorded on."""
+        if not hasattr(self, "_sets"):
+            self._sets = [self.io_set(), self.io_set(other=True)]
+            self._h2d = torch.cuda.Stream(device=self.dev)
+            self._d2h = torch.cuda.Stream(device=self.dev)
+        comp = torch.cuda.current_stream(self.dev)
+        mk = lambda: torch.cuda.Event(enable_timing=False)  # noqa: E731
+        ev_in, ev_comp, ev_out = [mk(), mk()], [mk(), mk()], [mk(), mk()]
+        start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        start.record(comp)
+        self._h2d.wait_event(start)
+        self._d2h.wait_event(start)
+        for i in range(steps):
+            s = i & 1
+            io = self._sets[s]
+            with torch.cuda.stream(self._h2d):
+                if i >= 2:
+                    self._h2d.wait_event(ev_comp[s])     # step i - 2 is done with set s
+                for k in ("pq", "pk", "pv", "dq", "dk", "dv", "pos"):
+                    io[k].copy_(self.pin[k], non_blocking=True)
+                ev_in[s].record(self._h2d)
+            comp.wait_event(ev_in[s])
+            if i >= 2:
+                comp.wait_event(ev_out[s])               # step i - 2's outputs are read
+            self.step(io=io)
+            ev_comp[s].record(comp)
+            with torch.cuda.stream(self._d2h):
+                self._d2h.wait_event(ev_comp[s])
+                self.pin_out_p.copy_(io["pout"], non_blocking=True)
+                self.pin_out_d.copy_(io["dout"], non_blocking=True)
+                ev_out[s].record(self._d2h)
+        for s in range(min(steps, 2)):
+            comp.wait_event(ev_out[s])
+        stop.record(comp)
+        return start, stop
 
     def e2e_bytes(self):
         h2d = sum(t.numel() * t.element_size() for t in self.pin.values())
@@ -308,15 +349,9 @@ def run_ours(args, rank, world, dev, dist_on):
     ms_total = _max_over_ranks(ms_total, dist_on, dev)
 
     # -- end-to-end region: host buffers in, results out, every step --
-    for _ in range(min(args.warmup, 3)):
-        layer.step_e2e()
+    layer.run_e2e(min(args.warmup, 3))
     _barrier_sync(dist_on)
-    s2 = torch.cuda.Event(enable_timing=True)
-    e2 = torch.cuda.Event(enable_timing=True)
-    s2.record()
-    for _ in range(args.steps):
-        layer.step_e2e()
-    e2.record()
+    s2, e2 = layer.run_e2e(args.steps)
     _barrier_sync(dist_on)
     ms_e2e = _max_over_ranks(s2.elapsed_time(e2), dist_on, dev)
     clocks = sampler.stop() if sampler else None
@@ -376,7 +411,9 @@ def run_ours(args, rank, world, dev, dist_on):
                             "algorithmic_per_launch": append_bytes()},
         "e2e": {"value": round(tok / (ms_e2e / K * 1e-3), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "ms_per_step": round(ms_e2e / K, 4)},
+                "ms_per_step": round(ms_e2e / K, 4),
+                "pipelined": "two device input/output sets; step i+1's upload and step "
+                             "i-1's download overlap step i's kernels"},
         "gpu_launches": LAUNCHES_PER_STEP * K,
         "clocks": clocks,
         "device_status": status,
