@@ -278,9 +278,13 @@ size_t gqa_decode_workspace_bytes(int B, int Hq, int D, int max_len);
  *   - Sizes whose gqa_decode_workspace_bytes(B, Hq, D, max_len_host) exceeds
  *     32 MiB return GQA_ERR_WORKSPACE (the 64 x 24-head x 2049-slot batched
  *     decode needs 26.4 MB).
- *   - The first call on a device looks up the array's device address (with
- *     that device current) and keeps it; make that first call before any stream
- *     capture.
+ *   - The array's device address belongs to the CUDA context the library's
+ *     module is loaded into.  The first call from a context (the device's
+ *     primary context, or a context the caller created and made current) looks
+ *     that address up and keeps it for that context; make that first call
+ *     before any stream capture.  A context destroyed and then replaced by a
+ *     new one with the same handle would find the old address: load the
+ *     library again after destroying a context it has run in.
  *   - Every call on a device uses the same array: calls that may overlap on the
  *     GPU (different streams without ordering) race and corrupt each other.
  *     Calls ordered on one stream are fine; no part of the array has to start
@@ -292,11 +296,14 @@ gqa_status gqa_decode_noalloc(const void *q, const void *k_cache, const void *v_
                               void *stream);
 
 /*
- * gqa_selftest_bounded_wait -- checks the failure path of the bounded waits
- * without a fault: one thread waits, for limit_ms (1 .. 10000), on an mbarrier
- * that nothing arrives on, gives up and ORs GQA_DEV_TIMEOUT into *status_dev
- * (required).  The context stays usable.  The paper has no counterpart of this
- * call; it is a property of this library.
+ * gqa_selftest_bounded_wait -- checks the bounded waits without a fault, through
+ * the same wait function every kernel uses (with its limit shortened to
+ * limit_ms, 1 .. 10000): one thread first waits on an mbarrier whose phase has
+ * completed, which must return at once (GQA_DEV_BAD_LEN is raised if it does
+ * not), then waits on an mbarrier that nothing arrives on, gives up after
+ * limit_ms and ORs GQA_DEV_TIMEOUT into *status_dev (required).  The context
+ * stays usable.  The paper has no counterpart of this call; it is a property of
+ * this library.
  */
 gqa_status gqa_selftest_bounded_wait(int32_t *status_dev, int limit_ms, void *stream);
 

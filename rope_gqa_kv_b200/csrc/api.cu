@@ -17,18 +17,21 @@ extern "C" const char *gqa_status_string(gqa_status s) {
 
 extern "C" int gqa_version(void) { return 200; }
 
-// One thread waits on an mbarrier that nothing arrives on.  The wait is the one
-// every kernel of the library uses, with its limit shortened to limit_ns: it
-// gives up, and the thread raises GQA_DEV_TIMEOUT instead of hanging.
+// One thread waits on an mbarrier that nothing arrives on, through
+// ptx::mbar_wait -- the function every kernel of the library waits with -- with
+// its limit shortened to limit_ns: the wait gives up, and the thread raises
+// GQA_DEV_TIMEOUT instead of hanging.  A second wait, on a barrier whose phase
+// has completed, must succeed at once (the success path of the same function).
 __global__ void selftest_wait_kernel(int32_t *status, unsigned long long limit_ns) {
-    __shared__ __align__(8) uint64_t bar;
-    const uint32_t b = gqa::ptx::smem_addr(&bar);
-    gqa::ptx::mbar_init(b, 1);
+    __shared__ __align__(8) uint64_t bar[2];
+    const uint32_t never = gqa::ptx::smem_addr(&bar[0]);
+    const uint32_t done = gqa::ptx::smem_addr(&bar[1]);
+    gqa::ptx::mbar_init(never, 1);
+    gqa::ptx::mbar_init(done, 1);
     gqa::ptx::fence_barrier_init();
-    const uint64_t t0 = gqa::ptx::globaltimer();
-    bool done = gqa::ptx::mbar_try_wait(b, 0);
-    while (!done && gqa::ptx::globaltimer() - t0 < limit_ns) done = gqa::ptx::mbar_try_wait(b, 0);
-    if (!done) gqa::report(status, GQA_DEV_TIMEOUT);
+    gqa::ptx::mbar_arrive(done);                       // completes phase 0 of `done`
+    if (!gqa::ptx::mbar_wait(done, 0, limit_ns)) gqa::report(status, GQA_DEV_BAD_LEN);
+    if (!gqa::ptx::mbar_wait(never, 0, limit_ns)) gqa::report(status, GQA_DEV_TIMEOUT);
 }
 
 extern "C" gqa_status gqa_selftest_bounded_wait(int32_t *status_dev, int limit_ms, void *stream) {

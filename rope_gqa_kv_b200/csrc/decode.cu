@@ -24,9 +24,15 @@
 //      the chunk's (m, l, o) go to the workspace.
 // A second kernel, launched as a programmatic dependent of the first, merges
 // the chunks of each (b, query head): M = max m_i,
-// o = sum_i 2^(m_i - M) o_i / sum_i 2^(m_i - M) l_i.  (Merging inside the
-// first kernel -- the last chunk to finish, found with an atomic ticket, merging
-// the rest -- measured slower: every CTA then has to fence its partial writes.)
+// o = sum_i 2^(m_i - M) o_i / sum_i 2^(m_i - M) l_i.  One warp per row, lanes
+// spanning D; every partial of the row is loaded before any is used, and the
+// kernel's few registers per CTA let all rows of a batch be resident at once,
+// so the merge costs about one memory round trip.  (Merging inside the first
+// kernel -- the last chunk to finish, found with an atomic ticket, merging the
+// rest -- measured slower: every CTA then has to fence its partial writes;
+// so did one thread-block cluster per row merging through distributed shared
+// memory, and CTAs streaming several chunks through per-warp rings: fewer,
+// longer-lived CTAs hide the copies' latency worse than many one-shot ones.)
 #include <algorithm>
 #include <mutex>
 
@@ -295,51 +301,68 @@ decode_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ kc,
 
 }
 
-// Merge the chunks of one (b, query head): one CTA per row, one thread per output
-// coordinate.  No barrier and one round trip to memory: each thread issues the
-// loads of its coordinate of up to 32 chunk partials at once, while every warp
-// reduces the chunk maxima and sums on its own with shuffles; the weights
-// 2^(m_i - M) then reach the threads by shuffle.  Rows of more than 32 chunks
-// repeat this per group of 32.
+// Merge the chunks of each (b, query head) row: one warp per row, four rows per
+// CTA, lane i owning coordinates 4i .. 4i+3.  For up to 32 chunks at a time the
+// lanes load every chunk's partial of their coordinates and lane i the chunk's
+// (m, l), all before any is used; the maximum and the weights 2^(m_i - M) then
+// travel by shuffle.  Rows of more than 32 chunks repeat this per group of 32,
+// rescaling what the earlier groups summed (online, like the split kernel).
+template <int D>
 __global__ void __launch_bounds__(128)
 decode_merge_kernel(const float *__restrict__ ws_ml, const float *__restrict__ ws_o,
-                    const int32_t *__restrict__ lens, int max_len, int Hq, int D, int Lmax,
-                    int n_splits, uint16_t *__restrict__ out) {
+                    const int32_t *__restrict__ lens, int max_len, int Hq, int Lmax,
+                    int n_splits, int n_rows, uint16_t *__restrict__ out) {
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    const int row = blockIdx.x;                   // b * Hq + h
+    const int lane = threadIdx.x & 31;
+    const int row = blockIdx.x * 4 + (threadIdx.x >> 5);   // b * Hq + h
+    if (row >= n_rows) return;
     const int b = row / Hq;
-    const int tid = threadIdx.x, lane = tid & 31;
     const int len = lens[b];
     uint16_t *o = out + (size_t)row * D;
+    constexpr int kLanes = D / 4;
+    const bool live = lane < kLanes;
     if (len < 1 || len > max_len || len > Lmax) {
-        for (int d = tid; d < D; d += blockDim.x) o[d] = 0;
+        if (live) *reinterpret_cast<uint2 *>(o + lane * 4) = make_uint2(0, 0);
         return;
     }
     const int ns = (len + kDecCH - 1) / kDecCH;
     const float *ml = ws_ml + (size_t)row * n_splits * 2;
-    const float *po = ws_o + (size_t)row * n_splits * D + tid;
-    const bool live = tid < D;
-    float M = -INFINITY;
-    for (int i = lane; i < ns; i += 32) M = fmaxf(M, ml[2 * i]);
-    M = warp_max(M);
-    float acc = 0.f, L = 0.f;
+    const float *po = ws_o + (size_t)row * n_splits * D + lane * 4;
+    float M = -INFINITY, L = 0.f;
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
     for (int base = 0; base < ns; base += 32) {
         const int n = min(32, ns - base);
-        float pv[32];
+        float4 pv[32];
 #pragma unroll
         for (int jj = 0; jj < 32; ++jj)
-            pv[jj] = (live && jj < n) ? po[(size_t)(base + jj) * D] : 0.f;
-        float w = 0.f;
-        if (lane < n) {
-            const float2 mi = *reinterpret_cast<const float2 *>(ml + 2 * (base + lane));
-            w = ex2(mi.x - M);
-            L = fmaf(w, mi.y, L);
-        }
+            pv[jj] = (live && jj < n)
+                         ? *reinterpret_cast<const float4 *>(po + (size_t)(base + jj) * D)
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float2 mi = lane < n ? *reinterpret_cast<const float2 *>(ml + 2 * (base + lane))
+                                   : make_float2(-INFINITY, 0.f);
+        const float mn = fmaxf(M, warp_max(mi.x));
+        const float alpha = ex2(M - mn);          // 0 on the first group
+        const float w = lane < n ? ex2(mi.x - mn) : 0.f;
+        L = fmaf(L, alpha, warp_sum(w * mi.y));
+        a0 *= alpha;
+        a1 *= alpha;
+        a2 *= alpha;
+        a3 *= alpha;
+        M = mn;
 #pragma unroll
-        for (int jj = 0; jj < 32; ++jj) acc = fmaf(__shfl_sync(0xffffffffu, w, jj), pv[jj], acc);
+        for (int jj = 0; jj < 32; ++jj) {
+            const float wj = __shfl_sync(0xffffffffu, w, jj);
+            a0 = fmaf(wj, pv[jj].x, a0);
+            a1 = fmaf(wj, pv[jj].y, a1);
+            a2 = fmaf(wj, pv[jj].z, a2);
+            a3 = fmaf(wj, pv[jj].w, a3);
+        }
     }
-    L = warp_sum(L);
-    if (live) o[tid] = (uint16_t)(pack_bf16x2(acc / L, 0.f) & 0xffffu);
+    if (live) {
+        const float inv = 1.f / L;
+        *reinterpret_cast<uint2 *>(o + lane * 4) =
+            make_uint2(pack_bf16x2(a0 * inv, a1 * inv), pack_bf16x2(a2 * inv, a3 * inv));
+    }
 }
 
 template <int D, int G>
@@ -372,11 +395,11 @@ cudaError_t launch_decode(const void *q, const void *kc, const void *vc, const i
                            lens, max_len, Hq, Hkv, Lmax, scale_log2, n_splits, n_sub, ws_ml, ws_o,
                            status);
     if (e != cudaSuccess) return e;
-    cfg.gridDim = dim3((unsigned)(B * Hq));
+    cfg.gridDim = dim3((unsigned)((B * Hq + 3) / 4));
     cfg.blockDim = dim3(128);
     cfg.dynamicSmemBytes = 0;
-    return cudaLaunchKernelEx(&cfg, decode_merge_kernel, (const float *)ws_ml, (const float *)ws_o,
-                              lens, max_len, Hq, D, Lmax, n_splits, static_cast<uint16_t *>(out));
+    return cudaLaunchKernelEx(&cfg, decode_merge_kernel<D>, (const float *)ws_ml, (const float *)ws_o,
+                              lens, max_len, Hq, Lmax, n_splits, B * Hq, static_cast<uint16_t *>(out));
 }
 
 // Query heads per CTA: the largest of {3, 2, 1} (D = 128) or {4, 3, 2, 1}
@@ -457,30 +480,60 @@ extern "C" gqa_status gqa_decode(const void *q, const void *k_cache, const void 
 // caller workspace.  The array is created with the module on every GPU that
 // loads the library and lives until the process exits; the decode needs no
 // part of it to start at zero.  Host code cannot use `g_noalloc_scratch` as an
-// address (it names a host-side stand-in), so the device address is looked up
-// once per device with cudaGetSymbolAddress.
+// address (it names a host-side stand-in), so the array's device address is
+// looked up with cudaGetSymbolAddress the first time a CUDA context calls, and
+// kept for that context: the address belongs to the context the module was
+// loaded into, so a caller that runs its own (non-primary) context on a device
+// gets that context's copy, never another context's.
 namespace {
 
 constexpr size_t kNoAllocScratchBytes = GQA_DECODE_NOALLOC_SCRATCH_BYTES;
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_noalloc_mutex;
-void *g_noalloc_ptr[kMaxDevices] = {};
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
 
-// Device address of the scratch array on the current device (looked up once).
-gqa_status noalloc_scratch(void **ptr) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return GQA_ERR_CUDA;
-    if (dev < 0 || dev >= kMaxDevices) return GQA_ERR_UNSUPPORTED;
-    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-    if (!g_noalloc_ptr[dev]) {
+CtxGetCurrentFn ctx_get_current() {
+    static CtxGetCurrentFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
         void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p)
-            return GQA_ERR_CUDA;
-        g_noalloc_ptr[dev] = p;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) ==
+                cudaSuccess && q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<CtxGetCurrentFn>(p);
+    });
+    return fn;
+}
+
+constexpr int kMaxContexts = 64;
+std::mutex g_noalloc_mutex;
+CUcontext g_noalloc_ctx[kMaxContexts] = {};
+void *g_noalloc_ptr[kMaxContexts] = {};
+int g_noalloc_n = 0;
+
+// Device address of the scratch array in the calling thread's current context.
+gqa_status noalloc_scratch(void **ptr) {
+    CtxGetCurrentFn cur = ctx_get_current();
+    if (!cur) return GQA_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    CUcontext ctx = nullptr;
+    if (cur(&ctx) != CUDA_SUCCESS) return GQA_ERR_CUDA;
+    for (int i = 0; ctx && i < g_noalloc_n; ++i)
+        if (g_noalloc_ctx[i] == ctx) {
+            *ptr = g_noalloc_ptr[i];
+            return GQA_OK;
+        }
+    // First call from this context (with no context current yet, the runtime
+    // makes the device's primary context current here).
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return GQA_ERR_CUDA;
+    if (cur(&ctx) != CUDA_SUCCESS || !ctx) return GQA_ERR_CUDA;
+    if (g_noalloc_n < kMaxContexts) {
+        g_noalloc_ctx[g_noalloc_n] = ctx;
+        g_noalloc_ptr[g_noalloc_n] = p;
+        ++g_noalloc_n;
     }
-    *ptr = g_noalloc_ptr[dev];
+    *ptr = p;
     return GQA_OK;
 }
 

@@ -217,9 +217,6 @@ template <int D, int kMode>
 __device__ void producer(const PfMaps &maps, PfSync &sy, uint8_t *smem, const PfGrid &g,
                          int32_t *status) {
     using S = PfShape<D>;
-    // The kernel is a programmatic dependent of the preceding one (normally the
-    // append that rotated q and filled the cache): wait for it before loading.
-    asm volatile("griddepcontrol.wait;" ::: "memory");
     int kc = 0, vc = 0, qc = 0;     // K, V tiles and Q pairs this CTA has loaded
     bool ok = true;
     PfSeq nxt = pf_w<kMode>(0) < g.n_items ? pf_seq<kMode>(g, pf_w<kMode>(0)) : pf_seq_none();
@@ -651,6 +648,13 @@ prefill_kernel(const __grid_constant__ PfMaps maps, uint16_t *__restrict__ out, 
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem = sy.tmem_base;
+    // The kernel is a programmatic dependent of the preceding one (normally the
+    // append that rotated q and filled the cache, or the kernel that computed
+    // pos0, n_tok or doc_start): every role reads what that kernel wrote -- the
+    // producer its tiles, all roles the per-sequence positions, counts and
+    // document starts -- so every thread waits for it once the prologue above
+    // (barriers, tensor memory, descriptor prefetch) is done.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 
     if (warp >= 8) {
         ptx::regs_dec<kControlRegs>();
@@ -721,8 +725,8 @@ gqa_status launch_prefill(const void *q, const void *kc, const void *vc, void *o
         return GQA_ERR_CUDA;
     const long long grid = items < sms ? items : sms;   // persistent: one CTA per SM
     // Programmatic dependent launch: the prologue (barriers, tensor memory,
-    // descriptor prefetch) overlaps the tail of the preceding kernel; the TMA
-    // producer waits for that kernel before its first load.
+    // descriptor prefetch) overlaps the tail of the preceding kernel; every
+    // thread then waits for that kernel before it reads anything.
     cudaLaunchAttribute pdl[1];
     pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     pdl[0].val.programmaticStreamSerializationAllowed = 1;
@@ -822,10 +826,13 @@ extern "C" gqa_status gqa_prefill_docs(const void *q, const void *k_cache, const
 namespace {
 
 // One thread per token: the first index t' <= t whose id equals id[t], by binary
-// search (ids are non-decreasing along a sequence; a decrease is reported).
+// search (ids are non-decreasing along a sequence; a decrease is reported).  It
+// lets a programmatic dependent (the documents prefill) start its prologue at
+// once; that kernel waits for this one to complete before reading doc_start.
 __global__ void __launch_bounds__(256)
 doc_start_kernel(const int32_t *__restrict__ doc_id, int32_t *__restrict__ doc_start, int B,
                  int T, int32_t *status) {
+    asm volatile("griddepcontrol.launch_dependents;");
     const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= (long long)B * T) return;
     const int b = (int)(i / T), t = (int)(i - (long long)b * T);

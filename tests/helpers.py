@@ -1,20 +1,23 @@
-"""Shared helpers for the GPU parity tests (no attention arithmetic here)."""
+"""Shared helpers for the GPU parity tests (no attention arithmetic here: the
+references come from the oracle and the bf16 floor built from it)."""
 import numpy as np
 import torch
 
 import oracle
 from rope_gqa_kv_b200 import inputs
 
-# Tolerance for floating-point outputs against the float64 oracle, on O(1)
-# outputs (bf16 inputs, fp32 accumulation, bf16 outputs): max |d| <= 1.5e-2 plus
-# half an ulp of the exact value in bf16 (the rounding of the answer to the
-# output format), and mean |d| <= 1e-3.  The 1e-2 of the stated bound cannot hold
-# for every element of a bf16 tensor-core path: an ideal pipeline with exact
-# arithmetic that only rounds the rotated q, k (as the cache stores them), the
-# probabilities (for the bf16 P.V product) and the output to bf16 has its worst
-# element at 0.0117 over all 50M outputs of the 8 x 2048 prompt and at 0.0119 on
-# a 2 x 200-token draw (mean 1.7e-4 .. 4.5e-4); 1.5e-2 covers that tail.
-MAX_ABS = 1.5e-2
+from ideal_pipeline import assert_floor_close, ideal_attention  # noqa: F401
+
+# Tolerance of the paths that keep fp32 probabilities (decode; RoPE and the
+# append, whose outputs are also checked to one ulp): max |d| <= 1e-2 plus half
+# an ulp of the exact value in bf16 (the rounding of the answer itself to the
+# output format: for |o| > 2.56 it alone exceeds 1e-2), and mean |d| <= 1e-3 --
+# the stated bound.  The tensor-core prefill paths (prompt, chunk, documents)
+# round the probabilities to bf16 for the P.V product, and no such pipeline
+# meets 1e-2 on every element; they are held to the bf16 floor instead,
+# element by element (ideal_pipeline.py).
+MAX_ABS = 1e-2
+DECODE_MAX_ABS = MAX_ABS
 MEAN_ABS = 1e-3
 # Gradients of the attention backward: the kernels round P and dS to bf16 for
 # the tensor cores (as flash-style backwards do) and sum many such products;
@@ -92,3 +95,47 @@ def assert_grad_close(got: torch.Tensor, want: np.ndarray, what: str):
     assert (d <= allow).all() and d.mean() <= GRAD_MEAN_ABS, \
         "%s: max |d| %.4g (worst %.3f of the bound), mean |d| %.3g" % (what, d.max(), worst, d.mean())
     return float(d.max()), float(d.mean())
+
+
+def prompt_refs(q_bits, k_bits, v_bits, qk_norm, doc_id=None, scaling=None):
+    """For a prompt prefill from position 0 on these bf16 inputs: the exact
+    result (the float64 oracle) and the bf16 floor (ideal, W) built from the
+    oracle's rotated q and K."""
+    B, T = q_bits.shape[:2]
+    exact, k_rot, v = oracle.prefill(q_bits, k_bits, v_bits, qk_norm, scaling=scaling,
+                                     doc_id=doc_id)
+    pos = oracle.positions(0, B, T)
+    q_rot = oracle.prep(q_bits, pos, qk_norm, scaling=scaling)
+    ideal, W = ideal_attention(q_rot, k_rot, v, pos, qdoc=doc_id, kdoc=doc_id)
+    return exact, ideal, W
+
+
+def chunk_refs(q_bits, k_bits, v_bits, kc, vc, pos0, qk_norm, n_tok=None):
+    """For a continuation chunk: the exact result and the bf16 floor.  kc / vc
+    [B, Hkv, Lmax, D] hold the cached prefix (bf16 bits or float64); the floor
+    sees the keys the oracle assembles -- the prefix, then the chunk's own
+    rotated keys -- with query t of sequence b at position pos0[b] + t.  Rows
+    t >= n_tok[b] are NaN in all three."""
+    B, T, Hkv = q_bits.shape[0], q_bits.shape[1], k_bits.shape[2]
+    D = q_bits.shape[3]
+    exact, k_rot = oracle.prefill_chunk(q_bits, k_bits, v_bits, kc, vc, pos0, qk_norm,
+                                        n_tok=n_tok)
+    pos0 = np.broadcast_to(np.asarray(pos0, dtype=np.int64), (B,))
+    n_tok = np.full(B, T, dtype=np.int64) if n_tok is None else np.asarray(n_tok, np.int64)
+    qpos = oracle.positions(pos0, B, T)
+    q_rot = oracle.prep(q_bits, qpos, qk_norm)
+    kw, vw, v_new = oracle.widen(kc), oracle.widen(vc), oracle.widen(v_bits)
+    Tk = max(1, int((pos0 + n_tok).max()))
+    keys = np.zeros((B, Tk, Hkv, D))
+    vals = np.zeros((B, Tk, Hkv, D))
+    for b in range(B):
+        P, n = int(pos0[b]), int(n_tok[b])
+        keys[b, :P] = kw[b, :, :P].transpose(1, 0, 2)
+        vals[b, :P] = vw[b, :, :P].transpose(1, 0, 2)
+        keys[b, P:P + n] = k_rot[b, :n]
+        vals[b, P:P + n] = v_new[b, :n]
+    ideal, W = ideal_attention(q_rot, keys, vals, qpos)
+    for b in range(B):
+        ideal[b, int(n_tok[b]):] = np.nan
+        W[b, int(n_tok[b]):] = np.nan
+    return exact, ideal, W

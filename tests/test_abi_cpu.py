@@ -190,3 +190,43 @@ def test_decode_graph_refuses_host_tensors():
     kc = torch.zeros(1, 1, 128, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         gqa.DecodeGraph(kc, kc.clone(), torch.zeros(1, dtype=torch.int32), 1)
+
+
+def _ptxas_registers(src):
+    """{kernel name: registers per thread} from ptxas's report for one source,
+    compiled exactly as the library build compiles it."""
+    import subprocess
+    import tempfile
+    with tempfile.TemporaryDirectory() as d:
+        cmd = ([gqa_build.nvcc()] + gqa_build.NVCC_FLAGS + ["-Xptxas", "-v", "-c", src, "-o",
+                                                         os.path.join(d, "x.o")])
+        r = subprocess.run(cmd, capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr[-2000:]
+    regs, name = {}, None
+    for ln in r.stderr.splitlines():
+        m = re.search(r"Compiling entry function '([^']+)'", ln)
+        if m:
+            name = m.group(1)
+        m = re.search(r"Used (\d+) registers", ln)
+        if m and name:
+            regs[name] = int(m.group(1))
+            name = None
+    return regs
+
+
+@pytest.mark.parametrize("src,pattern,launch_regs", [
+    ("prefill.cu", "prefill_kernel", 168),
+    ("backward.cu", "bwd_kv_kernel", 168),
+    ("backward.cu", "bwd_q_kernel", 168),
+])
+def test_tensor_core_kernels_keep_their_launch_registers(src, pattern, launch_regs):
+    """The tcgen05 kernels split their registers between warpgroups with
+    setmaxnreg (2 x 208 + 88 = 3 x 168), which only balances when ptxas gives
+    each thread exactly 168 at launch; the host refuses to launch them
+    otherwise (GQA_ERR_UNSUPPORTED).  A compiler that allocates differently is
+    caught here, on the CPU, instead of by a GPU run."""
+    regs = _ptxas_registers(os.path.join(gqa_build.CSRC, src))
+    found = {k: v for k, v in regs.items() if pattern in k}
+    assert found, "no %s instantiation in ptxas output" % pattern
+    wrong = {k: v for k, v in found.items() if v != launch_regs}
+    assert not wrong, "registers per thread differ from %d: %s" % (launch_regs, wrong)

@@ -257,3 +257,51 @@ def test_fewer_chunks_than_sms(cuda_lib):
 def test_lengths_around_unit_edges(cuda_lib):
     lens = [1, 63, 64, 65, 127, 128, 129, 191, 192, 640, 1, 2]
     _decode_vs_oracle(len(lens), 12, 4, 96, 640, lens, 93, "lengths around multiples of 64")
+
+
+def test_resume_from_host_copies_continues_bit_identically(cuda_lib):
+    """Checkpoint and resume of a generation (page "750美元从零训练3个LLM：一位开发者的
+    实战复盘", sections "3. 难点不在训练循环，而在基础设施" -- resuming after an
+    interruption -- and "5. 充分的冒烟测试与全程追踪" -- a checkpoint must load and
+    resume).  The caller owns the whole decode state: the caches and the
+    lengths.  Saved to host memory mid-generation, dropped from the device and
+    restored into fresh device buffers, the session continues exactly as an
+    uninterrupted one: every later output and the final caches bit for bit."""
+    w = inputs.BY_NAME["generation"]                 # 512-token prompt, 16q/4kv, D=64
+    x = inputs.make_inputs(w, decode_steps=24)
+    B, T = w.B, w.T
+    split = 9                                        # save after 9 generated tokens
+
+    def start():
+        kc, vc = x["k_cache"].to(DEV), x["v_cache"].to(DEV)
+        gqa.gqa_rope_append(x["q"].to(DEV), x["k"].to(DEV), x["v"].to(DEV), kc, vc,
+                            qk_norm=w.qk_norm)
+        return kc, vc, torch.full((B,), T, dtype=torch.int32, device=DEV)
+
+    def steps(kc, vc, pos, lo, hi):
+        outs = []
+        for q, k, v in x["steps"][lo:hi]:
+            outs.append(_decode_step(q.to(DEV), k.to(DEV), v.to(DEV), kc, vc, pos, w.qk_norm,
+                                     w.Lmax))
+            pos = pos + 1
+        return outs, pos
+
+    kc, vc, pos = start()
+    ref, pos = steps(kc, vc, pos, 0, len(x["steps"]))
+    torch.cuda.synchronize()
+    ref_k, ref_v = kc.cpu(), vc.cpu()
+
+    kc, vc, pos = start()
+    first, pos = steps(kc, vc, pos, 0, split)
+    torch.cuda.synchronize()
+    saved = (kc.cpu(), vc.cpu(), pos.cpu())          # the checkpoint: host copies
+    del kc, vc, pos
+    torch.cuda.empty_cache()
+    kc, vc, pos = (t.to(DEV) for t in saved)         # restored into new device buffers
+    rest, pos = steps(kc, vc, pos, split, len(x["steps"]))
+    torch.cuda.synchronize()
+    for s, (a, b) in enumerate(zip(ref, first + rest)):
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16)), "step %d" % s
+    assert torch.equal(kc.cpu().view(torch.int16), ref_k.view(torch.int16))
+    assert torch.equal(vc.cpu().view(torch.int16), ref_v.view(torch.int16))
+    assert int(pos[0]) == T + len(x["steps"])

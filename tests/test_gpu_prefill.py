@@ -2,9 +2,12 @@
 
 Each case runs the whole phase on the GPU through the C ABI -- gqa_rope_append
 on the prompt's q, k, v, then gqa_prefill -- and compares the output with the
-float64 oracle's prefill on the same bf16 inputs, element by element: fully at
-the sizes the oracle finishes in seconds (which still span several tiles and a
-ragged tail), and on sampled rows at the 3.8B-style full size.
+float64 oracle's prefill on the same bf16 inputs, element by element, at the
+sizes the oracle finishes in seconds (which still span several tiles and a
+ragged tail) and at the 3.8B-style full size the benchmark times (every one of
+its 50M outputs, a sequence at a time).  The bound is the bf16 floor of a
+tensor-core pipeline plus its stated margin (ideal_pipeline.py), and mean
+|d| <= 1e-3 against the exact result.
 """
 import numpy as np
 import pytest
@@ -14,7 +17,7 @@ import oracle
 import rope_gqa_kv_b200 as gqa
 from rope_gqa_kv_b200 import inputs
 
-from helpers import assert_close, bits
+from helpers import assert_floor_close, bits, prompt_refs
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -36,8 +39,8 @@ def test_named_workload_full_output(cuda_lib, name):
     w = inputs.BY_NAME[name]
     x = inputs.make_inputs(w, decode_steps=0)
     o = _run_phase(x, w)
-    want, _, _ = oracle.prefill(bits(x["q"]), bits(x["k"]), bits(x["v"]), w.qk_norm)
-    assert_close(o, want, name)
+    exact, ideal, W = prompt_refs(bits(x["q"]), bits(x["k"]), bits(x["v"]), w.qk_norm)
+    assert_floor_close(o, exact, ideal, W, name)
 
 
 @pytest.mark.parametrize("B,T,Hq,Hkv,D,qk", [
@@ -52,8 +55,8 @@ def test_shapes_and_tails(cuda_lib, B, T, Hq, Hkv, D, qk):
     w = inputs.custom("pf", B=B, Hq=Hq, Hkv=Hkv, D=D, T=T, qk_norm=qk, seed_index=T + D)
     x = inputs.make_inputs(w)
     o = _run_phase(x, w)
-    want, _, _ = oracle.prefill(bits(x["q"]), bits(x["k"]), bits(x["v"]), qk)
-    assert_close(o, want, "B%d T%d Hq%d Hkv%d D%d" % (B, T, Hq, Hkv, D))
+    exact, ideal, W = prompt_refs(bits(x["q"]), bits(x["k"]), bits(x["v"]), qk)
+    assert_floor_close(o, exact, ideal, W, "B%d T%d Hq%d Hkv%d D%d" % (B, T, Hq, Hkv, D))
 
 
 def test_output_rows_beyond_t_untouched(cuda_lib):
@@ -66,32 +69,23 @@ def test_output_rows_beyond_t_untouched(cuda_lib):
     assert (big[:, 70:] == 3.0).all()
 
 
-def _sample_rows(B, T, Hq, rng, n_random=400):
-    ts = [0, 1, 127, 128, 129, 255, 256, 511, 1000, 1023, 1024, T - 129, T - 2, T - 1]
-    rows = set()
-    for b in {0, B - 1}:
-        for h in {0, Hq // 2, Hq - 1}:
-            for t in ts:
-                if 0 <= t < T:
-                    rows.add((b * T + t) * Hq + h)
-    rows.update(rng.integers(0, B * T * Hq, size=n_random).tolist())
-    return np.array(sorted(rows), dtype=np.int64)
-
-
-def test_prefill_3p8b_full_size_sampled(cuda_lib):
-    """B=8, T=2048, Hq=24, Hkv=8, D=128, QK-norm: the launch the benchmark times."""
+def test_prefill_3p8b_full_size_every_element(cuda_lib):
+    """B=8, T=2048, Hq=24, Hkv=8, D=128, QK-norm: the launch the benchmark times,
+    every output element against the oracle (one sequence at a time: the
+    attention of a sequence depends on its own tokens only)."""
     w = inputs.BY_NAME["prefill_3p8b"]
     x = inputs.make_inputs(w)
-    o = _run_phase(x, w)
-    rows = _sample_rows(w.B, w.T, w.Hq, np.random.default_rng(0))
-    want, _, _ = oracle.prefill(bits(x["q"]), bits(x["k"]), bits(x["v"]), True, rows=rows)
-    got = o.reshape(-1, w.D)[torch.as_tensor(rows, device=DEV)]
-    assert_close(got, want.reshape(-1, w.D)[rows], "3.8B prefill (%d sampled rows)" % len(rows))
-    # properties that hold for every row: finite and bounded by the values' range
-    of = o.float()
-    assert torch.isfinite(of).all()
-    vmax = x["v"].float().abs().max().item()
-    assert of.abs().max().item() <= vmax + 1e-2
+    o = _run_phase(x, w).cpu()
+    worst, floor_max, means = 0.0, 0.0, []
+    for b in range(w.B):
+        sl = slice(b, b + 1)
+        exact, ideal, W = prompt_refs(bits(x["q"][sl]), bits(x["k"][sl]), bits(x["v"][sl]), True)
+        d, f, m = assert_floor_close(o[sl], exact, ideal, W, "3.8B prefill, sequence %d" % b)
+        worst, floor_max = max(worst, d), max(floor_max, f)
+        means.append(m)
+    assert np.mean(means) <= 1e-3
+    print("3.8B prefill: max|d| %.4g (floor %.4g), mean|d| %.3g over %d elements"
+          % (worst, floor_max, np.mean(means), o.numel()))
 
 
 def test_prefill_deterministic(cuda_lib):

@@ -7,8 +7,10 @@ over the cache.  Cases: whole outputs at sizes the oracle finishes in seconds
 (several tiles, prefixes that are not multiples of 128, ragged tails, every
 head_dim, MHA / GQA / MQA), per-sequence token counts with NaN padding, invalid
 sequences, agreement with gqa_prefill when every prefix is empty, a prompt
-prefilled in three chunks against one prefill, and sampled rows at the
-3.8B-style chunk size the benchmark times.
+prefilled in three chunks against one prefill, and every output element at
+the 3.8B-style chunk size the benchmark times.  The bound is the bf16 floor
+of a tensor-core pipeline plus its stated margin (ideal_pipeline.py), and mean
+|d| <= 1e-3 against the exact result.
 """
 import numpy as np
 import pytest
@@ -18,7 +20,7 @@ import oracle
 import rope_gqa_kv_b200 as gqa
 from rope_gqa_kv_b200 import inputs
 
-from helpers import assert_close, bits
+from helpers import assert_floor_close, bits, chunk_refs, ideal_attention, prompt_refs
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -39,10 +41,11 @@ def _run_chunk(x, w, n_tok=None, out=None):
     return o, dkc, dvc
 
 
-def _oracle_chunk(x, w, n_tok=None, rows=None):
-    return oracle.prefill_chunk(bits(x["q"]), bits(x["k"]), bits(x["v"]), bits(x["k_cache"]),
-                                bits(x["v_cache"]), x["lens"].numpy(), w.qk_norm, n_tok=n_tok,
-                                rows=rows)
+def _refs(x, w, n_tok=None, sl=slice(None)):
+    """(exact, ideal, W) of the chunk of sequences `sl`."""
+    return chunk_refs(bits(x["q"][sl]), bits(x["k"][sl]), bits(x["v"][sl]),
+                      bits(x["k_cache"][sl]), bits(x["v_cache"][sl]), x["lens"][sl].numpy(),
+                      w.qk_norm, n_tok=n_tok)
 
 
 @pytest.mark.parametrize("B,T,Hq,Hkv,D,qk,lo,hi", [
@@ -58,8 +61,9 @@ def test_chunk_shapes(cuda_lib, B, T, Hq, Hkv, D, qk, lo, hi):
                       cached_len_range=(lo, hi), seed_index=T + D + lo)
     x = inputs.make_inputs(w)
     o, _, _ = _run_chunk(x, w)
-    want, _ = _oracle_chunk(x, w)
-    assert_close(o, want, "chunk B%d T%d Hq%d Hkv%d D%d prefix U[%d,%d]" % (B, T, Hq, Hkv, D, lo, hi))
+    exact, ideal, W = _refs(x, w)
+    assert_floor_close(o, exact, ideal, W,
+                       "chunk B%d T%d Hq%d Hkv%d D%d prefix U[%d,%d]" % (B, T, Hq, Hkv, D, lo, hi))
 
 
 def test_chunk_token_counts_with_nan_padding(cuda_lib):
@@ -74,9 +78,10 @@ def test_chunk_token_counts_with_nan_padding(cuda_lib):
             x[key][b, n:] = float("nan")
     sentinel = torch.full((3, 300, 6, 128), 5.0, dtype=torch.bfloat16, device=DEV)
     o, _, _ = _run_chunk(x, w, n_tok=n_tok, out=sentinel)
-    want, _ = _oracle_chunk(x, w, n_tok=np.array(n_tok))
+    exact, ideal, W = _refs(x, w, n_tok=np.array(n_tok))
     for b, n in enumerate(n_tok):
-        assert_close(o[b, :n], want[b, :n], "sequence %d (%d tokens)" % (b, n))
+        assert_floor_close(o[b, :n], exact[b, :n], ideal[b, :n], W[b, :n],
+                           "sequence %d (%d tokens)" % (b, n))
         assert (o[b, n:] == 5.0).all(), "rows past n_tok[%d] were written" % b
 
 
@@ -115,8 +120,8 @@ def test_prompt_in_three_chunks_matches_one_prefill(cuda_lib):
     assert torch.equal(kc1[:, :, :T].view(torch.int16), kc2[:, :, :T].view(torch.int16))
     d = (chunked.float() - full.float()).abs()
     assert d.max().item() <= 1e-2, d.max().item()
-    want, _, _ = oracle.prefill(bits(q), bits(k), bits(v), True)
-    assert_close(chunked, want, "prompt in three chunks")
+    exact, ideal, W = prompt_refs(bits(q), bits(k), bits(v), True)
+    assert_floor_close(chunked, exact, ideal, W, "prompt in three chunks")
 
 
 def test_chunk_invalid_sequences(cuda_lib):
@@ -135,23 +140,28 @@ def test_chunk_invalid_sequences(cuda_lib):
     assert (out[0] == 7.0).all() and (out[2] == 7.0).all()
     keys = bits(kc[1:2].cpu())[:, :, :74].transpose(0, 2, 1, 3)
     vals = bits(vc[1:2].cpu())[:, :, :74].transpose(0, 2, 1, 3)
-    want = oracle.attention(oracle.bf16_to_f64(bits(q[1:2].cpu())), oracle.bf16_to_f64(keys),
-                            oracle.bf16_to_f64(vals), (10 + np.arange(T))[None, :])
-    assert_close(out[1:2], want, "valid sequence between invalid ones")
+    q64 = oracle.bf16_to_f64(bits(q[1:2].cpu()))
+    k64, v64 = oracle.bf16_to_f64(keys), oracle.bf16_to_f64(vals)
+    qpos = (10 + np.arange(T))[None, :]
+    exact = oracle.attention(q64, k64, v64, qpos)
+    ideal, W = ideal_attention(q64, k64, v64, qpos)
+    assert_floor_close(out[1:2], exact, ideal, W, "valid sequence between invalid ones")
 
 
-def test_chunk_3p8b_size_sampled(cuda_lib):
+def test_chunk_3p8b_size_every_element(cuda_lib):
     """8 sequences, prefixes U[512, 1536], 1024 new tokens, 24/8 heads, D=128,
-    QK-norm: the launch the benchmark times for continuation chunks."""
+    QK-norm: the launch the benchmark times for continuation chunks, every
+    output element against the oracle, one sequence at a time."""
     w = inputs.BY_NAME["chunked_prefill_3p8b"]
     x = inputs.make_inputs(w)
     o, _, _ = _run_chunk(x, w)
-    rng = np.random.default_rng(1)
-    ts = [0, 1, 127, 128, 255, 256, 511, 512, 767, 1000, 1022, 1023]
-    rows = {(b * w.T + t) * w.Hq + h for b in (0, 3, 7) for h in (0, 11, 23) for t in ts}
-    rows.update(rng.integers(0, w.B * w.T * w.Hq, size=300).tolist())
-    rows = np.array(sorted(rows), dtype=np.int64)
-    want, _ = _oracle_chunk(x, w, rows=rows)
-    got = o.reshape(-1, w.D)[torch.as_tensor(rows, device=DEV)]
-    assert_close(got, want.reshape(-1, w.D)[rows], "3.8B chunk (%d sampled rows)" % len(rows))
-    assert torch.isfinite(o.float()).all()
+    o = o.cpu()
+    worst, means = 0.0, []
+    for b in range(w.B):
+        exact, ideal, W = _refs(x, w, sl=slice(b, b + 1))
+        d, _, m = assert_floor_close(o[b:b + 1], exact, ideal, W, "3.8B chunk, sequence %d" % b)
+        worst = max(worst, d)
+        means.append(m)
+    assert np.mean(means) <= 1e-3
+    print("3.8B chunk: max|d| %.4g, mean|d| %.3g over %d elements" % (worst, np.mean(means),
+                                                                     o.numel()))

@@ -3,9 +3,11 @@
 Packed documents: query t sees only the earlier keys of its own document.  The
 GPU path (QK-norm + RoPE + append, document starts from the ids, the masked
 tcgen05 prefill) against the float64 oracle's prefill with the same document
-ids, at sizes the oracle finishes in seconds and on sampled rows of the
-3.8B-style packed workload; the start helper exactly; one document equal to
-gqa_prefill bit for bit; decreasing ids reported.
+ids, at sizes the oracle finishes in seconds and on every output element of
+the 3.8B-style packed workload, held to the bf16 floor of a tensor-core
+pipeline plus its stated margin (ideal_pipeline.py) and mean |d| <= 1e-3; the
+start helper exactly; one document equal to gqa_prefill bit for bit;
+decreasing ids reported; the start kernel and the prefill back to back.
 """
 import numpy as np
 import pytest
@@ -15,7 +17,7 @@ import oracle
 import rope_gqa_kv_b200 as gqa
 from rope_gqa_kv_b200 import inputs
 
-from helpers import assert_close, bits
+from helpers import assert_floor_close, bits, prompt_refs
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -68,9 +70,9 @@ def test_docs_vs_oracle(cuda_lib, B, T, Hq, Hkv, D, mean):
     ids[0, 5] = ids[0, 4] + 1          # a one-token document
     ids[0, 6:] += 2
     o = _run_docs(x, w, ids)
-    want, _, _ = oracle.prefill(bits(x["q"]), bits(x["k"]), bits(x["v"]), True,
-                                doc_id=ids.numpy())
-    assert_close(o, want, "documents B%d T%d D%d mean %g" % (B, T, D, mean))
+    exact, ideal, W = prompt_refs(bits(x["q"]), bits(x["k"]), bits(x["v"]), True,
+                                  doc_id=ids.numpy())
+    assert_floor_close(o, exact, ideal, W, "documents B%d T%d D%d mean %g" % (B, T, D, mean))
 
 
 def test_one_document_is_prefill_bit_for_bit(cuda_lib):
@@ -85,24 +87,52 @@ def test_one_document_is_prefill_bit_for_bit(cuda_lib):
     assert torch.equal(o.view(torch.int16), ref.view(torch.int16))
 
 
-def test_packed_docs_3p8b_size_sampled(cuda_lib):
+def test_doc_start_then_prefill_back_to_back(cuda_lib):
+    """gqa_doc_start followed at once by gqa_prefill_docs on the same stream, with
+    no synchronisation, five times with different document ids written into the
+    same start buffer: the prefill is a programmatic dependent of the start
+    kernel (which lets it begin its prologue early), so every role of the
+    prefill must wait for the starts of its own iteration, never read the
+    previous iteration's."""
+    B, T, Hq, Hkv, D = 2, 700, 6, 2, 128
+    w = inputs.custom("doc", B=B, Hq=Hq, Hkv=Hkv, D=D, T=T, qk_norm=True, seed_index=77)
+    x = inputs.make_inputs(w)
+    dq, dk, dv = x["q"].to(DEV), x["k"].to(DEV), x["v"].to(DEV)
+    kc, vc = x["k_cache"].to(DEV), x["v_cache"].to(DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    gqa.gqa_rope_append(dq, dk, dv, kc, vc, qk_norm=True, status=status)
+    means = (30.0, 700.0, 90.0, 1e6, 15.0)       # short, long, one per row, ...
+    ids_dev = [inputs.packed_doc_ids(B, T, m, seed=300 + i).to(DEV) for i, m in enumerate(means)]
+    starts = torch.full((B, T), -1, dtype=torch.int32, device=DEV)
+    torch.cuda.synchronize()
+    outs = []
+    for ids in ids_dev:
+        gqa.gqa_doc_start(ids, out=starts, status=status)
+        outs.append(gqa.gqa_prefill_docs(dq, kc, vc, starts, status=status))
+    torch.cuda.synchronize()
+    assert status.item() == 0, "device status %#x" % status.item()
+    for i, (ids, o) in enumerate(zip(ids_dev, outs)):
+        exact, ideal, W = prompt_refs(bits(x["q"]), bits(x["k"]), bits(x["v"]), True,
+                                      doc_id=ids.cpu().numpy())
+        assert_floor_close(o, exact, ideal, W, "back-to-back iteration %d" % i)
+
+
+def test_packed_docs_3p8b_size_every_element(cuda_lib):
     """8 x 2048 tokens of packed documents (mean 512 tokens), 24/8 heads, D=128,
-    QK-norm: the launch the benchmark times for document masking."""
+    QK-norm: the launch the benchmark times for document masking, every output
+    element against the oracle, one sequence at a time."""
     w = inputs.BY_NAME["prefill_3p8b"]
     x = inputs.make_inputs(w)
     ids = inputs.packed_doc_ids(w.B, w.T, 512.0, seed=2048)
-    o = _run_docs(x, w, ids)
-    rng = np.random.default_rng(2)
-    rows = rng.integers(0, w.B * w.T * w.Hq, size=400)
-    starts = _starts_np(ids.numpy())
-    # rows at document starts and ends, where the mask changes
-    for b in (0, 5):
-        for t in np.flatnonzero(np.diff(starts[b]) != 0)[:20]:
-            for tt in (t, t + 1):
-                rows = np.append(rows, (b * w.T + tt) * w.Hq + 7)
-    rows = np.unique(rows).astype(np.int64)
-    want, _, _ = oracle.prefill(bits(x["q"]), bits(x["k"]), bits(x["v"]), True, rows=rows,
-                                doc_id=ids.numpy())
-    got = o.reshape(-1, w.D)[torch.as_tensor(rows, device=DEV)]
-    assert_close(got, want.reshape(-1, w.D)[rows], "packed documents (%d rows)" % len(rows))
-    assert torch.isfinite(o.float()).all()
+    o = _run_docs(x, w, ids).cpu()
+    worst, means = 0.0, []
+    for b in range(w.B):
+        sl = slice(b, b + 1)
+        exact, ideal, W = prompt_refs(bits(x["q"][sl]), bits(x["k"][sl]), bits(x["v"][sl]), True,
+                                      doc_id=ids[sl].numpy())
+        d, _, m = assert_floor_close(o[sl], exact, ideal, W, "packed documents, sequence %d" % b)
+        worst = max(worst, d)
+        means.append(m)
+    assert np.mean(means) <= 1e-3
+    print("packed documents: max|d| %.4g, mean|d| %.3g over %d elements"
+          % (worst, np.mean(means), o.numel()))
