@@ -23,6 +23,10 @@ row's final maximum), so before the outputs are rounded the two differ by at
 most 2 * 2^-8 W = 2^-7 W, and after both round their outputs by at most that
 plus one bf16 ulp.  `assert_floor_close` holds the kernel to this bound plus a
 small stated slack, element by element.
+
+`ideal_attention_backward` is the same construction for the gradients: the
+roundings of P and dS where a bf16 backward hands them to the tensor core, and
+of dq, dk, dv, with W the sum of the absolute terms of each output.
 """
 from __future__ import annotations
 
@@ -40,6 +44,10 @@ P_ROUND = 2.0 ** -7      # 2 x (bf16 relative rounding bound 2^-8) per unit of W
 # scale * |q_i| * ulp(k_i) -- about 5e-3 for the largest normalised elements --
 # and the output by that times the weight of the key.
 SLACK = 3e-3
+# The backward's inputs are bf16 already (nothing is rotated): its slack covers
+# fp32 accumulation of dP = dO V^T, Delta and the three gradient sums, the
+# float32 log-sum-exp and the exp2 instruction.
+BW_SLACK = 1e-3
 
 
 def round_bf16(x: torch.Tensor) -> torch.Tensor:
@@ -131,3 +139,70 @@ def assert_floor_close(got, exact, ideal, W, what: str, slack: float = SLACK,
             "(<= %.3g)" % (what, int(over.sum()), g.size, i, g[i], ideal[i], exact[i],
                            d_ideal[i], margin[i], W[i], d_exact.mean(), mean_abs))
     return float(d_exact.max()), float(floor.max()), float(d_exact.mean())
+
+
+def _f64(t) -> torch.Tensor:
+    """float64 tensor of an array of values, or of bf16 bit patterns (uint16)."""
+    if isinstance(t, torch.Tensor):
+        t = t.detach().cpu()
+        return t.double() if t.dtype != torch.uint16 else t.view(torch.int16).view(torch.bfloat16).double()
+    a = np.asarray(t)
+    if a.dtype == np.uint16:
+        return torch.from_numpy(a.view(np.int16).copy()).view(torch.bfloat16).double()
+    return torch.as_tensor(a.astype(np.float64))
+
+
+def ideal_attention_backward(q, k, v, dout, o, lse, scale: float | None = None,
+                             rounded: bool = True):
+    """The bf16 floor of the attention backward, given the forward's outputs.
+
+    q, dout [B, T, Hq, D]; k, v [B, T, Hkv, D] (values, or bf16 bit patterns as
+    uint16); o [B, T, Hq, D] the forward output the backward is handed (bf16
+    values); lse [B, Hq, T] the forward's row log-sum-exp (natural log, the
+    float32 values handed).  Every step is
+    exact (float64) but the three roundings a bf16 tensor-core backward makes:
+    the probabilities P it feeds to dV = P^T dO, the dS = P (dP - Delta) it
+    feeds to dK = c dS^T Q and dQ = c dS K (Delta = rowsum(dO * o)), and the
+    three outputs.  P = exp(S - lse) is taken from the lse handed, as a kernel
+    that recomputes P does.  rounded=False skips the roundings (with the exact o
+    and lse it then equals the oracle's gradients).
+
+    Returns {"dq": (ideal, W), "dk": (ideal, W), "dv": (ideal, W)} in float64
+    numpy, dq [B, T, Hq, D], dk / dv [B, T, Hkv, D], with W the sum of the
+    absolute values of the terms each output sums (for dv: sum_i P_ij |dO_id|;
+    for dk: c sum_i |dS_ij| |Q_id|; for dq: c sum_j |dS_ij| |K_jd|; dk and dv
+    summed over the query heads of a group).  Rounding each term to bf16 moves
+    it by at most 2^-8 of itself, so a kernel that rounds the same terms after
+    fp32 arithmetic is within 2^-7 W of this pipeline before the outputs are
+    rounded: `assert_floor_close` applies unchanged.
+    """
+    q, k, v, do, o, lse = (_f64(t) for t in (q, k, v, dout, o, lse))
+    B, T, Hq, D = q.shape
+    Hkv = k.shape[2]
+    g = Hq // Hkv
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    rnd = round_bf16 if rounded else (lambda t: t)
+    dq = torch.zeros(B, T, Hq, D, dtype=torch.float64)
+    wq = torch.zeros_like(dq)
+    dk = torch.zeros(B, T, Hkv, D, dtype=torch.float64)
+    wk, dv, wv = torch.zeros_like(dk), torch.zeros_like(dk), torch.zeros_like(dk)
+    future = torch.ones(T, T, dtype=torch.bool).triu(1)
+    for b in range(B):
+        for h in range(Hq):
+            kh = h // g
+            Q, K, V, dO, O = q[b, :, h], k[b, :, kh], v[b, :, kh], do[b, :, h], o[b, :, h]
+            S = (Q @ K.T) * scale
+            P = torch.exp(S - lse[b, h][:, None]).masked_fill(future, 0.0)
+            delta = (dO * O).sum(dim=1, keepdim=True)
+            dS = P * (dO @ V.T - delta)
+            Pr, dSr = rnd(P), rnd(dS)
+            dv[b, :, kh] += Pr.T @ dO
+            wv[b, :, kh] += P.T @ dO.abs()
+            dk[b, :, kh] += dSr.T @ Q
+            wk[b, :, kh] += dS.abs().T @ Q.abs()
+            dq[b, :, h] = scale * (dSr @ K)
+            wq[b, :, h] = scale * (dS.abs() @ K.abs())
+    return {"dq": (rnd(dq).numpy(), wq.numpy()),
+            "dk": (rnd(scale * dk).numpy(), (scale * wk).numpy()),
+            "dv": (rnd(dv).numpy(), wv.numpy())}

@@ -3,9 +3,13 @@ against the float64 oracle's gradients.
 
 Full gradients at sizes the oracle finishes in seconds (ragged tails, MHA, GQA,
 MQA, every head_dim) and at the 3.8B layer's heads and length (T = 2048, 24/8
-heads, D = 128; one sequence); the forward's log-sum-exp; the forward output of
-gqa_prefill_lse equal to gqa_prefill's bit for bit; cache slots past T of dk /
-dv untouched; repeat runs bit-identical.
+heads, D = 128; one sequence), two ways: forward and backward on the GPU, every
+element within 2e-2 + one ulp of the oracle's gradient; and the backward alone,
+handed the oracle's own forward (its output rounded to bf16, its log-sum-exp to
+float32), every element within the bf16 floor of a tensor-core backward plus
+its margin (ideal_pipeline.py).  Also the forward's log-sum-exp; the forward
+output of gqa_prefill_lse equal to gqa_prefill's bit for bit; cache slots past
+T of dk / dv untouched; repeat runs bit-identical.
 """
 import numpy as np
 import pytest
@@ -15,6 +19,7 @@ import oracle
 import rope_gqa_kv_b200 as gqa
 
 from helpers import assert_grad_close, bits
+from ideal_pipeline import BW_SLACK, assert_floor_close, ideal_attention_backward
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -70,6 +75,40 @@ def test_backward_3p8b_heads_full_length(cuda_lib):
     assert_grad_close(dq, rq, "dq")
     assert_grad_close(dk[:, :, :2048].transpose(1, 2), rk, "dk")
     assert_grad_close(dv[:, :, :2048].transpose(1, 2), rv, "dv")
+
+
+def _backward_alone(q, kt, vt, dout, kc, vc, what):
+    """gqa_attention_backward handed the oracle's forward, against the floor."""
+    B, T, Hq, D = q.shape
+    rq, rk, rv, ro, rl = oracle.attention_backward(bits(q), bits(kt), bits(vt), bits(dout))
+    o16 = torch.as_tensor(ro).to(torch.bfloat16)
+    lse = torch.zeros(B, Hq, (T + 3) // 4 * 4, dtype=torch.float32)
+    lse[:, :, :T] = torch.as_tensor(rl).float()
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    dq, dk, dv = gqa.gqa_attention_backward(q.to(DEV), kc.to(DEV), vc.to(DEV), o16.to(DEV),
+                                            dout.to(DEV), lse.to(DEV), status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0, "device status %#x" % st.item()
+    ideal = ideal_attention_backward(bits(q), bits(kt), bits(vt), bits(dout), o16.double(),
+                                     lse[:, :, :T].double())
+    for name, got, exact in (("dq", dq, rq), ("dk", dk[:, :, :T].transpose(1, 2), rk),
+                             ("dv", dv[:, :, :T].transpose(1, 2), rv)):
+        d, f, m = assert_floor_close(got, exact, *ideal[name], "%s %s" % (what, name),
+                                     slack=BW_SLACK)
+        print("%s %s: max|d| %.4g (floor %.4g), mean|d| %.3g" % (what, name, d, f, m))
+
+
+@pytest.mark.parametrize("B,T,Hq,Hkv,D", [
+    (1, 128, 2, 1, 64),
+    (2, 300, 6, 2, 128),
+    (1, 513, 8, 8, 96),
+    (1, 385, 8, 1, 64),
+    (2, 1000, 8, 2, 128),
+    (1, 2048, 24, 8, 128),    # the 3.8B layer's heads, one sequence
+])
+def test_backward_alone_within_the_floor(cuda_lib, B, T, Hq, Hkv, D):
+    q, kt, vt, dout, kc, vc = _case(B, T, Hq, Hkv, D, seed=T + D + 1)
+    _backward_alone(q, kt, vt, dout, kc, vc, "B%d T%d Hq%d Hkv%d D%d" % (B, T, Hq, Hkv, D))
 
 
 def test_forward_with_lse_is_prefill_bit_for_bit(cuda_lib):
