@@ -24,12 +24,13 @@
 //                  the group's sum needs no atomics;
 //   bwd_q_kernel   per (b, query head, 128-query tile i), persistent: for every
 //                  key tile j <= i,  S = Q_i K_j^T, dP = dO_i V_j^T, dS in bf16 over
-//                  dP, dQ_i += dS K_j.
+//                  S, dQ_i += dS K_j.
 // The dK/dV kernel keeps two halves in flight (S^T / dP^T double-buffered in
 // tensor memory), so the tensor core works on one while the elementwise warps
-// work on the other.  The dQ kernel has no room for a second buffer next to dQ
-// and runs tile by tile (with 64-key halves its N = 64 MMAs re-read the whole
-// Q / dO operand per half and are bound by shared-memory bandwidth: slower).
+// work on the other.  The dQ kernel keeps S in two buffers and a single dP that
+// the warps release as soon as it is in registers, so S and dP of the next key
+// tile run while the warps work on this one (K and V in separate rings, 3 and 2
+// tiles deep, since K is held a step longer for dQ += dS K).
 // The same shared-memory tile serves as a K-major operand (the contraction over
 // D) and as an MN-major one (the contraction over its rows), as in the forward
 // kernel.  Warp roles (384 threads, three warpgroups): warps 0-7 elementwise +
@@ -69,23 +70,20 @@ struct BwShape {
     static constexpr int kStageBytes = 2 * kTileBytes + 2 * kVecBytes;   // multiple of 1024
     static constexpr int kOffStage = 2 * kTileBytes;
     static constexpr int kSmemKV = kOffStage + kStages * kStageBytes + 1024;
-    // dQ kernel: [Q_i | dO_i | stages of (K_j | V_j)]
-    static constexpr int kOffKV = 2 * kTileBytes;
-    static constexpr int kSmemQ = kOffKV + kStages * 2 * kTileBytes + 1024;
-    static_assert(kSmemKV <= 227 * 1024 && kSmemQ <= 227 * 1024, "shared memory per CTA");
-    // tensor memory columns: S [0,128) dP [128,256) then the fp32 accumulators
-    static constexpr uint32_t kColS = 0, kColDP = 128, kColAcc0 = 256, kColAcc1 = 384;
+    static_assert(kSmemKV <= 227 * 1024, "shared memory per CTA");
+    // dK/dV kernel tensor memory: the score buffers, then the fp32 accumulators
+    static constexpr uint32_t kColAcc0 = 256, kColAcc1 = 384;
 };
 
 struct BwMaps {
     CUtensorMap q, dout, k, v, lse, delta;
 };
 
-struct BwSync {
-    uint64_t fixed_full, fixed_empty;          // K_j/V_j (dK/dV kernel) or Q_i/dO_i (dQ kernel)
-    uint64_t st_full[2], st_empty[2];          // the ring
-    uint64_t s_full, p_full, acc_full, acc_empty;   // dQ kernel: one tile at a time
-    uint64_t h_full[2], h_done[2];                  // dK/dV kernel: two 64-query halves
+struct BwSync {                                 // the dK/dV kernel's barriers
+    uint64_t fixed_full, fixed_empty;          // K_j, V_j
+    uint64_t st_full[2], st_empty[2];          // the ring of (Q_i, dO_i, lse_i, Delta_i)
+    uint64_t acc_full, acc_empty;              // dK, dV accumulated / read out
+    uint64_t h_full[2], h_done[2];             // two 64-query halves
     uint64_t mma_done;
     uint32_t tmem_base;
 };
@@ -99,6 +97,12 @@ struct BwGrid {
 };
 
 __device__ __forceinline__ uint32_t A(const uint64_t &b) { return ptx::smem_addr(&b); }
+
+// Bring a tile of a 4-D tensor into L2 ahead of its load (no shared memory, no barrier).
+__device__ __forceinline__ void l2_prefetch_4d(const CUtensorMap *map, int c0, int c1, int c2, int c3) {
+    asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];"
+                 ::"l"(map), "r"(c0), "r"(c1), "r"(c2), "r"(c3) : "memory");
+}
 
 // The k-th item of this CTA: items are numbered longest first and dealt out in
 // rounds of gridDim.x in snake order (every other round backwards).
@@ -461,12 +465,39 @@ __device__ __forceinline__ void q_item(int w, const BwGrid &g, int &b, int &h, i
     h = rest - b * g.Hq;
 }
 
+// The dQ kernel's shared memory: [Q_i | dO_i | K ring (3 tiles) | V ring (2 tiles)],
+// and its tensor memory: S in two buffers [0,128) and [128,256) (dS is written
+// over the S it came from, packed bf16 in the buffer's first 64 columns), dP
+// [256, 384), the dQ accumulator [384, 384 + D).
 template <int D>
-__device__ void q_producer(const BwMaps &maps, BwSync &sy, uint8_t *smem, const BwGrid &g,
+struct BwQShape {
+    using S = BwShape<D>;
+    static constexpr int kStagesK = 3, kStagesV = 2;
+    static constexpr int kOffK = 2 * S::kTileBytes;
+    static constexpr int kOffV = kOffK + kStagesK * S::kTileBytes;
+    static constexpr int kSmem = kOffV + kStagesV * S::kTileBytes + 1024;
+    static_assert(kSmem <= 227 * 1024, "shared memory per CTA");
+    static constexpr uint32_t kColDP = 256, kColAcc = 384;
+};
+
+struct BwQSync {
+    uint64_t fixed_full, fixed_empty;          // Q_i, dO_i
+    uint64_t k_full[3], k_empty[3], v_full[2], v_empty[2];
+    uint64_t s_full[2], dp_full;               // S(u) in buffer u % 2; dP(u)
+    uint64_t dp_free;                          // dP(u) read into registers
+    uint64_t ds_full[2];                       // dS(u) written over S(u)
+    uint64_t acc_full, acc_empty;
+    uint64_t mma_done;
+    uint32_t tmem_base;
+};
+
+template <int D>
+__device__ void q_producer(const BwMaps &maps, BwQSync &sy, uint8_t *smem, const BwGrid &g,
                            int32_t *status) {
     using S = BwShape<D>;
+    using Q = BwQShape<D>;
     const int grp = g.Hq / g.Hkv;
-    int ic = 0, sc = 0;
+    int ic = 0, kc = 0, vc = 0;
     bool ok = true;
     for (int kk = 0, w = bw_w(0); w < g.n_items && ok; w = bw_w(++kk)) {
         int b, h, i;
@@ -482,71 +513,121 @@ __device__ void q_producer(const BwMaps &maps, BwSync &sy, uint8_t *smem, const 
                              A(sy.fixed_full), kb * 64, h, i * 128, b);
         }
         ++ic;
-        for (int j = 0; j <= i; ++j) {
-            const int st = sc % S::kStages;
-            ok = ptx::mbar_wait(A(sy.st_empty[st]), ((sc / S::kStages) & 1) ^ 1);
-            if (!ok) break;
-            uint8_t *base = smem + S::kOffKV + st * 2 * S::kTileBytes;
-            const uint32_t bar = A(sy.st_full[st]);
-            ptx::mbar_arrive_expect_tx(bar, 2 * S::kTileBytes);
+        if (bw_w(kk + 1) < g.n_items) {     // the next item's Q / dO into L2
+            int b2, h2, i2;
+            q_item(bw_w(kk + 1), g, b2, h2, i2);
             for (int kb = 0; kb < S::kBlocks; ++kb) {
-                ptx::tma_load_3d(ptx::smem_addr(base + kb * S::kBlockBytes), &maps.k, bar, kb * 64,
-                                 j * 128, b * g.Hkv + kvh);
-                ptx::tma_load_3d(ptx::smem_addr(base + S::kTileBytes + kb * S::kBlockBytes), &maps.v,
-                                 bar, kb * 64, j * 128, b * g.Hkv + kvh);
+                l2_prefetch_4d(&maps.q, kb * 64, h2, i2 * 128, b2);
+                l2_prefetch_4d(&maps.dout, kb * 64, h2, i2 * 128, b2);
             }
-            ++sc;
+        }
+        // K tiles run ahead of V tiles: S(u) needs K(u) before dP(u) needs V(u), and
+        // K(u) is held until dQ(u), a step after V(u) is released.
+        int jk = 0, jv = 0;
+        while (ok && jv <= i) {
+            if (jk <= i && jk < jv + Q::kStagesK) {
+                const int st = kc % Q::kStagesK;
+                ok = ptx::mbar_wait(A(sy.k_empty[st]), ((kc / Q::kStagesK) & 1) ^ 1);
+                if (!ok) break;
+                ptx::mbar_arrive_expect_tx(A(sy.k_full[st]), S::kTileBytes);
+                for (int kb = 0; kb < S::kBlocks; ++kb)
+                    ptx::tma_load_3d(ptx::smem_addr(smem + Q::kOffK + st * S::kTileBytes + kb * S::kBlockBytes),
+                                     &maps.k, A(sy.k_full[st]), kb * 64, jk * 128, b * g.Hkv + kvh);
+                ++kc;
+                ++jk;
+            }
+            if (jv < jk) {
+                const int st = vc % Q::kStagesV;
+                ok = ptx::mbar_wait(A(sy.v_empty[st]), ((vc / Q::kStagesV) & 1) ^ 1);
+                if (!ok) break;
+                ptx::mbar_arrive_expect_tx(A(sy.v_full[st]), S::kTileBytes);
+                for (int kb = 0; kb < S::kBlocks; ++kb)
+                    ptx::tma_load_3d(ptx::smem_addr(smem + Q::kOffV + st * S::kTileBytes + kb * S::kBlockBytes),
+                                     &maps.v, A(sy.v_full[st]), kb * 64, jv * 128, b * g.Hkv + kvh);
+                ++vc;
+                ++jv;
+            }
         }
     }
     if (!ok) {
         report(status, GQA_DEV_TIMEOUT);
         if (ic > 0) ptx::mbar_wait(A(sy.fixed_full), (ic - 1) & 1);
-        for (int s = (sc > S::kStages ? sc - S::kStages : 0); s < sc; ++s)
-            ptx::mbar_wait(A(sy.st_full[s % S::kStages]), (s / S::kStages) & 1);
+        for (int j = (kc > Q::kStagesK ? kc - Q::kStagesK : 0); j < kc; ++j)
+            ptx::mbar_wait(A(sy.k_full[j % Q::kStagesK]), (j / Q::kStagesK) & 1);
+        for (int j = (vc > Q::kStagesV ? vc - Q::kStagesV : 0); j < vc; ++j)
+            ptx::mbar_wait(A(sy.v_full[j % Q::kStagesV]), (j / Q::kStagesV) & 1);
     }
 }
 
+// The MMA thread walks the CTA's key tiles u (all items in turn).  Step u issues
+// S(u) into buffer u % 2 (free: dQ(u - 2) read it earlier in the same queue),
+// then dP(u) once the elementwise warps hold dP(u - 1) in registers, then
+// dQ(u - 1) += dS(u - 1) K once they have written dS(u - 1).  So S(u) and dP(u)
+// run while the warps work on tile u - 1.  At an item's first tile the
+// previous item's last dQ goes first (its epilogue waits for it).
 template <int D>
-__device__ void q_mma(BwSync &sy, uint8_t *smem, uint32_t tmem, const BwGrid &g, int32_t *status) {
+__device__ void q_mma(BwQSync &sy, uint8_t *smem, uint32_t tmem, const BwGrid &g, int32_t *status) {
     using S = BwShape<D>;
+    using Q = BwQShape<D>;
     using M = BwMma<D>;
     const uint32_t q_base = ptx::smem_addr(smem), do_base = q_base + S::kTileBytes;
-    int ic = 0, sc = 0, pc = 0, ac = 0;
+    const uint32_t k_base = ptx::smem_addr(smem + Q::kOffK), v_base = ptx::smem_addr(smem + Q::kOffV);
+    int ic = 0, ac = 0;
+    int u = 0;                    // key tiles of this CTA so far
+    bool prev_first = false;      // tile u - 1 was the first of its item
     bool ok = true;
+    // dQ(u - 1): needs dS(u - 1); the item's first tile also needs the accumulator
+    // drained by the previous item's epilogue; the item's last one completes dQ
+    auto issue_dq = [&](int t, bool first, bool last) {
+        if (!ptx::mbar_wait(A(sy.ds_full[t & 1]), (t >> 1) & 1)) return false;
+        if (first && !ptx::mbar_wait(A(sy.acc_empty), (ac & 1) ^ 1)) return false;
+        ptx::tc_fence_after();
+        M::ts(tmem + Q::kColAcc, tmem + 128 * (t & 1), k_base + (t % Q::kStagesK) * S::kTileBytes,
+              !first);
+        ptx::mma_commit(A(sy.k_empty[t % Q::kStagesK]));
+        if (last) {
+            ptx::mma_commit(A(sy.acc_full));
+            ++ac;
+        }
+        return true;
+    };
+    bool prev_last = false;
     for (int kk = 0, w = bw_w(0); w < g.n_items && ok; w = bw_w(++kk)) {
         int b, h, i;
         q_item(w, g, b, h, i);
-        ok = ptx::mbar_wait(A(sy.fixed_full), ic & 1);
-        if (!ok) break;
-        ++ic;
-        ptx::tc_fence_after();
-        for (int j = 0; j <= i && ok; ++j) {
-            const int st = sc % S::kStages;
-            ok = ptx::mbar_wait(A(sy.st_full[st]), (sc / S::kStages) & 1);
+        for (int j = 0; j <= i && ok; ++j, ++u) {
+            if (j == 0) {
+                if (u > 0) {
+                    ok = issue_dq(u - 1, prev_first, prev_last);
+                    if (!ok) break;
+                }
+                ok = ptx::mbar_wait(A(sy.fixed_full), ic & 1);
+                if (!ok) break;
+                ++ic;
+            }
+            const int ks = u % Q::kStagesK, vs = u % Q::kStagesV;
+            ok = ptx::mbar_wait(A(sy.k_full[ks]), (u / Q::kStagesK) & 1);
             if (!ok) break;
             ptx::tc_fence_after();
-            const uint32_t k_base = ptx::smem_addr(smem + S::kOffKV + st * 2 * S::kTileBytes);
-            const uint32_t v_base = k_base + S::kTileBytes;
-            M::ss(tmem + S::kColS, q_base, k_base);      // S  = Q_i K_j^T
-            M::ss(tmem + S::kColDP, do_base, v_base);    // dP = dO_i V_j^T
-            ptx::mma_commit(A(sy.s_full));
-            if (j == i) ptx::mma_commit(A(sy.fixed_empty));   // Q_i, dO_i no longer read
-            ok = ptx::mbar_wait(A(sy.p_full), pc & 1);
+            M::ss(tmem + 128 * (u & 1), q_base, k_base + ks * S::kTileBytes);     // S = Q_i K_j^T
+            ptx::mma_commit(A(sy.s_full[u & 1]));
+            ok = ptx::mbar_wait(A(sy.v_full[vs]), (u / Q::kStagesV) & 1);
+            if (ok && u > 0 && j > 0) ok = ptx::mbar_wait(A(sy.dp_free), (u - 1) & 1);
             if (!ok) break;
-            ++pc;
-            if (j == 0) {
-                ok = ptx::mbar_wait(A(sy.acc_empty), (ac & 1) ^ 1);
+            ptx::tc_fence_after();
+            M::ss(tmem + Q::kColDP, do_base, v_base + vs * S::kTileBytes);      // dP = dO_i V_j^T
+            ptx::mma_commit(A(sy.dp_full));
+            ptx::mma_commit(A(sy.v_empty[vs]));
+            if (j == i) ptx::mma_commit(A(sy.fixed_empty));                      // Q_i, dO_i read
+            if (j > 0) {
+                ok = issue_dq(u - 1, prev_first, prev_last);
                 if (!ok) break;
             }
-            ptx::tc_fence_after();
-            M::ts(tmem + S::kColAcc0, tmem + S::kColDP, k_base, j > 0);    // dQ += dS K_j
-            ptx::mma_commit(A(sy.st_empty[st]));
-            ++sc;
+            prev_first = j == 0;
+            prev_last = j == i;
         }
-        if (!ok) break;
-        ptx::mma_commit(A(sy.acc_full));
-        ++ac;
     }
+    if (ok && u > 0) ok = issue_dq(u - 1, prev_first, prev_last);
     if (!ok) report(status, GQA_DEV_TIMEOUT);
     ptx::mma_commit(A(sy.mma_done));
     ptx::mbar_wait(A(sy.mma_done), 0);
@@ -570,15 +651,17 @@ __device__ __forceinline__ void q_block(const uint32_t (&sv)[64], const uint32_t
     }
 }
 
+// thread = query row (TMEM lane); warp w takes lane quadrant w % 4 and key
+// columns [64 (w / 4), 64 (w / 4) + 64) of each tile.
 template <int D>
-__device__ void q_elementwise(BwSync &sy, uint32_t tmem, const BwGrid &g, int32_t *status) {
-    using S = BwShape<D>;
+__device__ void q_elementwise(BwQSync &sy, uint32_t tmem, const BwGrid &g, int32_t *status) {
+    using Q = BwQShape<D>;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int quad = warp & 3, half = warp >> 2;
     const int r = quad * 32 + lane;
     const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
     const int col0 = 64 * half;                  // this warp's 64 key columns
-    int sc = 0, ac = 0;
+    int u = 0, ac = 0;
     bool ok = true;
     // this row's log-sum-exp and Delta, fetched one item ahead
     auto fetch = [&](int w, float &l2, float &dl) {
@@ -597,29 +680,34 @@ __device__ void q_elementwise(BwSync &sy, uint32_t tmem, const BwGrid &g, int32_
         const float lse2 = nl2, dlt = ndl;
         if (bw_w(kk + 1) < g.n_items) fetch(bw_w(kk + 1), nl2, ndl);
         const int qrow = i * 128 + r;
-        for (int j = 0; j <= i && ok; ++j) {
-            ok = __all_sync(0xffffffffu, ptx::mbar_wait(A(sy.s_full), sc & 1));
+        for (int j = 0; j <= i && ok; ++j, ++u) {
+            ok = __all_sync(0xffffffffu, ptx::mbar_wait(A(sy.s_full[u & 1]), (u >> 1) & 1) &&
+                                             ptx::mbar_wait(A(sy.dp_full), u & 1));
             if (!ok) break;
-            ++sc;
             ptx::tc_fence_after();
+            const uint32_t sbuf = lane_addr + 128 * (u & 1);
             uint32_t sv[64], dv[64];
-            ptx::tmem_ld32(lane_addr + S::kColS + col0, *reinterpret_cast<uint32_t(*)[32]>(sv));
-            ptx::tmem_ld32(lane_addr + S::kColS + col0 + 32, *reinterpret_cast<uint32_t(*)[32]>(sv + 32));
-            ptx::tmem_ld32(lane_addr + S::kColDP + col0, *reinterpret_cast<uint32_t(*)[32]>(dv));
-            ptx::tmem_ld32(lane_addr + S::kColDP + col0 + 32, *reinterpret_cast<uint32_t(*)[32]>(dv + 32));
+            ptx::tmem_ld32(sbuf + col0, *reinterpret_cast<uint32_t(*)[32]>(sv));
+            ptx::tmem_ld32(sbuf + col0 + 32, *reinterpret_cast<uint32_t(*)[32]>(sv + 32));
+            ptx::tmem_ld32(lane_addr + Q::kColDP + col0, *reinterpret_cast<uint32_t(*)[32]>(dv));
+            ptx::tmem_ld32(lane_addr + Q::kColDP + col0 + 32, *reinterpret_cast<uint32_t(*)[32]>(dv + 32));
             ptx::tmem_wait_ld();
-            ew_sync();            // every dP column is in registers before any store
+            // dP is in registers: the next dP may overwrite it
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(A(sy.dp_free));
+            ew_sync();            // every S column is in registers before dS is stored over S
             uint32_t dd[32];
             if (j == i)
                 q_block<true>(sv, dv, j * 128 + col0, qrow, g.scale_log2, lse2, dlt, dd);
             else
                 q_block<false>(sv, dv, j * 128 + col0, qrow, g.scale_log2, lse2, dlt, dd);
-            ptx::tmem_st16(lane_addr + S::kColDP + col0 / 2, *reinterpret_cast<uint32_t(*)[16]>(dd));
-            ptx::tmem_st16(lane_addr + S::kColDP + col0 / 2 + 16, *reinterpret_cast<uint32_t(*)[16]>(dd + 16));
+            ptx::tmem_st16(sbuf + col0 / 2, *reinterpret_cast<uint32_t(*)[16]>(dd));
+            ptx::tmem_st16(sbuf + col0 / 2 + 16, *reinterpret_cast<uint32_t(*)[16]>(dd + 16));
             ptx::tmem_wait_st();
             ptx::tc_fence_before();
             __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(A(sy.p_full));
+            if (lane == 0) ptx::mbar_arrive(A(sy.ds_full[u & 1]));
         }
         if (!ok) break;
         ok = __all_sync(0xffffffffu, ptx::mbar_wait(A(sy.acc_full), ac & 1));
@@ -629,7 +717,7 @@ __device__ void q_elementwise(BwSync &sy, uint32_t tmem, const BwGrid &g, int32_
         uint16_t *dst = g.d0 + (((size_t)b * g.T + qrow) * g.Hq + h) * D;
         for (int c = half; c < D / 32; c += 2) {
             uint32_t a[32];
-            ptx::tmem_ld32(lane_addr + S::kColAcc0 + 32 * c, a);
+            ptx::tmem_ld32(lane_addr + Q::kColAcc + 32 * c, a);
             ptx::tmem_wait_ld();
             uint32_t wq[16];
 #pragma unroll
@@ -661,8 +749,6 @@ __device__ __forceinline__ void bw_setup(BwSync &sy) {
             ptx::mbar_init(A(sy.st_full[s]), 1);
             ptx::mbar_init(A(sy.st_empty[s]), 1);
         }
-        ptx::mbar_init(A(sy.s_full), 1);
-        ptx::mbar_init(A(sy.p_full), kEwWarps);     // one elected lane per elementwise warp
         ptx::mbar_init(A(sy.acc_full), 1);
         ptx::mbar_init(A(sy.acc_empty), kEwWarps);
         for (int h = 0; h < 2; ++h) {
@@ -718,15 +804,45 @@ bwd_kv_kernel(const __grid_constant__ BwMaps maps, BwGrid g, int32_t *status) {
     bw_teardown(sy);
 }
 
+__device__ __forceinline__ void bwq_setup(BwQSync &sy) {
+    if (threadIdx.x == 0) {
+        ptx::mbar_init(A(sy.fixed_full), 1);
+        ptx::mbar_init(A(sy.fixed_empty), 1);
+        for (int s = 0; s < 3; ++s) {
+            ptx::mbar_init(A(sy.k_full[s]), 1);
+            ptx::mbar_init(A(sy.k_empty[s]), 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            ptx::mbar_init(A(sy.v_full[s]), 1);
+            ptx::mbar_init(A(sy.v_empty[s]), 1);
+            ptx::mbar_init(A(sy.s_full[s]), 1);
+            ptx::mbar_init(A(sy.ds_full[s]), kEwWarps);   // one elected lane per elementwise warp
+        }
+        ptx::mbar_init(A(sy.dp_full), 1);
+        ptx::mbar_init(A(sy.dp_free), kEwWarps);
+        ptx::mbar_init(A(sy.acc_full), 1);
+        ptx::mbar_init(A(sy.acc_empty), kEwWarps);
+        ptx::mbar_init(A(sy.mma_done), 1);
+        ptx::fence_barrier_init();
+    }
+    if ((threadIdx.x >> 5) == kBwMmaWarp) {
+        ptx::tmem_alloc(ptx::smem_addr(&sy.tmem_base), 512);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+}
+
 template <int D>
 __global__ void __launch_bounds__(kBwThreads, 1)
 bwd_q_kernel(const __grid_constant__ BwMaps maps, BwGrid g, int32_t *status) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    __shared__ BwSync sy;
+    __shared__ BwQSync sy;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    bw_setup(sy);
+    bwq_setup(sy);
     asm volatile("griddepcontrol.wait;" ::: "memory");
     const uint32_t tmem = sy.tmem_base;
     if (warp >= kEwWarps) {
@@ -742,7 +858,12 @@ bwd_q_kernel(const __grid_constant__ BwMaps maps, BwGrid g, int32_t *status) {
         ptx::regs_inc<kBwEwRegs>();
         q_elementwise<D>(sy, tmem, g, status);
     }
-    bw_teardown(sy);
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == kBwMmaWarp) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(sy.tmem_base, 512);
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -856,15 +977,15 @@ gqa_status launch_backward(const void *q, const void *k, const void *v, const vo
     // 3. dQ
     {
         auto kern = bwd_q_kernel<D>;
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kSmemQ) !=
-            cudaSuccess)
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 BwQShape<D>::kSmem) != cudaSuccess)
             return GQA_ERR_CUDA;
         BwGrid gq = g;
         gq.n_items = g.nT * B * Hq;
         gq.d0 = static_cast<uint16_t *>(dq);
         gq.d1 = nullptr;
         const int grid = gq.n_items < sms ? gq.n_items : sms;
-        if (launch_pdl(kern, dim3(grid), dim3(kBwThreads), S::kSmemQ, s, maps, gq, status) !=
+        if (launch_pdl(kern, dim3(grid), dim3(kBwThreads), BwQShape<D>::kSmem, s, maps, gq, status) !=
             cudaSuccess)
             return GQA_ERR_CUDA;
     }
