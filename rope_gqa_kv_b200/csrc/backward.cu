@@ -119,21 +119,21 @@ template <int D>
 struct BwMma {
     using S = BwShape<D>;
     // D(tmem) = A(smem, K-major 128 x D) . B(smem, K-major 128 x D)^T : 128 x 128
-    static __device__ __forceinline__ void ss(uint32_t d, uint32_t a, uint32_t b) {
+    static __device__ __forceinline__ void ss(uint32_t go, uint32_t d, uint32_t a, uint32_t b) {
         constexpr uint32_t id = ptx::idesc_bf16_f32(128, 128, false);
 #pragma unroll
         for (int ks = 0; ks < S::kKSteps; ++ks) {
             const uint32_t off = (ks >> 2) * S::kBlockBytes + (ks & 3) * 32;
-            ptx::mma_ss(d, ptx::smem_desc_sw128(a + off, 16, 1024),
+            ptx::mma_ss_if(go, d, ptx::smem_desc_sw128(a + off, 16, 1024),
                         ptx::smem_desc_sw128(b + off, 16, 1024), id, ks > 0);
         }
     }
     // D(tmem, 128 x D) (+)= A(tmem, bf16 128 x 128) . B(smem, 128 rows x D, MN-major)
-    static __device__ __forceinline__ void ts(uint32_t d, uint32_t a_tmem, uint32_t b, bool acc) {
+    static __device__ __forceinline__ void ts(uint32_t go, uint32_t d, uint32_t a_tmem, uint32_t b, bool acc) {
         constexpr uint32_t id = ptx::idesc_bf16_f32(128, D, true);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
-            ptx::mma_ts(d, a_tmem + ks * 8, ptx::smem_desc_sw128(b + ks * 2048, S::kBlockBytes, 1024),
+            ptx::mma_ts_if(go, d, a_tmem + ks * 8, ptx::smem_desc_sw128(b + ks * 2048, S::kBlockBytes, 1024),
                         id, (acc || ks > 0) ? 1u : 0u);
     }
 };
@@ -143,21 +143,21 @@ template <int D>
 struct BwMmaHalf {
     using S = BwShape<D>;
     // D(tmem, 128 x 64) = A(smem, K-major 128 x D) . B(smem, 64 rows of a K-major tile)^T
-    static __device__ __forceinline__ void ss(uint32_t d, uint32_t a, uint32_t b) {
+    static __device__ __forceinline__ void ss(uint32_t go, uint32_t d, uint32_t a, uint32_t b) {
         constexpr uint32_t id = ptx::idesc_bf16_f32(128, 64, false);
 #pragma unroll
         for (int ks = 0; ks < S::kKSteps; ++ks) {
             const uint32_t off = (ks >> 2) * S::kBlockBytes + (ks & 3) * 32;
-            ptx::mma_ss(d, ptx::smem_desc_sw128(a + off, 16, 1024),
+            ptx::mma_ss_if(go, d, ptx::smem_desc_sw128(a + off, 16, 1024),
                         ptx::smem_desc_sw128(b + off, 16, 1024), id, ks > 0);
         }
     }
     // D(tmem, 128 x D) (+)= A(tmem, bf16 128 x 64) . B(smem, 64 rows x D, MN-major)
-    static __device__ __forceinline__ void ts(uint32_t d, uint32_t a_tmem, uint32_t b, bool acc) {
+    static __device__ __forceinline__ void ts(uint32_t go, uint32_t d, uint32_t a_tmem, uint32_t b, bool acc) {
         constexpr uint32_t id = ptx::idesc_bf16_f32(128, D, true);
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
-            ptx::mma_ts(d, a_tmem + ks * 8, ptx::smem_desc_sw128(b + ks * 2048, S::kBlockBytes, 1024),
+            ptx::mma_ts_if(go, d, a_tmem + ks * 8, ptx::smem_desc_sw128(b + ks * 2048, S::kBlockBytes, 1024),
                         id, (acc || ks > 0) ? 1u : 0u);
     }
 };
@@ -271,6 +271,7 @@ __device__ void kv_mma(BwSync &sy, uint8_t *smem, uint32_t tmem, const BwGrid &g
     const uint32_t k_base = ptx::smem_addr(smem), v_base = k_base + S::kTileBytes;
     int ic = 0, sc = 0, hc = 0, ac = 0;    // items, stages and halves consumed, accumulators
     bool ok = true;
+    const uint32_t go = ptx::elect_one();   // the lane that issues
     auto stage_base = [&](int st) {
         return ptx::smem_addr(smem + S::kOffStage + st * S::kStageBytes);
     };
@@ -278,21 +279,21 @@ __device__ void kv_mma(BwSync &sy, uint8_t *smem, uint32_t tmem, const BwGrid &g
     auto issue_scores = [&](int u, int st, int h) {
         const uint32_t buf = tmem + 128 * (u & 1);
         const uint32_t qb = stage_base(st) + h * 64 * 128;
-        M::ss(buf, k_base, qb);                          // S^T  = K_j Q_half^T
-        M::ss(buf + 64, v_base, qb + S::kTileBytes);     // dP^T = V_j dO_half^T
-        ptx::mma_commit(A(sy.h_full[u & 1]));
+        M::ss(go, buf, k_base, qb);                          // S^T  = K_j Q_half^T
+        M::ss(go, buf + 64, v_base, qb + S::kTileBytes);     // dP^T = V_j dO_half^T
+        ptx::mma_commit_if(go, A(sy.h_full[u & 1]));
     };
     for (int kk = 0, w = bw_w(0); w < g.n_items && ok; w = bw_w(++kk)) {
         int b, kvh, j;
         kv_item(w, g, b, kvh, j);
-        ok = ptx::mbar_wait(A(sy.fixed_full), ic & 1);
+        ok = ptx::mbar_wait_warp(A(sy.fixed_full), ic & 1);
         if (!ok) break;
         ++ic;
         ptx::tc_fence_after();
         const int n_half = 2 * grp * (g.nT - j);        // halves of this item
         const int sc0 = sc;
         // prologue: the scores of the first two halves (one stage)
-        ok = ptx::mbar_wait(A(sy.st_full[sc0 % S::kStages]), (sc0 / S::kStages) & 1);
+        ok = ptx::mbar_wait_warp(A(sy.st_full[sc0 % S::kStages]), (sc0 / S::kStages) & 1);
         if (!ok) break;
         ptx::tc_fence_after();
         issue_scores(hc, sc0 % S::kStages, 0);
@@ -300,23 +301,23 @@ __device__ void kv_mma(BwSync &sy, uint8_t *smem, uint32_t tmem, const BwGrid &g
         for (int x = 0; x < n_half && ok; ++x) {
             const int u = hc + x;
             const int st = (sc0 + x / 2) % S::kStages;
-            ok = ptx::mbar_wait(A(sy.h_done[u & 1]), (u >> 1) & 1);   // P^T, dS^T of half u
+            ok = ptx::mbar_wait_warp(A(sy.h_done[u & 1]), (u >> 1) & 1);   // P^T, dS^T of half u
             if (!ok) break;
             if (x == 0) {       // the previous item's epilogue has read dK, dV
-                ok = ptx::mbar_wait(A(sy.acc_empty), (ac & 1) ^ 1);
+                ok = ptx::mbar_wait_warp(A(sy.acc_empty), (ac & 1) ^ 1);
                 if (!ok) break;
             }
             ptx::tc_fence_after();
             const uint32_t buf = tmem + 128 * (u & 1);
             const uint32_t qb = stage_base(st) + (x & 1) * 64 * 128;
-            M::ts(tmem + S::kColAcc0, buf, qb + S::kTileBytes, x > 0);   // dV += P^T dO_half
-            M::ts(tmem + S::kColAcc1, buf + 64, qb, x > 0);              // dK += dS^T Q_half
-            if (x & 1) ptx::mma_commit(A(sy.st_empty[st]));              // both halves done
+            M::ts(go, tmem + S::kColAcc0, buf, qb + S::kTileBytes, x > 0);   // dV += P^T dO_half
+            M::ts(go, tmem + S::kColAcc1, buf + 64, qb, x > 0);              // dK += dS^T Q_half
+            if (x & 1) ptx::mma_commit_if(go, A(sy.st_empty[st]));              // both halves done
             // the scores of half u + 2 go into the buffer just consumed
             if (x + 2 < n_half) {
                 const int st2 = (sc0 + (x + 2) / 2) % S::kStages;
                 if (!(x & 1)) {
-                    ok = ptx::mbar_wait(A(sy.st_full[st2]), ((sc0 + (x + 2) / 2) / S::kStages) & 1);
+                    ok = ptx::mbar_wait_warp(A(sy.st_full[st2]), ((sc0 + (x + 2) / 2) / S::kStages) & 1);
                     if (!ok) break;
                     ptx::tc_fence_after();
                 }
@@ -326,13 +327,13 @@ __device__ void kv_mma(BwSync &sy, uint8_t *smem, uint32_t tmem, const BwGrid &g
         if (!ok) break;
         hc += n_half;
         sc += n_half / 2;
-        ptx::mma_commit(A(sy.acc_full));
-        ptx::mma_commit(A(sy.fixed_empty));
+        ptx::mma_commit_if(go, A(sy.acc_full));
+        ptx::mma_commit_if(go, A(sy.fixed_empty));
         ++ac;
     }
-    if (!ok) report(status, GQA_DEV_TIMEOUT);
-    ptx::mma_commit(A(sy.mma_done));
-    ptx::mbar_wait(A(sy.mma_done), 0);
+    if (!ok && go) report(status, GQA_DEV_TIMEOUT);
+    ptx::mma_commit_if(go, A(sy.mma_done));
+    ptx::mbar_wait_warp(A(sy.mma_done), 0);
 }
 
 // Elementwise work of the dK/dV kernel on one 64-query half: thread = key row r
@@ -576,17 +577,18 @@ __device__ void q_mma(BwQSync &sy, uint8_t *smem, uint32_t tmem, const BwGrid &g
     int u = 0;                    // key tiles of this CTA so far
     bool prev_first = false;      // tile u - 1 was the first of its item
     bool ok = true;
+    const uint32_t go = ptx::elect_one();   // the lane that issues
     // dQ(u - 1): needs dS(u - 1); the item's first tile also needs the accumulator
     // drained by the previous item's epilogue; the item's last one completes dQ
     auto issue_dq = [&](int t, bool first, bool last) {
-        if (!ptx::mbar_wait(A(sy.ds_full[t & 1]), (t >> 1) & 1)) return false;
-        if (first && !ptx::mbar_wait(A(sy.acc_empty), (ac & 1) ^ 1)) return false;
+        if (!ptx::mbar_wait_warp(A(sy.ds_full[t & 1]), (t >> 1) & 1)) return false;
+        if (first && !ptx::mbar_wait_warp(A(sy.acc_empty), (ac & 1) ^ 1)) return false;
         ptx::tc_fence_after();
-        M::ts(tmem + Q::kColAcc, tmem + 128 * (t & 1), k_base + (t % Q::kStagesK) * S::kTileBytes,
+        M::ts(go, tmem + Q::kColAcc, tmem + 128 * (t & 1), k_base + (t % Q::kStagesK) * S::kTileBytes,
               !first);
-        ptx::mma_commit(A(sy.k_empty[t % Q::kStagesK]));
+        ptx::mma_commit_if(go, A(sy.k_empty[t % Q::kStagesK]));
         if (last) {
-            ptx::mma_commit(A(sy.acc_full));
+            ptx::mma_commit_if(go, A(sy.acc_full));
             ++ac;
         }
         return true;
@@ -601,24 +603,24 @@ __device__ void q_mma(BwQSync &sy, uint8_t *smem, uint32_t tmem, const BwGrid &g
                     ok = issue_dq(u - 1, prev_first, prev_last);
                     if (!ok) break;
                 }
-                ok = ptx::mbar_wait(A(sy.fixed_full), ic & 1);
+                ok = ptx::mbar_wait_warp(A(sy.fixed_full), ic & 1);
                 if (!ok) break;
                 ++ic;
             }
             const int ks = u % Q::kStagesK, vs = u % Q::kStagesV;
-            ok = ptx::mbar_wait(A(sy.k_full[ks]), (u / Q::kStagesK) & 1);
+            ok = ptx::mbar_wait_warp(A(sy.k_full[ks]), (u / Q::kStagesK) & 1);
             if (!ok) break;
             ptx::tc_fence_after();
-            M::ss(tmem + 128 * (u & 1), q_base, k_base + ks * S::kTileBytes);     // S = Q_i K_j^T
-            ptx::mma_commit(A(sy.s_full[u & 1]));
-            ok = ptx::mbar_wait(A(sy.v_full[vs]), (u / Q::kStagesV) & 1);
-            if (ok && u > 0 && j > 0) ok = ptx::mbar_wait(A(sy.dp_free), (u - 1) & 1);
+            M::ss(go, tmem + 128 * (u & 1), q_base, k_base + ks * S::kTileBytes);     // S = Q_i K_j^T
+            ptx::mma_commit_if(go, A(sy.s_full[u & 1]));
+            ok = ptx::mbar_wait_warp(A(sy.v_full[vs]), (u / Q::kStagesV) & 1);
+            if (ok && u > 0 && j > 0) ok = ptx::mbar_wait_warp(A(sy.dp_free), (u - 1) & 1);
             if (!ok) break;
             ptx::tc_fence_after();
-            M::ss(tmem + Q::kColDP, do_base, v_base + vs * S::kTileBytes);      // dP = dO_i V_j^T
-            ptx::mma_commit(A(sy.dp_full));
-            ptx::mma_commit(A(sy.v_empty[vs]));
-            if (j == i) ptx::mma_commit(A(sy.fixed_empty));                      // Q_i, dO_i read
+            M::ss(go, tmem + Q::kColDP, do_base, v_base + vs * S::kTileBytes);      // dP = dO_i V_j^T
+            ptx::mma_commit_if(go, A(sy.dp_full));
+            ptx::mma_commit_if(go, A(sy.v_empty[vs]));
+            if (j == i) ptx::mma_commit_if(go, A(sy.fixed_empty));                      // Q_i, dO_i read
             if (j > 0) {
                 ok = issue_dq(u - 1, prev_first, prev_last);
                 if (!ok) break;
@@ -628,9 +630,9 @@ __device__ void q_mma(BwQSync &sy, uint8_t *smem, uint32_t tmem, const BwGrid &g
         }
     }
     if (ok && u > 0) ok = issue_dq(u - 1, prev_first, prev_last);
-    if (!ok) report(status, GQA_DEV_TIMEOUT);
-    ptx::mma_commit(A(sy.mma_done));
-    ptx::mbar_wait(A(sy.mma_done), 0);
+    if (!ok && go) report(status, GQA_DEV_TIMEOUT);
+    ptx::mma_commit_if(go, A(sy.mma_done));
+    ptx::mbar_wait_warp(A(sy.mma_done), 0);
 }
 
 template <bool kDiag>
@@ -794,7 +796,7 @@ bwd_kv_kernel(const __grid_constant__ BwMaps maps, BwGrid g, int32_t *status) {
             if (lane == 0) kv_producer<D>(maps, sy, smem, g, status);
             __syncwarp();
         } else if (warp == kBwMmaWarp) {
-            if (lane == 0) kv_mma<D>(sy, smem, tmem, g, status);
+            kv_mma<D>(sy, smem, tmem, g, status);   // the whole warp
             __syncwarp();
         }
     } else {
@@ -851,7 +853,7 @@ bwd_q_kernel(const __grid_constant__ BwMaps maps, BwGrid g, int32_t *status) {
             if (lane == 0) q_producer<D>(maps, sy, smem, g, status);
             __syncwarp();
         } else if (warp == kBwMmaWarp) {
-            if (lane == 0) q_mma<D>(sy, smem, tmem, g, status);
+            q_mma<D>(sy, smem, tmem, g, status);   // the whole warp
             __syncwarp();
         }
     } else {

@@ -18,7 +18,8 @@
 //   warps 0-3  softmax of tile 0 (thread = query row = TMEM lane), 208 registers
 //   warps 4-7  softmax of tile 1, 208 registers
 //   warp 8     TMA producer: Q tiles, then a K ring and a V ring    } 88
-//   warp 9     MMA issuer (one thread): S_t = Q_t K^T, O_t += P_t V } registers
+//   warp 9     MMA issuer: S_t = Q_t K^T, O_t += P_t V (one elected } registers
+//              lane issues; the whole warp runs the loop)           }
 //   warps 10-11 idle (they complete the third warpgroup)            }
 // Tensor memory (512 columns): S0 [0,128) S1 [128,256) fp32 scores, with the
 // bf16 probabilities P_t written over the first 64 columns of S_t; O0 [256, 256+D)
@@ -278,6 +279,7 @@ __device__ void mma_issuer(PfSync &sy, uint8_t *smem, uint32_t tmem, const PfGri
                            int32_t *status) {
     using S = PfShape<D>;
     constexpr bool kPHalves = kPHalvesOf<kMode>;
+    const uint32_t go = ptx::elect_one();   // the lane that issues
     constexpr uint32_t idS = ptx::idesc_bf16_f32(128, 128, false);
     constexpr uint32_t idO = ptx::idesc_bf16_f32(128, D, true);
     const uint32_t q_base = ptx::smem_addr(smem + S::kOffQ);
@@ -290,17 +292,17 @@ __device__ void mma_issuer(PfSync &sy, uint8_t *smem, uint32_t tmem, const PfGri
 #pragma unroll
         for (int ks = 0; ks < S::kKSteps; ++ks) {
             const uint32_t off = (ks >> 2) * S::kBlockBytes + (ks & 3) * 32;
-            ptx::mma_ss(tmem + t * 128, ptx::smem_desc_sw128(qa + off, 16, 1024),
+            ptx::mma_ss_if(go, tmem + t * 128, ptx::smem_desc_sw128(qa + off, 16, 1024),
                         ptx::smem_desc_sw128(ka + off, 16, 1024), idS, ks > 0);
         }
-        ptx::mma_commit(A(sy.s_full[t]));
+        ptx::mma_commit_if(go, A(sy.s_full[t]));
     };
     // O_t (+)= P_t V over key rows [16 k0, 16 k1) of the tile.
     auto issue_pv = [&](int t, int vst, bool acc, int k0, int k1) {
         const uint32_t va = v_base + vst * S::kTileBytes;
 #pragma unroll
         for (int ks = k0; ks < k1; ++ks)
-            ptx::mma_ts(tmem + 256 + t * 128, tmem + t * 128 + ks * 8,
+            ptx::mma_ts_if(go, tmem + 256 + t * 128, tmem + t * 128 + ks * 8,
                         ptx::smem_desc_sw128(va + ks * 2048, S::kBlockBytes, 1024), idO,
                         (acc || ks > 0) ? 1u : 0u);
     };
@@ -310,15 +312,15 @@ __device__ void mma_issuer(PfSync &sy, uint8_t *smem, uint32_t tmem, const PfGri
     // and documents no different, so they hand P over whole).
     auto issue_pv_halves = [&](int t, int vst, bool acc, int pc) {
         if (!kPHalves) {
-            if (!ptx::mbar_wait(A(sy.p_full[t]), pc & 1)) return false;
+            if (!ptx::mbar_wait_warp(A(sy.p_full[t]), pc & 1)) return false;
             ptx::tc_fence_after();
             issue_pv(t, vst, acc, 0, 8);
             return true;
         }
-        if (!ptx::mbar_wait(A(sy.p_half[t]), pc & 1)) return false;
+        if (!ptx::mbar_wait_warp(A(sy.p_half[t]), pc & 1)) return false;
         ptx::tc_fence_after();
         issue_pv(t, vst, acc, 0, 4);
-        if (!ptx::mbar_wait(A(sy.p_full[t]), pc & 1)) return false;
+        if (!ptx::mbar_wait_warp(A(sy.p_full[t]), pc & 1)) return false;
         ptx::tc_fence_after();
         issue_pv(t, vst, true, 4, 8);
         return true;
@@ -333,8 +335,8 @@ __device__ void mma_issuer(PfSync &sy, uint8_t *smem, uint32_t tmem, const PfGri
         if (pf_w<kMode>(k + 1) < g.n_items) nxt = pf_seq<kMode>(g, pf_w<kMode>(k + 1));
         if (I.n_kv == 0) continue;
         const int kc0 = kc;           // K ring index of key tile lo0
-        ok = ptx::mbar_wait(A(sy.q_full), qc & 1) &&
-             ptx::mbar_wait(A(sy.k_full[kc0 % S::kStagesK]), (kc0 / S::kStagesK) & 1);
+        ok = ptx::mbar_wait_warp(A(sy.q_full), qc & 1) &&
+             ptx::mbar_wait_warp(A(sy.k_full[kc0 % S::kStagesK]), (kc0 / S::kStagesK) & 1);
         if (!ok) break;
         ++qc;
         ptx::tc_fence_after();
@@ -343,11 +345,11 @@ __device__ void mma_issuer(PfSync &sy, uint8_t *smem, uint32_t tmem, const PfGri
         const bool t1_first = I.has1 && I.lo1 == I.lo0;
         issue_s(0, kc0 % S::kStagesK);
         if (t1_first) issue_s(1, kc0 % S::kStagesK);
-        ptx::mma_commit(A(sy.k_empty[kc0 % S::kStagesK]));
-        if (I.n_kv - I.lo0 == 1) ptx::mma_commit(A(sy.q_empty));   // Q no longer read
+        ptx::mma_commit_if(go, A(sy.k_empty[kc0 % S::kStagesK]));
+        if (I.n_kv - I.lo0 == 1) ptx::mma_commit_if(go, A(sy.q_empty));   // Q no longer read
         for (int j = I.lo0; j < I.n_kv && ok; ++j) {
             const int vst = vc % S::kStagesV;
-            ok = ptx::mbar_wait(A(sy.v_full[vst]), (vc / S::kStagesV) & 1);
+            ok = ptx::mbar_wait_warp(A(sy.v_full[vst]), (vc / S::kStagesV) & 1);
             if (!ok) break;
             const int jn = j + 1;
             const int kidx = kc0 + (jn - I.lo0);
@@ -358,12 +360,12 @@ __device__ void mma_issuer(PfSync &sy, uint8_t *smem, uint32_t tmem, const PfGri
                 if (!ok) break;
                 ++pc0;
                 if (jn < I.n0) {
-                    ok = ptx::mbar_wait(A(sy.k_full[kst]), (kidx / S::kStagesK) & 1);
+                    ok = ptx::mbar_wait_warp(A(sy.k_full[kst]), (kidx / S::kStagesK) & 1);
                     if (!ok) break;
                     k_next = true;
                     issue_s(0, kst);
                 } else {
-                    ptx::mma_commit(A(sy.o_final[0]));
+                    ptx::mma_commit_if(go, A(sy.o_final[0]));
                 }
             }
             if (I.has1 && j >= I.lo1 && j < I.n1) {
@@ -372,36 +374,36 @@ __device__ void mma_issuer(PfSync &sy, uint8_t *smem, uint32_t tmem, const PfGri
                 ++pc1;
                 if (jn < I.n1) {
                     if (!k_next) {
-                        ok = ptx::mbar_wait(A(sy.k_full[kst]), (kidx / S::kStagesK) & 1);
+                        ok = ptx::mbar_wait_warp(A(sy.k_full[kst]), (kidx / S::kStagesK) & 1);
                         if (!ok) break;
                         k_next = true;
                     }
                     issue_s(1, kst);
                 } else {
-                    ptx::mma_commit(A(sy.o_final[1]));
+                    ptx::mma_commit_if(go, A(sy.o_final[1]));
                 }
             } else if (kMode == kDocs && I.has1 && jn == I.lo1) {
                 // tile 1's first scores, on the next key tile
                 if (!k_next) {
-                    ok = ptx::mbar_wait(A(sy.k_full[kst]), (kidx / S::kStagesK) & 1);
+                    ok = ptx::mbar_wait_warp(A(sy.k_full[kst]), (kidx / S::kStagesK) & 1);
                     if (!ok) break;
                     k_next = true;
                 }
                 issue_s(1, kst);
             }
-            ptx::mma_commit(A(sy.v_empty[vst]));
+            ptx::mma_commit_if(go, A(sy.v_empty[vst]));
             ++vc;
             if (k_next) {
-                ptx::mma_commit(A(sy.k_empty[kst]));
-                if (jn == I.n_kv - 1) ptx::mma_commit(A(sy.q_empty));   // last S of the item
+                ptx::mma_commit_if(go, A(sy.k_empty[kst]));
+                if (jn == I.n_kv - 1) ptx::mma_commit_if(go, A(sy.q_empty));   // last S of the item
             }
         }
         kc = kc0 + (I.n_kv - I.lo0);
     }
-    if (!ok) report(status, GQA_DEV_TIMEOUT);
+    if (!ok && go) report(status, GQA_DEV_TIMEOUT);
     // No MMA may still be writing tensor memory when it is released.
-    ptx::mma_commit(A(sy.mma_done));
-    ptx::mbar_wait(A(sy.mma_done), 0);
+    ptx::mma_commit_if(go, A(sy.mma_done));
+    ptx::mbar_wait_warp(A(sy.mma_done), 0);
 }
 
 template <int D, int kMode>
@@ -459,10 +461,18 @@ __device__ void softmax_tile(PfSync &sy, uint8_t *smem, uint32_t tmem, int t, co
             const int key0 = j * 128;
             if constexpr (kMode == kDocs) {
                 if (key0 < dstart || key0 + 127 > qlim) {
+                    // this row's valid columns [lo, hi] of the tile, as a bit mask per 32
+                    const int lo = dstart - key0, hi = qlim - key0;
 #pragma unroll
-                    for (int c = 0; c < 128; ++c)
-                        if (key0 + c < dstart || key0 + c > qlim)
-                            sv[c >> 5][c & 31] = __float_as_uint(-INFINITY);
+                    for (int ch = 0; ch < 4; ++ch) {
+                        const int a = lo - 32 * ch, z = hi - 32 * ch;
+                        uint32_t msk = 0u;
+                        if (z >= 0 && a <= 31)
+                            msk = (0xffffffffu >> (31 - min(z, 31))) & (0xffffffffu << max(a, 0));
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            if (!(msk & (1u << e))) sv[ch][e] = __float_as_uint(-INFINITY);
+                    }
                 }
             } else if (key0 + 127 > lim0) {
 #pragma unroll
@@ -662,7 +672,7 @@ prefill_kernel(const __grid_constant__ PfMaps maps, uint16_t *__restrict__ out, 
             if (lane == 0) producer<D, kMode>(maps, sy, smem, g, status);
             __syncwarp();
         } else if (warp == kMmaWarp) {
-            if (lane == 0) mma_issuer<D, kMode>(sy, smem, tmem, g, status);
+            mma_issuer<D, kMode>(sy, smem, tmem, g, status);   // the whole warp
             __syncwarp();
         }
     } else {

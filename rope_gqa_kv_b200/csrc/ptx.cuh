@@ -204,6 +204,50 @@ __device__ __forceinline__ void mma_commit(uint32_t bar) {
         ::"r"(bar) : "memory");
 }
 
+// 1 in exactly one lane of a converged warp, 0 in the others.
+__device__ __forceinline__ uint32_t elect_one() {
+    uint32_t r;
+    asm volatile("{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\tselp.u32 %0, 1, 0, e;\n\t}"
+                 : "=r"(r));
+    return r;
+}
+// Forms of mma_ss / mma_ts / mma_commit that issue only where `go` is nonzero.
+// The whole MMA warp runs the issuing code and one elected lane issues: the
+// descriptors and addresses are then warp-uniform values, which the compiler
+// keeps in the uniform datapath the tcgen05 instructions read (issuing from a
+// single-lane branch measured 4-10 % slower over whole kernels).
+__device__ __forceinline__ void mma_ss_if(uint32_t go, uint32_t d_tmem, uint64_t a_desc,
+                                          uint64_t b_desc, uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, g;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "setp.ne.b32 g, %5, 0;\n\t"
+        "@g tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(go)
+        : "memory");
+}
+__device__ __forceinline__ void mma_ts_if(uint32_t go, uint32_t d_tmem, uint32_t a_tmem,
+                                          uint64_t b_desc, uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, g;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "setp.ne.b32 g, %5, 0;\n\t"
+        "@g tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(go)
+        : "memory");
+}
+__device__ __forceinline__ void mma_commit_if(uint32_t go, uint32_t bar) {
+    asm volatile(
+        "{\n\t.reg .pred g;\n\t"
+        "setp.ne.b32 g, %1, 0;\n\t"
+        "@g tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}"
+        ::"r"(bar), "r"(go) : "memory");
+}
+// A bounded wait taken by a whole warp: every lane returns the same answer.
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity) {
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity));
+}
+
 __device__ __forceinline__ void tmem_wait_ld() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
