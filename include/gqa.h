@@ -209,7 +209,9 @@ gqa_status gqa_attention_backward(const void *q, const void *k, const void *v, c
                                   float scale, void *ws, size_t ws_bytes, int32_t *status_dev,
                                   void *stream);
 
-/* Bytes of workspace gqa_attention_backward needs (0 on invalid sizes). */
+/* Bytes of workspace gqa_attention_backward needs (0 on invalid sizes): two
+ * float32 arrays [B, Hq, round_up(T, 4)], rowsum(dout * out) and the forward's
+ * log-sum-exp scaled to base 2. */
 size_t gqa_backward_workspace_bytes(int B, int T, int Hq);
 
 /*

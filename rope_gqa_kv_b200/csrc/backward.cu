@@ -13,7 +13,8 @@
 // recomputed from the forward's row log-sum-exp, never stored.
 //
 // Three launches:
-//   delta_kernel   Delta[b, h, t] = sum_d dO * O (HBM-bound, 16-byte loads);
+//   delta_kernel   Delta[b, h, t] = sum_d dO * O (HBM-bound, 16-byte loads), and
+//                  the exponent offset -lse[b, h, t] log2(e) the dK/dV kernel reads;
 //   bwd_kv_kernel  per (b, KV head, 128-key tile j), persistent: for every query
 //                  head of the group and every query tile i >= j, in halves of 64
 //                  queries,
@@ -55,7 +56,6 @@ constexpr uint32_t kBwEwRegs = 208, kBwCtlRegs = 88;   // 2 * 208 + 88 = 3 * 168
 static_assert(2 * kBwEwRegs + kBwCtlRegs == 3 * 168 && kBwThreads == 3 * 128,
               "register split must balance");
 constexpr int kEwWarps = 8;                 // elementwise warps: 2 per TMEM lane quadrant
-constexpr int kEwBarrier = 1;               // named barrier of the elementwise warps
 constexpr float kLog2e = 1.4426950408889634f;
 
 template <int D>
@@ -98,6 +98,15 @@ struct BwGrid {
 
 __device__ __forceinline__ uint32_t A(const uint64_t &b) { return ptx::smem_addr(&b); }
 
+// d = a * b on a pair of floats (one f32x2 instruction).
+__device__ __forceinline__ void fmul2(float &d0, float &d1, float a0, float a1, float b0, float b1) {
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d0), "=f"(d1)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
 // Bring a tile of a 4-D tensor into L2 ahead of its load (no shared memory, no barrier).
 __device__ __forceinline__ void l2_prefetch_4d(const CUtensorMap *map, int c0, int c1, int c2, int c3) {
     asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];"
@@ -109,10 +118,6 @@ __device__ __forceinline__ void l2_prefetch_4d(const CUtensorMap *map, int c0, i
 __device__ __forceinline__ int bw_w(int k) {
     const int G = gridDim.x, c = blockIdx.x;
     return k * G + ((k & 1) ? G - 1 - c : c);
-}
-
-__device__ __forceinline__ void ew_sync() {
-    asm volatile("bar.sync %0, %1;" ::"n"(kEwBarrier), "n"(kEwWarps * 32) : "memory");
 }
 
 template <int D>
@@ -168,7 +173,8 @@ struct BwMmaHalf {
 template <int D>
 __global__ void __launch_bounds__(256)
 delta_kernel(const uint16_t *__restrict__ out, const uint16_t *__restrict__ dout,
-             float *__restrict__ delta, int B, int T, int Hq, int stride) {
+             const float *__restrict__ lse, float *__restrict__ delta, float *__restrict__ nl2,
+             int B, int T, int Hq, int stride) {
     constexpr int kChunks = D / 8;                       // 16-byte pieces per row
     constexpr int kTPR = kChunks > 8 ? 16 : 8;            // lanes per row (power of two)
     asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -193,7 +199,9 @@ delta_kernel(const uint16_t *__restrict__ out, const uint16_t *__restrict__ dout
         const int h = (int)(row % Hq);
         const long long bt = row / Hq;
         const int t = (int)(bt % T), b = (int)(bt / T);
-        delta[((size_t)b * Hq + h) * stride + t] = acc;
+        const size_t off = ((size_t)b * Hq + h) * stride + t;
+        delta[off] = acc;
+        nl2[off] = -lse[off] * kLog2e;          // the exponent's offset, base 2
     }
 }
 
@@ -310,8 +318,8 @@ __device__ void kv_mma(BwSync &sy, uint8_t *smem, uint32_t tmem, const BwGrid &g
             ptx::tc_fence_after();
             const uint32_t buf = tmem + 128 * (u & 1);
             const uint32_t qb = stage_base(st) + (x & 1) * 64 * 128;
-            M::ts(go, tmem + S::kColAcc0, buf, qb + S::kTileBytes, x > 0);   // dV += P^T dO_half
-            M::ts(go, tmem + S::kColAcc1, buf + 64, qb, x > 0);              // dK += dS^T Q_half
+            M::ts(go, tmem + S::kColAcc0, buf + 16, qb + S::kTileBytes, x > 0);   // dV += P^T dO_half
+            M::ts(go, tmem + S::kColAcc1, buf + 80, qb, x > 0);                   // dK += dS^T Q_half
             if (x & 1) ptx::mma_commit_if(go, A(sy.st_empty[st]));              // both halves done
             // the scores of half u + 2 go into the buffer just consumed
             if (x + 2 < n_half) {
@@ -338,36 +346,40 @@ __device__ void kv_mma(BwSync &sy, uint8_t *smem, uint32_t tmem, const BwGrid &g
 
 // Elementwise work of the dK/dV kernel on one 64-query half: thread = key row r
 // of tile j; warp w takes lane quadrant w % 4 and the half's columns
-// [32 (w / 4), 32 (w / 4) + 32).  Both warps of a quadrant load their S^T and
-// dP^T columns before either stores P^T / dS^T (packed bf16, on the lower
-// columns) over them, hence the barrier between loads and stores.
+// [32 (w / 4), 32 (w / 4) + 32).  P^T and dS^T (packed bf16) go to columns
+// [16, 48) and [80, 112) of the half's buffer: each warp writes only columns it
+// has itself loaded (S^T [32 p, 32 p + 32) -> P^T [16 + 16 p, 32 + 16 p), and
+// likewise for dP^T), so the two warps of a quadrant need no barrier.  Pairs of
+// elements go through the f32x2 instructions.
 template <int D, bool kEdge>
 __device__ __forceinline__ void kv_block(const uint32_t (&sv)[32], const uint32_t (&dv)[32],
-                                         const float *lse_v, const float *del_v, int qbase,
+                                         const float *nl_v, const float *del_v, int qbase,
                                          int key, int T, float sl2, uint32_t (&pp)[16],
                                          uint32_t (&dd)[16]) {
 #pragma unroll
     for (int c4 = 0; c4 < 8; ++c4) {
-        const float4 l4 = *reinterpret_cast<const float4 *>(lse_v + 4 * c4);
+        const float4 l4 = *reinterpret_cast<const float4 *>(nl_v + 4 * c4);   // -lse log2(e)
         const float4 d4 = *reinterpret_cast<const float4 *>(del_v + 4 * c4);
-        const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+        const float nl[4] = {l4.x, l4.y, l4.z, l4.w};
         const float dl[4] = {d4.x, d4.y, d4.z, d4.w};
-        float p[4], ds[4];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int e = 4 * c4 + u;
-            float pv = ex2(fmaf(__uint_as_float(sv[e]), sl2, -lv[u] * kLog2e));
+        for (int h = 0; h < 2; ++h) {
+            const int e = 4 * c4 + 2 * h;
+            float x0, x1, y0, y1, d0, d1;
+            ptx::ffma2(x0, x1, __uint_as_float(sv[e]), __uint_as_float(sv[e + 1]), sl2, sl2,
+                       nl[2 * h], nl[2 * h + 1]);
+            float p0 = ex2(x0), p1 = ex2(x1);
             if (kEdge) {
                 const int query = qbase + e;
-                if (query < key || query >= T) pv = 0.f;
+                if (query < key || query >= T) p0 = 0.f;
+                if (query + 1 < key || query + 1 >= T) p1 = 0.f;
             }
-            p[u] = pv;
-            ds[u] = pv * (__uint_as_float(dv[e]) - dl[u]);
+            ptx::fsub2(y0, y1, __uint_as_float(dv[e]), __uint_as_float(dv[e + 1]), dl[2 * h],
+                       dl[2 * h + 1]);
+            fmul2(d0, d1, p0, p1, y0, y1);
+            pp[e / 2] = pack_bf16x2(p0, p1);
+            dd[e / 2] = pack_bf16x2(d0, d1);
         }
-        pp[2 * c4] = pack_bf16x2(p[0], p[1]);
-        pp[2 * c4 + 1] = pack_bf16x2(p[2], p[3]);
-        dd[2 * c4] = pack_bf16x2(ds[0], ds[1]);
-        dd[2 * c4 + 1] = pack_bf16x2(ds[2], ds[3]);
     }
 }
 
@@ -395,22 +407,21 @@ __device__ void kv_elementwise(BwSync &sy, uint8_t *smem, uint32_t tmem, const B
             if (!ok) break;
             ptx::tc_fence_after();
             const int col = 64 * (x & 1) + 32 * part;          // first query column of this warp
-            const float *lse_v = reinterpret_cast<const float *>(
+            const float *nl_v = reinterpret_cast<const float *>(      // -lse log2(e)
                 smem + S::kOffStage + st * S::kStageBytes + 2 * S::kTileBytes) + col;
-            const float *del_v = lse_v + 128;
+            const float *del_v = nl_v + 128;
             const uint32_t buf = lane_addr + 128 * (u & 1);
             uint32_t sv[32], dv[32];
             ptx::tmem_ld32(buf + 32 * part, sv);
             ptx::tmem_ld32(buf + 64 + 32 * part, dv);
             ptx::tmem_wait_ld();
-            ew_sync();
             uint32_t pp[16], dd[16];
             if (i == j || (i + 1) * 128 > g.T)                   // some (query, key) masked
-                kv_block<D, true>(sv, dv, lse_v, del_v, i * 128 + col, key, g.T, g.scale_log2, pp, dd);
+                kv_block<D, true>(sv, dv, nl_v, del_v, i * 128 + col, key, g.T, g.scale_log2, pp, dd);
             else
-                kv_block<D, false>(sv, dv, lse_v, del_v, i * 128 + col, key, g.T, g.scale_log2, pp, dd);
-            ptx::tmem_st16(buf + 16 * part, pp);
-            ptx::tmem_st16(buf + 64 + 16 * part, dd);
+                kv_block<D, false>(sv, dv, nl_v, del_v, i * 128 + col, key, g.T, g.scale_log2, pp, dd);
+            ptx::tmem_st16(buf + 16 + 16 * part, pp);
+            ptx::tmem_st16(buf + 80 + 16 * part, dd);
             ptx::tmem_wait_st();
             ptx::tc_fence_before();
             __syncwarp();
@@ -468,8 +479,9 @@ __device__ __forceinline__ void q_item(int w, const BwGrid &g, int &b, int &h, i
 
 // The dQ kernel's shared memory: [Q_i | dO_i | K ring (3 tiles) | V ring (2 tiles)],
 // and its tensor memory: S in two buffers [0,128) and [128,256) (dS is written
-// over the S it came from, packed bf16 in the buffer's first 64 columns), dP
-// [256, 384), the dQ accumulator [384, 384 + D).
+// over the S it came from, packed bf16 in the buffer's columns [32, 96): each
+// warp writes only columns it has loaded, so no barrier), dP [256, 384), the dQ
+// accumulator [384, 384 + D).
 template <int D>
 struct BwQShape {
     using S = BwShape<D>;
@@ -584,7 +596,7 @@ __device__ void q_mma(BwQSync &sy, uint8_t *smem, uint32_t tmem, const BwGrid &g
         if (!ptx::mbar_wait_warp(A(sy.ds_full[t & 1]), (t >> 1) & 1)) return false;
         if (first && !ptx::mbar_wait_warp(A(sy.acc_empty), (ac & 1) ^ 1)) return false;
         ptx::tc_fence_after();
-        M::ts(go, tmem + Q::kColAcc, tmem + 128 * (t & 1), k_base + (t % Q::kStagesK) * S::kTileBytes,
+        M::ts(go, tmem + Q::kColAcc, tmem + 128 * (t & 1) + 32, k_base + (t % Q::kStagesK) * S::kTileBytes,
               !first);
         ptx::mma_commit_if(go, A(sy.k_empty[t % Q::kStagesK]));
         if (last) {
@@ -641,15 +653,18 @@ __device__ __forceinline__ void q_block(const uint32_t (&sv)[64], const uint32_t
                                         uint32_t (&dd)[32]) {
 #pragma unroll
     for (int e2 = 0; e2 < 32; ++e2) {
-        float ds[2];
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const int e = 2 * e2 + u;
-            float pv = ex2(fmaf(__uint_as_float(sv[e]), sl2, -lse2));
-            if (kDiag && key0 + e > qrow) pv = 0.f;
-            ds[u] = pv * (__uint_as_float(dv[e]) - dlt);
+        const int e = 2 * e2;
+        float x0, x1, y0, y1, d0, d1;
+        ptx::ffma2(x0, x1, __uint_as_float(sv[e]), __uint_as_float(sv[e + 1]), sl2, sl2, -lse2,
+                   -lse2);
+        float p0 = ex2(x0), p1 = ex2(x1);
+        if (kDiag) {
+            if (key0 + e > qrow) p0 = 0.f;
+            if (key0 + e + 1 > qrow) p1 = 0.f;
         }
-        dd[e2] = pack_bf16x2(ds[0], ds[1]);
+        ptx::fsub2(y0, y1, __uint_as_float(dv[e]), __uint_as_float(dv[e + 1]), dlt, dlt);
+        fmul2(d0, d1, p0, p1, y0, y1);
+        dd[e2] = pack_bf16x2(d0, d1);
     }
 }
 
@@ -698,14 +713,13 @@ __device__ void q_elementwise(BwQSync &sy, uint32_t tmem, const BwGrid &g, int32
             ptx::tc_fence_before();
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(A(sy.dp_free));
-            ew_sync();            // every S column is in registers before dS is stored over S
             uint32_t dd[32];
             if (j == i)
                 q_block<true>(sv, dv, j * 128 + col0, qrow, g.scale_log2, lse2, dlt, dd);
             else
                 q_block<false>(sv, dv, j * 128 + col0, qrow, g.scale_log2, lse2, dlt, dd);
-            ptx::tmem_st16(sbuf + col0 / 2, *reinterpret_cast<uint32_t(*)[16]>(dd));
-            ptx::tmem_st16(sbuf + col0 / 2 + 16, *reinterpret_cast<uint32_t(*)[16]>(dd + 16));
+            ptx::tmem_st16(sbuf + 32 + col0 / 2, *reinterpret_cast<uint32_t(*)[16]>(dd));
+            ptx::tmem_st16(sbuf + 32 + col0 / 2 + 16, *reinterpret_cast<uint32_t(*)[16]>(dd + 16));
             ptx::tmem_wait_st();
             ptx::tc_fence_before();
             __syncwarp();
@@ -896,6 +910,7 @@ gqa_status launch_backward(const void *q, const void *k, const void *v, const vo
                            int32_t *status, cudaStream_t s) {
     using S = BwShape<D>;
     const int ls = lse_stride_of(T);
+    float *nl2 = delta + (size_t)B * Hq * ls;         // -lse log2(e), written with Delta
     BwMaps maps;
     {
         const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)Hq, (cuuint64_t)T, (cuuint64_t)B};
@@ -912,7 +927,7 @@ gqa_status launch_backward(const void *q, const void *k, const void *v, const vo
         if (!encode(&maps.k, k, 3, dims, str, box)) return GQA_ERR_CUDA;
         if (!encode(&maps.v, v, 3, dims, str, box)) return GQA_ERR_CUDA;
     }
-    if (!encode_f32_2d(&maps.lse, lse, (cuuint64_t)T, (cuuint64_t)B * Hq, (cuuint64_t)ls * 4, 128))
+    if (!encode_f32_2d(&maps.lse, nl2, (cuuint64_t)T, (cuuint64_t)B * Hq, (cuuint64_t)ls * 4, 128))
         return GQA_ERR_CUDA;
     if (!encode_f32_2d(&maps.delta, delta, (cuuint64_t)T, (cuuint64_t)B * Hq, (cuuint64_t)ls * 4,
                        128))
@@ -948,7 +963,8 @@ gqa_status launch_backward(const void *q, const void *k, const void *v, const vo
         cfg.attrs = pdl;
         cfg.numAttrs = 1;
         if (cudaLaunchKernelEx(&cfg, delta_kernel<D>, static_cast<const uint16_t *>(out),
-                               static_cast<const uint16_t *>(dout), delta, B, T, Hq, ls) !=
+                               static_cast<const uint16_t *>(dout), lse, delta, nl2, B, T, Hq,
+                               ls) !=
             cudaSuccess)
             return GQA_ERR_CUDA;
     }
@@ -999,7 +1015,7 @@ gqa_status launch_backward(const void *q, const void *k, const void *v, const vo
 
 extern "C" size_t gqa_backward_workspace_bytes(int B, int T, int Hq) {
     if (B < 1 || T < 1 || Hq < 1) return 0;
-    return (size_t)B * Hq * gqa::lse_stride_of(T) * 4;
+    return 2 * (size_t)B * Hq * gqa::lse_stride_of(T) * 4;    // Delta, then -lse log2(e)
 }
 
 extern "C" gqa_status gqa_attention_backward(const void *q, const void *k, const void *v,
@@ -1028,7 +1044,7 @@ extern "C" gqa_status gqa_attention_backward(const void *q, const void *k, const
         return GQA_ERR_UNSUPPORTED;
     const float sc = scale > 0.f ? scale : 1.0f / sqrtf((float)D);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    float *delta = static_cast<float *>(ws);
+    float *delta = static_cast<float *>(ws);          // [B, Hq, lse stride] each
     switch (D) {
         case 64: return gqa::launch_backward<64>(q, k, v, out, dout, lse, dq, dk, dv, B, T, Hq, Hkv, Lmax, sc, delta, status_dev, s);
         case 96: return gqa::launch_backward<96>(q, k, v, out, dout, lse, dq, dk, dv, B, T, Hq, Hkv, Lmax, sc, delta, status_dev, s);

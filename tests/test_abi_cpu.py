@@ -154,7 +154,8 @@ def test_backward_validation(lib):
     assert lib.gqa_attention_backward(*args(Hq=5)) == 1
     assert lib.gqa_attention_backward(*args(wsb=ctypes.c_size_t(16))) == 6
     assert lib.gqa_attention_backward(*args(w=None)) == 6
-    assert lib.gqa_backward_workspace_bytes(2, 1001, 24) == 2 * 24 * 1004 * 4
+    # Delta and the scaled log-sum-exp, float32 [B, Hq, round_up(T, 4)] each
+    assert lib.gqa_backward_workspace_bytes(2, 1001, 24) == 2 * (2 * 24 * 1004 * 4)
     assert lib.gqa_backward_workspace_bytes(0, 10, 1) == 0
     assert lib.gqa_prefill_lse(f, f, f, f, None, 1, 10, 4, 2, 64, 128, 0.0, None, None) == 1
 
