@@ -32,6 +32,12 @@
 // rescale O_t in TMEM as soon as its next scores are ready.  O_t is only
 // rescaled when the running maximum grows by more than 2^8 (the stale maximum
 // otherwise keeps p <= 256, exact in the final normalisation).
+// The output leaves through shared memory: a softmax group normalises O_t 64
+// columns at a time into its 16 KB staging (128-byte swizzle) and one of its
+// threads stores the block with the output's tensor map (whole lines; storing
+// each thread's row straight from registers writes 16 bytes of 32 rows per
+// instruction and cost 10 % of the prompt kernel).  Tiles with rows past the
+// sequence's end (the ragged last tile, chunks) store their valid rows directly.
 //
 // Documents packed into one sequence (page "训练3.8B LLM…", section "无效的方法":
 // masking at document boundaries, flex-attention style): query t sees only keys
@@ -77,20 +83,22 @@ struct PfShape {
     static constexpr int kBlocks = (D + 63) / 64;           // 128-byte column blocks
     static constexpr int kBlockBytes = 128 * 128;           // 128 rows x 128 bytes
     static constexpr int kTileBytes = kBlocks * kBlockBytes;
-    // K and V rings: as deep as the 227 KB of shared memory allows next to the
-    // two Q tiles (D = 128: K 3 + V 2 stages of 32 KB; D = 64: 4 + 4 of 16 KB).
-    static constexpr int kStagesK = D == 64 ? 4 : 3;
+    // K and V rings next to the two Q tiles and the output staging (D = 128:
+    // K 2 + V 2 stages of 32 KB; D = 64: 4 + 4 of 16 KB); the staging holds one
+    // 64-column block of an output tile per softmax group (2 x 16 KB).
+    static constexpr int kStagesK = D == 64 ? 4 : 2;
     static constexpr int kStagesV = D == 64 ? 4 : 2;
     static constexpr int kOffQ = 0;
     static constexpr int kOffK = 2 * kTileBytes;
     static constexpr int kOffV = kOffK + kStagesK * kTileBytes;
-    static constexpr int kSmem = kOffV + kStagesV * kTileBytes + 1024;   // + 1 KB alignment slack
+    static constexpr int kOffO = kOffV + kStagesV * kTileBytes;
+    static constexpr int kSmem = kOffO + 2 * kBlockBytes + 1024;   // + 1 KB alignment slack
     static_assert(kSmem <= 227 * 1024, "shared memory per CTA");
     static constexpr int kKSteps = D / 16;
 };
 
 struct PfMaps {
-    CUtensorMap q, k, v;
+    CUtensorMap q, k, v, o;
 };
 
 struct PfSync {
@@ -407,8 +415,9 @@ __device__ void mma_issuer(PfSync &sy, uint8_t *smem, uint32_t tmem, const PfGri
 }
 
 template <int D, int kMode>
-__device__ void softmax_tile(PfSync &sy, uint8_t *smem, uint32_t tmem, int t, const PfGrid &g,
-                             float scale_log2, uint16_t *__restrict__ out, int32_t *status) {
+__device__ void softmax_tile(const PfMaps &maps, PfSync &sy, uint8_t *smem, uint32_t tmem, int t,
+                             const PfGrid &g, float scale_log2, uint16_t *__restrict__ out,
+                             int32_t *status) {
     constexpr bool kPHalves = kPHalvesOf<kMode>;
     using S = PfShape<D>;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -417,6 +426,7 @@ __device__ void softmax_tile(PfSync &sy, uint8_t *smem, uint32_t tmem, int t, co
     const uint32_t s_col = t * 128, o_col = 256 + t * 128;
     const int T = g.T;
     int sc = 0, oc = 0;             // scores and outputs of this tile received
+    const bool st_issuer = (warp & 3) == 0 && lane == 0;   // issues the group's output stores
     int vc = 0;                     // V tiles of the items before this one
     bool ok = true;
     PfSeq nxt = pf_w<kMode>(0) < g.n_items ? pf_seq<kMode>(g, pf_w<kMode>(0)) : pf_seq_none();
@@ -574,28 +584,65 @@ __device__ void softmax_tile(PfSync &sy, uint8_t *smem, uint32_t tmem, int t, co
         if (kMode == kPromptLse && qrow < T)   // natural-log LSE of the scaled scores
             g.lse[((size_t)I.b * g.Hq + I.h) * g.lse_stride + qrow] =
                 (m + log2f(l)) * 0.69314718055994531f;
+        if (q_first + 128 <= I.N) {
+            // Every row of the tile is an output row: the group writes O into its
+            // shared-memory staging (128-byte swizzle, 64 columns at a time) and
+            // one thread stores the block with the tensor map, so the global
+            // writes are whole lines instead of 16 bytes from 32 rows at once.
+            uint8_t *stg = smem + S::kOffO + t * S::kBlockBytes;
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-            uint32_t o[32];
-            ptx::tmem_ld32(lane_addr + o_col + 32 * c, o);
-            ptx::tmem_wait_ld();
-            uint32_t w4[16];
+            for (int cb = 0; cb < S::kBlocks; ++cb) {
+                uint32_t o[64];
+                ptx::tmem_ld32(lane_addr + o_col + 64 * cb, *reinterpret_cast<uint32_t(*)[32]>(o));
+                if (64 * cb + 32 < D)
+                    ptx::tmem_ld32(lane_addr + o_col + 64 * cb + 32,
+                                   *reinterpret_cast<uint32_t(*)[32]>(o + 32));
+                ptx::tmem_wait_ld();
+                uint32_t w[32];
 #pragma unroll
-            for (int e = 0; e < 16; ++e)
-                w4[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l,
-                                    __uint_as_float(o[2 * e + 1]) * inv_l);
-            if (qrow < I.N) {
-                uint4 *d4 = reinterpret_cast<uint4 *>(dst + 32 * c);
-                d4[0] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-                d4[1] = make_uint4(w4[4], w4[5], w4[6], w4[7]);
-                d4[2] = make_uint4(w4[8], w4[9], w4[10], w4[11]);
-                d4[3] = make_uint4(w4[12], w4[13], w4[14], w4[15]);
+                for (int e = 0; e < 32; ++e)
+                    w[e] = 64 * cb + 2 * e < D
+                               ? pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l,
+                                             __uint_as_float(o[2 * e + 1]) * inv_l)
+                               : 0u;
+                if (st_issuer) ptx::bulk_wait_read0();     // the last store has read the staging
+                ptx::named_bar_sync(1 + t, 128);
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    *reinterpret_cast<uint4 *>(stg + row * 128 + ((c ^ (row & 7)) << 4)) =
+                        make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+                ptx::fence_proxy_async_shared();
+                ptx::named_bar_sync(1 + t, 128);
+                if (st_issuer) {
+                    ptx::tma_store_4d(&maps.o, ptx::smem_addr(stg), 64 * cb, I.h, q_first, I.b);
+                    ptx::bulk_commit();
+                }
+            }
+        } else {
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t o[32];
+                ptx::tmem_ld32(lane_addr + o_col + 32 * c, o);
+                ptx::tmem_wait_ld();
+                uint32_t w4[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    w4[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l,
+                                        __uint_as_float(o[2 * e + 1]) * inv_l);
+                if (qrow < I.N) {
+                    uint4 *d4 = reinterpret_cast<uint4 *>(dst + 32 * c);
+                    d4[0] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                    d4[1] = make_uint4(w4[4], w4[5], w4[6], w4[7]);
+                    d4[2] = make_uint4(w4[8], w4[9], w4[10], w4[11]);
+                    d4[3] = make_uint4(w4[12], w4[13], w4[14], w4[15]);
+                }
             }
         }
         // the next item's first P hand-over (after this read of O) lets the
         // MMA overwrite O with that item's first product
         ptx::tc_fence_before();
     }
+    if (st_issuer) ptx::bulk_wait0();          // the output stores have completed
     if (!ok && lane == 0) report(status, GQA_DEV_TIMEOUT);
 }
 
@@ -677,7 +724,7 @@ prefill_kernel(const __grid_constant__ PfMaps maps, uint16_t *__restrict__ out, 
         }
     } else {
         ptx::regs_inc<kSoftmaxRegs>();
-        softmax_tile<D, kMode>(sy, smem, tmem, warp >> 2, g, scale_log2, out, status);
+        softmax_tile<D, kMode>(maps, sy, smem, tmem, warp >> 2, g, scale_log2, out, status);
     }
     ptx::tc_fence_before();
     __syncthreads();
@@ -703,6 +750,7 @@ gqa_status launch_prefill(const void *q, const void *kc, const void *vc, void *o
                                    (cuuint64_t)T * Hq * D * 2};
         const cuuint32_t box[4] = {64, 1, 128, 1};
         if (!encode(&maps.q, q, 4, dims, str, box)) return GQA_ERR_CUDA;
+        if (!encode(&maps.o, out, 4, dims, str, box)) return GQA_ERR_CUDA;
     }
     {
         // A prompt (no pos0): rows beyond T are outside the map, so the copies
