@@ -69,14 +69,15 @@ struct BwShape {
     // dK/dV kernel: [K_j | V_j | stages of (Q_i | dO_i | lse_i | delta_i)]
     static constexpr int kStageBytes = 2 * kTileBytes + 2 * kVecBytes;   // multiple of 1024
     static constexpr int kOffStage = 2 * kTileBytes;
-    static constexpr int kSmemKV = kOffStage + kStages * kStageBytes + 1024;
+    static constexpr int kOffOut = kOffStage + kStages * kStageBytes;   // dK/dV staging, 64 columns
+    static constexpr int kSmemKV = kOffOut + kBlockBytes + 1024;
     static_assert(kSmemKV <= 227 * 1024, "shared memory per CTA");
     // dK/dV kernel tensor memory: the score buffers, then the fp32 accumulators
     static constexpr uint32_t kColAcc0 = 256, kColAcc1 = 384;
 };
 
 struct BwMaps {
-    CUtensorMap q, dout, k, v, lse, delta;
+    CUtensorMap q, dout, k, v, lse, delta, dk, dv;
 };
 
 struct BwSync {                                 // the dK/dV kernel's barriers
@@ -384,8 +385,8 @@ __device__ __forceinline__ void kv_block(const uint32_t (&sv)[32], const uint32_
 }
 
 template <int D>
-__device__ void kv_elementwise(BwSync &sy, uint8_t *smem, uint32_t tmem, const BwGrid &g,
-                               int32_t *status) {
+__device__ void kv_elementwise(const BwMaps &maps, BwSync &sy, uint8_t *smem, uint32_t tmem,
+                               const BwGrid &g, int32_t *status) {
     using S = BwShape<D>;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int quad = warp & 3, part = warp >> 2;
@@ -394,6 +395,7 @@ __device__ void kv_elementwise(BwSync &sy, uint8_t *smem, uint32_t tmem, const B
     const int grp = g.Hq / g.Hkv;
     int hc = 0, sc = 0, ac = 0;
     bool ok = true;
+    const bool st_issuer = threadIdx.x == 0;      // stores the staged dK / dV blocks
     for (int kk = 0, w = bw_w(0); w < g.n_items && ok; w = bw_w(++kk)) {
         int b, kvh, j;
         kv_item(w, g, b, kvh, j);
@@ -436,25 +438,63 @@ __device__ void kv_elementwise(BwSync &sy, uint8_t *smem, uint32_t tmem, const B
         ++ac;
         ptx::tc_fence_after();
         const size_t row = ((size_t)b * g.Hkv + kvh) * g.Lmax + key;
-        for (int c = part; c < D / 32; c += 2) {
-            uint32_t va[32], ka[32];
-            ptx::tmem_ld32(lane_addr + S::kColAcc0 + 32 * c, va);
-            ptx::tmem_ld32(lane_addr + S::kColAcc1 + 32 * c, ka);
-            ptx::tmem_wait_ld();
-            uint32_t wv[16], wk[16];
+        if ((j + 1) * 128 <= g.T) {
+            // a whole key tile: dV, then c dK, 64 columns at a time through the
+            // staging (128-byte swizzle; warp part p writes the block's columns
+            // [32 p, 32 p + 32) of its row), stored by one thread with the tensor map
+            uint8_t *stg = smem + S::kOffOut;
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-                wv[e] = pack_bf16x2(__uint_as_float(va[2 * e]), __uint_as_float(va[2 * e + 1]));
-                wk[e] = pack_bf16x2(__uint_as_float(ka[2 * e]) * g.scale,
-                                    __uint_as_float(ka[2 * e + 1]) * g.scale);
-            }
-            if (key < g.T) {
-                uint4 *dvp = reinterpret_cast<uint4 *>(g.d1 + row * D + 32 * c);
-                uint4 *dkp = reinterpret_cast<uint4 *>(g.d0 + row * D + 32 * c);
+            for (int blk = 0; blk < 2 * S::kBlocks; ++blk) {
+                const int tsr = blk / S::kBlocks, cb = blk % S::kBlocks;   // 0: dV, 1: dK
+                const int c = 2 * cb + part;                               // 32-column chunk
+                uint32_t w[16] = {};
+                if (32 * c < D) {
+                    uint32_t a[32];
+                    ptx::tmem_ld32(lane_addr + (tsr ? S::kColAcc1 : S::kColAcc0) + 32 * c, a);
+                    ptx::tmem_wait_ld();
+                    const float f = tsr ? g.scale : 1.f;
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        w[e] = pack_bf16x2(__uint_as_float(a[2 * e]) * f, __uint_as_float(a[2 * e + 1]) * f);
+                }
+                if (st_issuer) ptx::bulk_wait_read0();   // the last store has read the staging
+                ptx::named_bar_sync(2, kEwWarps * 32);
 #pragma unroll
                 for (int y = 0; y < 4; ++y) {
-                    dvp[y] = make_uint4(wv[4 * y], wv[4 * y + 1], wv[4 * y + 2], wv[4 * y + 3]);
-                    dkp[y] = make_uint4(wk[4 * y], wk[4 * y + 1], wk[4 * y + 2], wk[4 * y + 3]);
+                    const int ch = 4 * part + y;                              // 16-byte chunk of the row
+                    *reinterpret_cast<uint4 *>(stg + r * 128 + ((ch ^ (r & 7)) << 4)) =
+                        make_uint4(w[4 * y], w[4 * y + 1], w[4 * y + 2], w[4 * y + 3]);
+                }
+                ptx::fence_proxy_async_shared();
+                ptx::named_bar_sync(2, kEwWarps * 32);
+                if (st_issuer) {
+                    ptx::tma_store_3d(tsr ? &maps.dk : &maps.dv, ptx::smem_addr(stg), 64 * cb, j * 128,
+                                      b * g.Hkv + kvh);
+                    ptx::bulk_commit();
+                }
+            }
+        } else {
+            // the ragged last key tile: its rows below T, straight from registers
+            for (int c = part; c < D / 32; c += 2) {
+                uint32_t va[32], ka[32];
+                ptx::tmem_ld32(lane_addr + S::kColAcc0 + 32 * c, va);
+                ptx::tmem_ld32(lane_addr + S::kColAcc1 + 32 * c, ka);
+                ptx::tmem_wait_ld();
+                uint32_t wv[16], wk[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    wv[e] = pack_bf16x2(__uint_as_float(va[2 * e]), __uint_as_float(va[2 * e + 1]));
+                    wk[e] = pack_bf16x2(__uint_as_float(ka[2 * e]) * g.scale,
+                                        __uint_as_float(ka[2 * e + 1]) * g.scale);
+                }
+                if (key < g.T) {
+                    uint4 *dvp = reinterpret_cast<uint4 *>(g.d1 + row * D + 32 * c);
+                    uint4 *dkp = reinterpret_cast<uint4 *>(g.d0 + row * D + 32 * c);
+#pragma unroll
+                    for (int y = 0; y < 4; ++y) {
+                        dvp[y] = make_uint4(wv[4 * y], wv[4 * y + 1], wv[4 * y + 2], wv[4 * y + 3]);
+                        dkp[y] = make_uint4(wk[4 * y], wk[4 * y + 1], wk[4 * y + 2], wk[4 * y + 3]);
+                    }
                 }
             }
         }
@@ -462,6 +502,7 @@ __device__ void kv_elementwise(BwSync &sy, uint8_t *smem, uint32_t tmem, const B
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(A(sy.acc_empty));
     }
+    if (st_issuer) ptx::bulk_wait0();          // the dK / dV stores have completed
     if (!ok && lane == 0) report(status, GQA_DEV_TIMEOUT);
 }
 
@@ -815,7 +856,7 @@ bwd_kv_kernel(const __grid_constant__ BwMaps maps, BwGrid g, int32_t *status) {
         }
     } else {
         ptx::regs_inc<kBwEwRegs>();
-        kv_elementwise<D>(sy, smem, tmem, g, status);
+        kv_elementwise<D>(maps, sy, smem, tmem, g, status);
     }
     bw_teardown(sy);
 }
@@ -926,6 +967,8 @@ gqa_status launch_backward(const void *q, const void *k, const void *v, const vo
         const cuuint32_t box[3] = {64, 128, 1};
         if (!encode(&maps.k, k, 3, dims, str, box)) return GQA_ERR_CUDA;
         if (!encode(&maps.v, v, 3, dims, str, box)) return GQA_ERR_CUDA;
+        if (!encode(&maps.dk, dk, 3, dims, str, box)) return GQA_ERR_CUDA;
+        if (!encode(&maps.dv, dv, 3, dims, str, box)) return GQA_ERR_CUDA;
     }
     if (!encode_f32_2d(&maps.lse, nl2, (cuuint64_t)T, (cuuint64_t)B * Hq, (cuuint64_t)ls * 4, 128))
         return GQA_ERR_CUDA;

@@ -26,7 +26,7 @@
 // O1 [384, 384+D) fp32 accumulators.
 // The tensor core alternates between the tiles -- PV0(j), S0(j+1), PV1(j),
 // S1(j+1) -- so the softmax of one tile runs while the other tile's two MMAs
-// execute.  In a prompt the softmax hands P over in two halves (key columns
+// execute.  The softmax hands P over in two halves (key columns
 // 0-63, then 64-127) and the first half's P V product runs while it computes
 // the second half.  A commit after S_t(j+1) also covers PV_t(j), so the softmax may
 // rescale O_t in TMEM as soon as its next scores are ready.  O_t is only
@@ -118,9 +118,6 @@ __device__ __forceinline__ uint32_t A(const uint64_t &b) { return ptx::smem_addr
 // prefix, a prompt of packed documents, or a prompt that also stores each row's
 // log-sum-exp for the backward.
 constexpr int kPrompt = 0, kChunkMode = 1, kDocs = 2, kPromptLse = 3;
-// whether the softmax hands P to the MMA issuer in two halves (prompts)
-template <int kMode>
-constexpr bool kPHalvesOf = kMode == kPrompt || kMode == kPromptLse;
 
 struct PfItem {
     int b, h, kvh, q0, n0, n1, n_kv;
@@ -286,7 +283,6 @@ template <int D, int kMode>
 __device__ void mma_issuer(PfSync &sy, uint8_t *smem, uint32_t tmem, const PfGrid &g,
                            int32_t *status) {
     using S = PfShape<D>;
-    constexpr bool kPHalves = kPHalvesOf<kMode>;
     const uint32_t go = ptx::elect_one();   // the lane that issues
     constexpr uint32_t idS = ptx::idesc_bf16_f32(128, 128, false);
     constexpr uint32_t idO = ptx::idesc_bf16_f32(128, D, true);
@@ -314,17 +310,10 @@ __device__ void mma_issuer(PfSync &sy, uint8_t *smem, uint32_t tmem, const PfGri
                         ptx::smem_desc_sw128(va + ks * 2048, S::kBlockBytes, 1024), idO,
                         (acc || ks > 0) ? 1u : 0u);
     };
-    // Prompts: P_t arrives in two halves (key columns 0-63, then 64-127), and
-    // the product with the first half runs while the softmax computes the
-    // second (2 % faster on the 8 x 2048 prompt; chunks measured 2.7 % slower
-    // and documents no different, so they hand P over whole).
+    // P_t arrives in two halves (key columns 0-63, then 64-127), and the
+    // product with the first half runs while the softmax computes the second
+    // (2 % faster on the 8 x 2048 prompt, 4 % on chunks and documents).
     auto issue_pv_halves = [&](int t, int vst, bool acc, int pc) {
-        if (!kPHalves) {
-            if (!ptx::mbar_wait_warp(A(sy.p_full[t]), pc & 1)) return false;
-            ptx::tc_fence_after();
-            issue_pv(t, vst, acc, 0, 8);
-            return true;
-        }
         if (!ptx::mbar_wait_warp(A(sy.p_half[t]), pc & 1)) return false;
         ptx::tc_fence_after();
         issue_pv(t, vst, acc, 0, 4);
@@ -418,7 +407,6 @@ template <int D, int kMode>
 __device__ void softmax_tile(const PfMaps &maps, PfSync &sy, uint8_t *smem, uint32_t tmem, int t,
                              const PfGrid &g, float scale_log2, uint16_t *__restrict__ out,
                              int32_t *status) {
-    constexpr bool kPHalves = kPHalvesOf<kMode>;
     using S = PfShape<D>;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int row = (warp & 3) * 32 + lane;
@@ -558,7 +546,7 @@ __device__ void softmax_tile(const PfMaps &maps, PfSync &sy, uint8_t *smem, uint
                         ptx::fadd2(lb0, lb1, lb0, lb1, p0, p1);
                 }
                 ptx::tmem_st16(lane_addr + s_col + 16 * c, p);
-                if (kPHalves && c == 1) {
+                if (c == 1) {
                     clear_v_tail();
                     // first half of P (key columns 0-63) to the tensor core
                     ptx::tmem_wait_st();
@@ -569,7 +557,6 @@ __device__ void softmax_tile(const PfMaps &maps, PfSync &sy, uint8_t *smem, uint
             }
 #undef SV
             l += (la0 + la1) + (lb0 + lb1);
-            if (!kPHalves) clear_v_tail();
             ptx::tmem_wait_st();
             ptx::tc_fence_before();
             __syncwarp();
