@@ -329,13 +329,16 @@ def _max_over_ranks(x: float, dist_on: bool, dev) -> float:
 def run_ours(args, rank, world, dev, dist_on):
     layer = Layer(dev)
     peaks, peak_src = load_peaks()
-    for _ in range(args.warmup):
-        layer.step()
-    torch.cuda.synchronize()
     sampler = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
     if sampler:
         sampler.start()
         time.sleep(0.3)
+    # The warm-up steps run after the sampler's start-up pause, right before the
+    # timed steps, so that those begin on a busy GPU rather than on clocks
+    # ramping up from an idle wait.
+    for _ in range(args.warmup):
+        layer.step()
+    torch.cuda.synchronize()
 
     # -- device-resident timed region (per-kernel events on the launching stream) --
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
