@@ -94,3 +94,34 @@ def test_prefill_deterministic(cuda_lib):
     a = _run_phase(x, w)
     b = _run_phase(x, w)
     assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+def test_item_counter_slots_recycle_and_run_concurrently(cuda_lib):
+    """Items are taken from a launch-wide counter (one of 256 slots, round robin,
+    reset by the launch's last CTA): 300 launches in a row -- every slot used
+    more than once -- and two launches in flight at once on two streams all give
+    the same output bits."""
+    w = inputs.BY_NAME["prefill_3p8b"]
+    x = inputs.make_inputs(w)
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    dq, dk, dv = x["q"].to(DEV), x["k"].to(DEV), x["v"].to(DEV)
+    dkc, dvc = x["k_cache"].to(DEV), x["v_cache"].to(DEV)
+    gqa.gqa_rope_append(dq, dk, dv, dkc, dvc, qk_norm=True, max_pos0=0, status=st)
+    ref = gqa.gqa_prefill(dq, dkc, dvc, status=st)
+    out = torch.empty_like(ref)
+    for _ in range(300):
+        gqa.gqa_prefill(dq, dkc, dvc, out=out, status=st)
+    torch.cuda.synchronize()
+    assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    o1, o2 = torch.empty_like(ref), torch.empty_like(ref)
+    torch.cuda.synchronize()
+    for _ in range(5):
+        with torch.cuda.stream(s1):
+            gqa.gqa_prefill(dq, dkc, dvc, out=o1, status=st, stream=s1)
+        with torch.cuda.stream(s2):
+            gqa.gqa_prefill(dq, dkc, dvc, out=o2, status=st, stream=s2)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    assert torch.equal(o1.view(torch.int16), ref.view(torch.int16))
+    assert torch.equal(o2.view(torch.int16), ref.view(torch.int16))
