@@ -206,7 +206,9 @@ gqa_status gqa_prefill_lse(const void *q, const void *k_cache, const void *v_cac
  *   ws, ws_bytes: device scratch of gqa_backward_workspace_bytes(B, T, Hq) bytes
  *     (16-byte aligned; contents on entry do not matter).
  * Three launches (rowsum(dout * out); dk and dv per key tile; dq per query
- * tile), each a programmatic dependent of the one before.  Device errors:
+ * tile), each a programmatic dependent of the one before; the dq launch starts
+ * on the SMs the dk/dv launch frees and ends after it.  Errors:
+ * GQA_ERR_INVALID_ARG also for B > 65535 or T * Hq >= 2^31.  Device errors:
  * GQA_DEV_TIMEOUT.
  */
 gqa_status gqa_attention_backward(const void *q, const void *k, const void *v, const void *out,

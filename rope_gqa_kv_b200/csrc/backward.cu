@@ -26,12 +26,18 @@
 //   bwd_q_kernel   per (b, query head, 128-query tile i), persistent: for every
 //                  key tile j <= i,  S = Q_i K_j^T, dP = dO_i V_j^T, dS in bf16 over
 //                  S, dQ_i += dS K_j.
+// The dQ kernel needs only Delta, not dK / dV: the dK/dV kernel lets it launch
+// right away (its CTAs take the SMs the dK/dV kernel's CTAs free), and it waits
+// for the dK/dV kernel only before it exits, so the launch ends with both done.
 // The dK/dV kernel keeps two halves in flight (S^T / dP^T double-buffered in
 // tensor memory), so the tensor core works on one while the elementwise warps
 // work on the other.  The dQ kernel keeps S in two buffers and a single dP that
 // the warps release as soon as it is in registers, so S and dP of the next key
 // tile run while the warps work on this one (K and V in separate rings, 3 and 2
-// tiles deep, since K is held a step longer for dQ += dS K).
+// tiles deep, since K is held a step longer for dQ += dS K); the warps drain a
+// tile's dQ after the first key tile of their next item, so the wait for its
+// last MMA overlaps that work, and they transpose 16-byte pieces within groups
+// of four lanes so each store writes 64 contiguous bytes of eight rows.
 // The same shared-memory tile serves as a K-major operand (the contraction over
 // D) and as an MN-major one (the contraction over its rows), as in the forward
 // kernel.  Warp roles (384 threads, three warpgroups): warps 0-7 elementwise +
@@ -169,40 +175,53 @@ struct BwMmaHalf {
 };
 
 // ---------------------------------------------------------------------------
-// Delta = rowsum(dO * O): TPR lanes per (b, t, h) row, 16-byte loads
+// Delta = rowsum(dO * O): TPR lanes per (t, h) row of sequence blockIdx.y, 16-byte
+// loads, kPasses rows per lane with all their loads issued before the first sum
 // ---------------------------------------------------------------------------
-template <int D>
+template <int D, int kPasses>
 __global__ void __launch_bounds__(256)
 delta_kernel(const uint16_t *__restrict__ out, const uint16_t *__restrict__ dout,
              const float *__restrict__ lse, float *__restrict__ delta, float *__restrict__ nl2,
-             int B, int T, int Hq, int stride) {
+             int T, int Hq, int stride) {
     constexpr int kChunks = D / 8;                       // 16-byte pieces per row
     constexpr int kTPR = kChunks > 8 ? 16 : 8;            // lanes per row (power of two)
+    constexpr int kRowsPerPass = 256 / kTPR;
     asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;");
-    const int lane = threadIdx.x & 31, j = lane % kTPR;
-    const long long row = ((long long)blockIdx.x * 256 + threadIdx.x) / kTPR;
-    const bool live = row < (long long)B * T * Hq;
-    float acc = 0.f;
-    if (live && j < kChunks) {
-        const uint4 a = *reinterpret_cast<const uint4 *>(out + row * D + 8 * j);
-        const uint4 c = *reinterpret_cast<const uint4 *>(dout + row * D + 8 * j);
-        const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, cw[4] = {c.x, c.y, c.z, c.w};
+    const int j = threadIdx.x % kTPR, b = blockIdx.y;
+    const int n_rows = T * Hq;                           // rows (t, h) of sequence b
+    const int r0 = blockIdx.x * (kRowsPerPass * kPasses) + threadIdx.x / kTPR;
+    const uint16_t *ob = out + (size_t)b * n_rows * D, *gb = dout + (size_t)b * n_rows * D;
+    // every pass's loads are issued before the first is used
+    uint4 a[kPasses], c[kPasses];
+#pragma unroll
+    for (int p = 0; p < kPasses; ++p) {
+        const int r = r0 + p * kRowsPerPass;
+        if (r < n_rows && j < kChunks) {
+            a[p] = __ldcs(reinterpret_cast<const uint4 *>(ob + (size_t)r * D + 8 * j));
+            c[p] = *reinterpret_cast<const uint4 *>(gb + (size_t)r * D + 8 * j);
+        } else {
+            a[p] = c[p] = make_uint4(0u, 0u, 0u, 0u);
+        }
+    }
+#pragma unroll
+    for (int p = 0; p < kPasses; ++p) {
+        const uint32_t aw[4] = {a[p].x, a[p].y, a[p].z, a[p].w}, cw[4] = {c[p].x, c[p].y, c[p].z, c[p].w};
+        float acc = 0.f;
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             acc = fmaf(bf16lo(aw[e]), bf16lo(cw[e]), acc);
             acc = fmaf(bf16hi(aw[e]), bf16hi(cw[e]), acc);
         }
-    }
 #pragma unroll
-    for (int o = kTPR / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (live && j == 0) {
-        const int h = (int)(row % Hq);
-        const long long bt = row / Hq;
-        const int t = (int)(bt % T), b = (int)(bt / T);
-        const size_t off = ((size_t)b * Hq + h) * stride + t;
-        delta[off] = acc;
-        nl2[off] = -lse[off] * kLog2e;          // the exponent's offset, base 2
+        for (int o = kTPR / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        const int r = r0 + p * kRowsPerPass;
+        if (r < n_rows && j == 0) {
+            const int t = r / Hq, h = r - t * Hq;
+            const size_t off = ((size_t)b * Hq + h) * stride + t;
+            delta[off] = acc;
+            nl2[off] = -lse[off] * kLog2e;          // the exponent's offset, base 2
+        }
     }
 }
 
@@ -709,6 +728,14 @@ __device__ __forceinline__ void q_block(const uint32_t (&sv)[64], const uint32_t
     }
 }
 
+__device__ __forceinline__ uint4 shfl_xor_u4(uint4 v, int m) {
+    v.x = __shfl_xor_sync(0xffffffffu, v.x, m);
+    v.y = __shfl_xor_sync(0xffffffffu, v.y, m);
+    v.z = __shfl_xor_sync(0xffffffffu, v.z, m);
+    v.w = __shfl_xor_sync(0xffffffffu, v.w, m);
+    return v;
+}
+
 // thread = query row (TMEM lane); warp w takes lane quadrant w % 4 and key
 // columns [64 (w / 4), 64 (w / 4) + 64) of each tile.
 template <int D>
@@ -730,7 +757,59 @@ __device__ void q_elementwise(BwQSync &sy, uint32_t tmem, const BwGrid &g, int32
         l2 = qrow < g.T ? g.lse[off] * kLog2e : 0.f;
         dl = qrow < g.T ? g.delta[off] : 0.f;
     };
+    // Drain item (b, h, i)'s dQ: called after the next item's first key tile, so
+    // the wait for the last dQ MMA overlaps that tile's work.
+    auto drain = [&](int b, int h, int i) -> bool {
+        if (!__all_sync(0xffffffffu, ptx::mbar_wait(A(sy.acc_full), ac & 1))) return false;
+        ++ac;
+        ptx::tc_fence_after();
+        // Each lane holds 64 bytes of its own row per 32 columns.  A 4 x 4 transpose
+        // of 16-byte pieces within each group of four lanes gives lane 4m + p piece p
+        // of rows 4m .. 4m + 3, so one store writes 64 contiguous bytes of eight rows
+        // (instead of 16 bytes of 32 rows).
+        const int p = lane & 3;
+        const int row_q = i * 128 + quad * 32 + (lane & ~3);   // the group's first row
+        for (int c = half; c < D / 32; c += 2) {
+            uint32_t a[32];
+            ptx::tmem_ld32(lane_addr + Q::kColAcc + 32 * c, a);
+            ptx::tmem_wait_ld();
+            uint4 x[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                x[e] = make_uint4(pack_bf16x2(__uint_as_float(a[8 * e]) * g.scale, __uint_as_float(a[8 * e + 1]) * g.scale),
+                                  pack_bf16x2(__uint_as_float(a[8 * e + 2]) * g.scale, __uint_as_float(a[8 * e + 3]) * g.scale),
+                                  pack_bf16x2(__uint_as_float(a[8 * e + 4]) * g.scale, __uint_as_float(a[8 * e + 5]) * g.scale),
+                                  pack_bf16x2(__uint_as_float(a[8 * e + 6]) * g.scale, __uint_as_float(a[8 * e + 7]) * g.scale));
+            // stage 1 (lanes p, p ^ 1): slot 2a + r holds piece 2a + (p & 1) of row (p & 2) | r
+#pragma unroll
+            for (int pr = 0; pr < 4; pr += 2) {
+                const bool odd = p & 1;
+                const uint4 snd = odd ? x[pr] : x[pr + 1];
+                const uint4 rcv = shfl_xor_u4(snd, 1);
+                if (odd) x[pr] = rcv; else x[pr + 1] = rcv;
+            }
+            // stage 2 (lanes p, p ^ 2): slot s holds piece p of row s
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                const bool hi = p & 2;
+                const uint4 snd = hi ? x[r] : x[2 + r];
+                const uint4 rcv = shfl_xor_u4(snd, 2);
+                if (hi) x[r] = rcv; else x[2 + r] = rcv;
+            }
+#pragma unroll
+            for (int s2 = 0; s2 < 4; ++s2) {
+                const int row = row_q + s2;
+                if (row < g.T)
+                    *reinterpret_cast<uint4 *>(g.d0 + (((size_t)b * g.T + row) * g.Hq + h) * D + 32 * c + 8 * p) = x[s2];
+            }
+        }
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(A(sy.acc_empty));
+        return true;
+    };
     float nl2 = 0.f, ndl = 0.f;
+    int pb = 0, ph = 0, pi = 0;                 // the previous item
     if (bw_w(0) < g.n_items) fetch(bw_w(0), nl2, ndl);
     for (int kk = 0, w = bw_w(0); w < g.n_items && ok; w = bw_w(++kk)) {
         int b, h, i;
@@ -765,33 +844,14 @@ __device__ void q_elementwise(BwQSync &sy, uint32_t tmem, const BwGrid &g, int32
             ptx::tc_fence_before();
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(A(sy.ds_full[u & 1]));
+            if (j == 0 && kk > 0) ok = drain(pb, ph, pi);
         }
         if (!ok) break;
-        ok = __all_sync(0xffffffffu, ptx::mbar_wait(A(sy.acc_full), ac & 1));
-        if (!ok) break;
-        ++ac;
-        ptx::tc_fence_after();
-        uint16_t *dst = g.d0 + (((size_t)b * g.T + qrow) * g.Hq + h) * D;
-        for (int c = half; c < D / 32; c += 2) {
-            uint32_t a[32];
-            ptx::tmem_ld32(lane_addr + Q::kColAcc + 32 * c, a);
-            ptx::tmem_wait_ld();
-            uint32_t wq[16];
-#pragma unroll
-            for (int e = 0; e < 16; ++e)
-                wq[e] = pack_bf16x2(__uint_as_float(a[2 * e]) * g.scale,
-                                    __uint_as_float(a[2 * e + 1]) * g.scale);
-            if (qrow < g.T) {
-                uint4 *d4 = reinterpret_cast<uint4 *>(dst + 32 * c);
-#pragma unroll
-                for (int x = 0; x < 4; ++x)
-                    d4[x] = make_uint4(wq[4 * x], wq[4 * x + 1], wq[4 * x + 2], wq[4 * x + 3]);
-            }
-        }
-        ptx::tc_fence_before();
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(A(sy.acc_empty));
+        pb = b;
+        ph = h;
+        pi = i;
     }
+    if (ok && bw_w(0) < g.n_items) ok = drain(pb, ph, pi);
     if (!ok && lane == 0) report(status, GQA_DEV_TIMEOUT);
 }
 
@@ -844,6 +904,9 @@ bwd_kv_kernel(const __grid_constant__ BwMaps maps, BwGrid g, int32_t *status) {
     bw_setup(sy);
     // Delta (and the forward's outputs) come from the kernels before this one.
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    // Delta is complete: the dQ kernel, which reads nothing this kernel writes,
+    // may start on the SMs this kernel's CTAs free.
+    asm volatile("griddepcontrol.launch_dependents;");
     const uint32_t tmem = sy.tmem_base;
     if (warp >= kEwWarps) {
         ptx::regs_dec<kBwCtlRegs>();
@@ -900,7 +963,6 @@ bwd_q_kernel(const __grid_constant__ BwMaps maps, BwGrid g, int32_t *status) {
     __shared__ BwQSync sy;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     bwq_setup(sy);
-    asm volatile("griddepcontrol.wait;" ::: "memory");
     const uint32_t tmem = sy.tmem_base;
     if (warp >= kEwWarps) {
         ptx::regs_dec<kBwCtlRegs>();
@@ -915,6 +977,10 @@ bwd_q_kernel(const __grid_constant__ BwMaps maps, BwGrid g, int32_t *status) {
         ptx::regs_inc<kBwEwRegs>();
         q_elementwise<D>(sy, tmem, g, status);
     }
+    // Launched once every dK/dV CTA had seen Delta complete (no wait needed at the
+    // start); wait for the dK/dV kernel here, so this launch's end means both are
+    // done for whatever the stream runs next.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     ptx::tc_fence_before();
     __syncthreads();
     if (warp == kBwMmaWarp) {
@@ -998,15 +1064,16 @@ gqa_status launch_backward(const void *q, const void *k, const void *v, const vo
         pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
         pdl[0].val.programmaticStreamSerializationAllowed = 1;
         cudaLaunchConfig_t cfg = {};
-        const long long rows = (long long)B * T * Hq;
         const int tpr = D / 8 > 8 ? 16 : 8;
-        cfg.gridDim = dim3((unsigned)((rows * tpr + 255) / 256));
+        constexpr int kPasses = 2;             // rows per lane (4 and 8 measured slower)
+        const long long per_cta = 256 / tpr * kPasses;
+        cfg.gridDim = dim3((unsigned)(((long long)T * Hq + per_cta - 1) / per_cta), (unsigned)B);
         cfg.blockDim = dim3(256);
         cfg.stream = s;
         cfg.attrs = pdl;
         cfg.numAttrs = 1;
-        if (cudaLaunchKernelEx(&cfg, delta_kernel<D>, static_cast<const uint16_t *>(out),
-                               static_cast<const uint16_t *>(dout), lse, delta, nl2, B, T, Hq,
+        if (cudaLaunchKernelEx(&cfg, delta_kernel<D, kPasses>, static_cast<const uint16_t *>(out),
+                               static_cast<const uint16_t *>(dout), lse, delta, nl2, T, Hq,
                                ls) !=
             cudaSuccess)
             return GQA_ERR_CUDA;
@@ -1078,6 +1145,7 @@ extern "C" gqa_status gqa_attention_backward(const void *q, const void *k, const
     if (Lmax % 128 != 0) return GQA_ERR_INVALID_ARG;
     if (T > Lmax) return GQA_ERR_CAPACITY;
     if ((long long)((T + 127) / 128) * B * Hq > 0x7fffffffLL) return GQA_ERR_INVALID_ARG;
+    if ((long long)T * Hq > 0x7fffffffLL || B > 65535) return GQA_ERR_INVALID_ARG;  // Delta's grid
     const size_t need = gqa_backward_workspace_bytes(B, T, Hq);
     if (!ws || ws_bytes < need || !aligned16(ws)) return GQA_ERR_WORKSPACE;
     int dev = 0, major = 0;
