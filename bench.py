@@ -427,10 +427,10 @@ def run_ours(args, rank, world, dev, dist_on):
         "clocks": clocks,
         "device_status": status,
     }
-    line["next_rows"] = {"chunked_prefill": measure_chunk(dev, peaks, tag),
-                         "rope_scaling": measure_scaled_append(layer, peaks, tag),
-                         "doc_masked_prefill": measure_docs(layer, peaks, tag),
-                         "attention_backward": measure_backward(layer, peaks, tag)}
+    line["next_rows"] = {"chunked_prefill": with_clocks(measure_chunk, dev, peaks, tag),
+                         "rope_scaling": with_clocks(measure_scaled_append, layer, peaks, tag),
+                         "doc_masked_prefill": with_clocks(measure_docs, layer, peaks, tag),
+                         "attention_backward": with_clocks(measure_backward, layer, peaks, tag)}
     step = {"C4": {"workload": "B=8 T=2048 24q/8kv D=128, QK-norm (the timed step's prefill)",
                    "prefill_append_us": round(t_append_p / K * 1e3, 2),
                    "prefill_kernel_us": round(pf_ms * 1e3, 2),
@@ -449,6 +449,21 @@ def run_ours(args, rank, world, dev, dist_on):
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline()
     return line
+
+
+def with_clocks(measure, *args):
+    """One kernel timed alone, with its own clock record: the sampler starts, the
+    GPU idles through the sampler's start-up pause, then the measurement runs
+    (its warm-up launches included) while the clocks are sampled."""
+    sampler = ClockSampler(torch.cuda.current_device())
+    sampler.start()
+    time.sleep(0.3)
+    try:
+        row = measure(*args)
+    finally:
+        clocks = sampler.stop()
+    row["clocks"] = clocks
+    return row
 
 
 def measure_scaled_append(layer, peaks, tag, reps: int = 30):
