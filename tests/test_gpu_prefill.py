@@ -50,6 +50,8 @@ def test_named_workload_full_output(cuda_lib, name):
     (1, 385, 8, 1, 64, True),         # MQA, three pairs, ragged
     (1, 256, 4, 2, 128, False),       # T == Lmax exactly
     (3, 129, 6, 3, 96, True),         # one row into the second tile
+    (2, 300, 6, 2, 128, True),        # 3 heads per KV head, 3 tiles: items of one tile
+                                      # and two heads, of two tiles, and one single tile
 ])
 def test_shapes_and_tails(cuda_lib, B, T, Hq, Hkv, D, qk):
     w = inputs.custom("pf", B=B, Hq=Hq, Hkv=Hkv, D=D, T=T, qk_norm=qk, seed_index=T + D)

@@ -62,6 +62,7 @@ def test_decreasing_ids_are_reported(cuda_lib):
     (2, 700, 6, 2, 128, 60.0),      # many short documents, several per tile
     (2, 600, 8, 8, 96, 250.0),      # MHA, documents spanning tiles
     (3, 385, 4, 1, 64, 1000.0),     # MQA, mostly one document per row
+    (2, 300, 6, 2, 128, 90.0),      # 3 heads per KV head over 3 tiles (a single-tile item)
 ])
 def test_docs_vs_oracle(cuda_lib, B, T, Hq, Hkv, D, mean):
     w = inputs.custom("doc", B=B, Hq=Hq, Hkv=Hkv, D=D, T=T, qk_norm=True, seed_index=T + D)
