@@ -13,7 +13,8 @@
 // recomputed from the forward's row log-sum-exp, never stored.
 //
 // Three launches:
-//   delta_kernel   Delta[b, h, t] = sum_d dO * O (HBM-bound, 16-byte loads), and
+//   delta_kernel   Delta[b, h, t] = sum_d dO * O (HBM-bound, 16-byte loads, two
+//                  rows per lane), and
 //                  the exponent offset -lse[b, h, t] log2(e) the dK/dV kernel reads;
 //   bwd_kv_kernel  per (b, KV head, 128-key tile j), persistent: for every query
 //                  head of the group and every query tile i >= j, in halves of 64
@@ -34,8 +35,8 @@
 // work on the other.  The dQ kernel keeps S in two buffers and a single dP that
 // the warps release as soon as it is in registers, so S and dP of the next key
 // tile run while the warps work on this one (K and V in separate rings, 3 and 2
-// tiles deep, since K is held a step longer for dQ += dS K); the warps drain a
-// tile's dQ after the first key tile of their next item, so the wait for its
+// tiles deep, since K is held a step longer for dQ += dS K); the warps drain an
+// item's dQ after the first key tile of their next item, so the wait for its
 // last MMA overlaps that work, and they transpose 16-byte pieces within groups
 // of four lanes so each store writes 64 contiguous bytes of eight rows.
 // The same shared-memory tile serves as a K-major operand (the contraction over
@@ -43,7 +44,7 @@
 // kernel.  Warp roles (384 threads, three warpgroups): warps 0-7 elementwise +
 // epilogue (thread = TMEM lane; warps w and w + 4 share lane quadrant w and take
 // 64 of the 128 columns each; 208 registers), warp 8 TMA producer, warp 9 MMA
-// issuer, warps 10-11 idle (88 registers), as in the forward kernel.  Every mbarrier wait is
+// issuer, warps 10-11 idle (88 registers), the forward kernel's roles.  Every mbarrier wait is
 // bounded (1 s) and raises GQA_DEV_TIMEOUT; tensor memory is released only after
 // the MMA thread has seen its last MMA complete.
 #include <cuda.h>
