@@ -161,9 +161,12 @@ rope_append_kernel(uint16_t *__restrict__ q, const uint16_t *__restrict__ k,
     using S = RopeShape<D>;
     __shared__ __align__(16) float cs[TB][S::kHalf];
     __shared__ __align__(16) float sn[TB][S::kHalf];
-    // A kernel launched after this one as a programmatic dependent (the prefill
-    // or the decode) may start its prologue now; it waits for this grid to
-    // complete before it reads anything written here.
+    // Launched as a programmatic dependent of whatever precedes it on the stream
+    // (which may have produced q, k, v or pos0): wait for it before reading.  A
+    // kernel launched after this one the same way (the prefill or the decode)
+    // may then start its prologue; it waits for this grid to complete before it
+    // reads anything written here.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;");
 
     const int nblk = (T + TB - 1) / TB;
@@ -302,6 +305,7 @@ rope_append_tok_kernel(uint16_t *__restrict__ q, const uint16_t *__restrict__ k,
     using S = RopeShape<D>;
     __shared__ __align__(16) float cs[kTokWarps][S::kHalf];
     __shared__ __align__(16) float sn[kTokWarps][S::kHalf];
+    asm volatile("griddepcontrol.wait;" ::: "memory");     // as in rope_append_kernel
     asm volatile("griddepcontrol.launch_dependents;");
 
     const int nblk = (T + kTokWarps - 1) / kTokWarps;
@@ -435,17 +439,31 @@ RopeTable make_table(int D, const gqa_rope_params &p) {
     return t;
 }
 
+// A launch as a programmatic dependent of the preceding kernel on the stream: its
+// launch overlaps that kernel's last CTAs (the kernel waits for it on entry).
+template <typename K, typename... Args>
+cudaError_t launch_pdl(K kern, unsigned grid, unsigned block, cudaStream_t s, Args... args) {
+    cudaLaunchAttribute pdl[1];
+    pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.stream = s;
+    cfg.attrs = pdl;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 template <int D, int TB>
 cudaError_t launch(void *q, const void *k, const void *v, void *kc, void *vc,
                    const int32_t *pos0, int32_t *new_len, int B, int T, int Hq, int Hkv,
                    int Lmax, const gqa_rope_params &p, int32_t *status, cudaStream_t s) {
     const unsigned grid = (unsigned)B * (unsigned)((T + TB - 1) / TB);
-    rope_append_kernel<D, TB><<<grid, kThreads, 0, s>>>(
-        static_cast<uint16_t *>(q), static_cast<const uint16_t *>(k),
-        static_cast<const uint16_t *>(v), static_cast<uint16_t *>(kc),
-        static_cast<uint16_t *>(vc), pos0, new_len, T, Hq, Hkv, Lmax, p.qk_norm, p.eps,
-        make_table(D, p), status);
-    return cudaGetLastError();
+    return launch_pdl(rope_append_kernel<D, TB>, grid, kThreads, s, static_cast<uint16_t *>(q),
+                      static_cast<const uint16_t *>(k), static_cast<const uint16_t *>(v),
+                      static_cast<uint16_t *>(kc), static_cast<uint16_t *>(vc), pos0, new_len, T,
+                      Hq, Hkv, Lmax, p.qk_norm, p.eps, make_table(D, p), status);
 }
 
 template <int D>
@@ -457,12 +475,11 @@ cudaError_t launch_tb(void *q, const void *k, const void *v, void *kc, void *vc,
     // tokens over enough warps.
     if (T >= kTokWarps) {
         const unsigned grid = (unsigned)B * (unsigned)((T + kTokWarps - 1) / kTokWarps);
-        rope_append_tok_kernel<D><<<grid, kTokWarps * 32, 0, s>>>(
-            static_cast<uint16_t *>(q), static_cast<const uint16_t *>(k),
-            static_cast<const uint16_t *>(v), static_cast<uint16_t *>(kc),
-            static_cast<uint16_t *>(vc), pos0, new_len, T, Hq, Hkv, Lmax, p.qk_norm, p.eps,
-            make_table(D, p), status);
-        return cudaGetLastError();
+        return launch_pdl(rope_append_tok_kernel<D>, grid, kTokWarps * 32, s,
+                          static_cast<uint16_t *>(q), static_cast<const uint16_t *>(k),
+                          static_cast<const uint16_t *>(v), static_cast<uint16_t *>(kc),
+                          static_cast<uint16_t *>(vc), pos0, new_len, T, Hq, Hkv, Lmax,
+                          p.qk_norm, p.eps, make_table(D, p), status);
     }
     return launch<D, 1>(q, k, v, kc, vc, pos0, new_len, B, T, Hq, Hkv, Lmax, p, status, s);
 }
