@@ -43,6 +43,29 @@ def test_named_workload_full_output(cuda_lib, name):
     assert_floor_close(o, exact, ideal, W, name)
 
 
+def _sweep_shapes(n, seed):
+    """n seeded small shapes (B <= 3, T <= 420, 1-6 query heads per KV head,
+    D in {64, 96, 128}), for the pairing of (query tile, head) tiles into items:
+    odd and even tile counts, single-tile items, T below one tile."""
+    r = np.random.default_rng(seed)
+    out = []
+    for _ in range(n):
+        G = int(r.choice([1, 2, 3, 4, 6]))
+        Hkv = int(r.integers(1, 4))
+        out.append((int(r.integers(1, 4)), int(r.integers(1, 421)), G * Hkv, Hkv,
+                    int(r.choice([64, 96, 128])), bool(r.integers(0, 2))))
+    return out
+
+
+@pytest.mark.parametrize("B,T,Hq,Hkv,D,qk", _sweep_shapes(10, 2026))
+def test_seeded_shape_sweep(cuda_lib, B, T, Hq, Hkv, D, qk):
+    w = inputs.custom("pf", B=B, Hq=Hq, Hkv=Hkv, D=D, T=T, qk_norm=qk, seed_index=3 * T + D)
+    x = inputs.make_inputs(w)
+    o = _run_phase(x, w)
+    exact, ideal, W = prompt_refs(bits(x["q"]), bits(x["k"]), bits(x["v"]), qk)
+    assert_floor_close(o, exact, ideal, W, "sweep B%d T%d Hq%d Hkv%d D%d" % (B, T, Hq, Hkv, D))
+
+
 @pytest.mark.parametrize("B,T,Hq,Hkv,D,qk", [
     (2, 1, 4, 2, 64, False),          # a single token
     (1, 200, 6, 2, 128, True),        # ragged second tile

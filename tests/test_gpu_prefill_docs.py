@@ -76,6 +76,30 @@ def test_docs_vs_oracle(cuda_lib, B, T, Hq, Hkv, D, mean):
     assert_floor_close(o, exact, ideal, W, "documents B%d T%d D%d mean %g" % (B, T, D, mean))
 
 
+def _sweep_shapes(n, seed):
+    """n seeded small shapes with a mean document length each (B <= 3, T <= 420,
+    1-6 query heads per KV head, D in {64, 96, 128})."""
+    r = np.random.default_rng(seed)
+    out = []
+    for _ in range(n):
+        G = int(r.choice([1, 2, 3, 4, 6]))
+        Hkv = int(r.integers(1, 4))
+        out.append((int(r.integers(1, 4)), int(r.integers(1, 421)), G * Hkv, Hkv,
+                    int(r.choice([64, 96, 128])), float(r.choice([20.0, 100.0, 400.0]))))
+    return out
+
+
+@pytest.mark.parametrize("B,T,Hq,Hkv,D,mean", _sweep_shapes(6, 2027))
+def test_docs_seeded_shape_sweep(cuda_lib, B, T, Hq, Hkv, D, mean):
+    w = inputs.custom("doc", B=B, Hq=Hq, Hkv=Hkv, D=D, T=T, qk_norm=True, seed_index=5 * T + D)
+    x = inputs.make_inputs(w)
+    ids = inputs.packed_doc_ids(B, T, mean, seed=7 * T + Hq)
+    o = _run_docs(x, w, ids)
+    exact, ideal, W = prompt_refs(bits(x["q"]), bits(x["k"]), bits(x["v"]), True,
+                                  doc_id=ids.numpy())
+    assert_floor_close(o, exact, ideal, W, "documents sweep B%d T%d Hq%d Hkv%d D%d" % (B, T, Hq, Hkv, D))
+
+
 def test_one_document_is_prefill_bit_for_bit(cuda_lib):
     w = inputs.custom("doc", B=2, Hq=6, Hkv=2, D=128, T=500, qk_norm=True, seed_index=91)
     x = inputs.make_inputs(w)
