@@ -724,13 +724,13 @@ def measure_chunk(dev, peaks, tag, reps: int = 30):
 # ---------------------------------------------------------------------------
 # the oracle on the host cores (reported baseline / reference arm)
 # ---------------------------------------------------------------------------
-_BASELINE_INPUTS = []
+_CPU_BASELINE_INPUTS = []
 
 
 def _baseline_inputs():
-    if not _BASELINE_INPUTS:
-        _BASELINE_INPUTS.append((inputs.make_inputs(PREFILL), inputs.make_inputs(DECODE)))
-    return _BASELINE_INPUTS[0]
+    if not _CPU_BASELINE_INPUTS:
+        _CPU_BASELINE_INPUTS.append((inputs.make_inputs(PREFILL), inputs.make_inputs(DECODE)))
+    return _CPU_BASELINE_INPUTS[0]
 
 
 def oracle_step(nthreads: int = 0) -> float:
