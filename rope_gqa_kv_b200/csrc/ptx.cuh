@@ -107,7 +107,7 @@ __device__ __forceinline__ uint64_t policy_evict_last() {
     return p;
 }
 
-// 2-D tiled tensor load (no multicast); coordinates innermost first.
+// 2-D tiled tensor load into this CTA's shared memory; coordinates innermost first.
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, uint32_t bar,
                                             int c0, int c1) {
     asm volatile(
@@ -117,7 +117,7 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
         : "memory");
 }
 
-// 3-D tiled tensor load (no multicast); coordinates innermost first.
+// 3-D tiled tensor load into this CTA's shared memory; coordinates innermost first.
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, uint32_t bar,
                                             int c0, int c1, int c2) {
     asm volatile(
@@ -137,7 +137,7 @@ __device__ __forceinline__ void tma_load_3d_hint(uint32_t dst, const CUtensorMap
         : "memory");
 }
 
-// 4-D tiled tensor load (no multicast).
+// 4-D tiled tensor load into this CTA's shared memory.
 __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap *map, uint32_t bar,
                                             int c0, int c1, int c2, int c3) {
     asm volatile(
