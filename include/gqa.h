@@ -143,8 +143,9 @@ gqa_status gqa_rope_append(void *q, const void *k, const void *v, void *k_cache,
  * never read).  Tensor-core kernel (tcgen05 / TMEM, TMA-fed), fp32 softmax.
  *   T <= Lmax.  Alignment: 16 bytes for every pointer.
  * Device errors: GQA_DEV_TIMEOUT (a bounded pipeline wait expired).
- * Scheduling: with four or more query-tile pairs per SM, the CTAs take pairs
- * from a counter in device memory (one of 256 slots per device, taken round
+ * Scheduling: work items are pairs of 128-row query tiles that share a KV
+ * head (two heads of one tile, or two consecutive tiles); with four or more
+ * items per SM, the CTAs take items from a counter in device memory (one of 256 slots per device, taken round
  * robin by each call and reset by its last CTA), so up to 256 calls of
  * gqa_prefill, _chunk, _docs or _lse may be in flight on a device at once; a
  * CUDA graph replays the slot it captured, so replays of one graph must not
