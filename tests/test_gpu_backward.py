@@ -128,3 +128,31 @@ def test_slots_past_t_untouched_and_deterministic(cuda_lib):
     _, _, (dq2, dk2, dv2) = _run(q, dout, kc, vc, dk=sentinel.clone(), dv=sentinel.clone())
     for a, b in ((dq1, dq2), (dk1, dk2), (dv1, dv2)):
         assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+def test_back_to_back_calls_share_a_workspace(cuda_lib):
+    """Five backward calls on one stream with no synchronisation between them,
+    one workspace, a different output gradient each time and the results read
+    only at the end: each call's three launches are programmatic dependents
+    (the dQ launch starts while the dK/dV launch still runs, and waits for it
+    before it ends), so a call must not overwrite the workspace's Delta while
+    the call before still reads it, and each result must equal that of the same
+    call run alone, bit for bit."""
+    B, T, Hq, Hkv, D = 2, 700, 6, 2, 128
+    q, _, _, _, kc, vc = _case(B, T, Hq, Hkv, D, seed=77)
+    dq_, dkc, dvc = q.to(DEV), kc.to(DEV), vc.to(DEV)
+    o, lse = gqa.gqa_prefill_lse(dq_, dkc, dvc)
+    g = torch.Generator().manual_seed(78)
+    douts = [torch.randn(B, T, Hq, D, generator=g).to(torch.bfloat16).to(DEV) for _ in range(5)]
+    ws = torch.empty(gqa.gqa_backward_workspace_bytes(B, T, Hq), dtype=torch.uint8, device=DEV)
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    torch.cuda.synchronize()
+    chained = [gqa.gqa_attention_backward(dq_, dkc, dvc, o, d, lse, workspace=ws, status=st)
+               for d in douts]
+    torch.cuda.synchronize()
+    assert st.item() == 0, "device status %#x" % st.item()
+    for i, d in enumerate(douts):
+        alone = gqa.gqa_attention_backward(dq_, dkc, dvc, o, d, lse)
+        torch.cuda.synchronize()
+        for a, b, name in zip(chained[i], alone, ("dq", "dk", "dv")):
+            assert torch.equal(a.view(torch.int16), b.view(torch.int16)), "call %d: %s differs" % (i, name)
