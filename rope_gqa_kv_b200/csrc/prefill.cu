@@ -112,7 +112,7 @@ struct PfMaps {
 
 struct PfSync {
     uint64_t item_full[4], item_empty[4];   // the CTA's item ring (producer -> the other roles)
-    int item[4][6];                         // item number (-1: no more), then its PfSeq
+    int item[4][16];                        // item number (-1: no more), then its PfItem
     uint64_t q_full, q_empty;
     uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
     uint64_t s_full[2], p_half[2], p_full[2], o_final[2];
@@ -151,8 +151,9 @@ struct PfGrid {
 // Items are dealt out dynamically: the producer takes the next item number from
 // the launch's counter when it starts loading that item, i.e. once it has issued
 // every load of the item before (items are numbered longest first, so this is
-// greedy longest-first scheduling), reads the item's sequence data, and passes
-// both to the CTA's other roles through a four-slot ring in shared memory.
+// greedy longest-first scheduling), reads the item's sequence data, decodes
+// the item and passes it to the CTA's other roles through a four-slot ring in
+// shared memory.
 // (Static dealing left the CTAs' finish times max/mean 1.05 apart on a prompt
 // and 1.17 on documents and chunks.)  Item number -1 marks the end.
 constexpr int kItemReaders = 9;        // the 8 softmax warps and the MMA warp
@@ -262,16 +263,48 @@ __device__ __forceinline__ PfItem pf_item(int w, const PfGrid &g, PfSeq sq) {
     return it;
 }
 
-// The x-th item of this CTA and its sequence data, read from the ring (waits
-// for the producer); a wait that times out reads as the end.
-__device__ __forceinline__ int pf_item_at(PfSync &sy, int x, PfSeq &q) {
+// The producer decodes each item once and passes the result through the ring:
+// decoding takes a chain of integer divisions, and in the softmax and MMA warps
+// that chain sat on the item boundary's critical path (about 0.3 us per item
+// at the 8 x 2048 prompt, waiting behind the exponentials for the SFU).
+__device__ __forceinline__ void pf_item_put(volatile int *e, int w, const PfItem &I) {
+    e[0] = w;
+    e[1] = I.b;
+    e[2] = I.h;
+    e[3] = I.kvh;
+    e[4] = I.q0;
+    e[5] = I.n0;
+    e[6] = I.n1;
+    e[7] = I.n_kv;
+    e[8] = I.h1;
+    e[9] = I.q1;
+    e[10] = I.lo0;
+    e[11] = I.lo1;
+    e[12] = I.P;
+    e[13] = I.N;
+    e[14] = I.r_valid;
+    e[15] = I.has1 ? 1 : 0;
+}
+// The x-th item of this CTA, decoded, read from the ring (waits for the
+// producer); a wait that times out reads as the end.
+__device__ __forceinline__ int pf_item_at(PfSync &sy, int x, PfItem &I) {
     if (!ptx::mbar_wait_warp(A(sy.item_full[x & 3]), (x >> 2) & 1)) return -1;
     const volatile int *e = sy.item[x & 3];
-    q.P = e[1];
-    q.N = e[2];
-    q.lo0 = e[3];
-    q.lo1 = e[4];
-    q.bad = e[5] != 0;
+    I.b = e[1];
+    I.h = e[2];
+    I.kvh = e[3];
+    I.q0 = e[4];
+    I.n0 = e[5];
+    I.n1 = e[6];
+    I.n_kv = e[7];
+    I.h1 = e[8];
+    I.q1 = e[9];
+    I.lo0 = e[10];
+    I.lo1 = e[11];
+    I.P = e[12];
+    I.N = e[13];
+    I.r_valid = e[14];
+    I.has1 = e[15] != 0;
     return e[0];
 }
 
@@ -292,17 +325,11 @@ __device__ void producer(const PfMaps &maps, PfSync &sy, uint8_t *smem, const Pf
         int w = dynamic ? atomicAdd(g.work, 1) : pf_static_w<kMode>(k);
         if (w >= g.n_items) w = -1;
         const PfSeq sq = w >= 0 ? pf_seq<kMode>(g, w) : pf_seq_none();
-        volatile int *e = sy.item[s];
-        e[0] = w;
-        e[1] = sq.P;
-        e[2] = sq.N;
-        e[3] = sq.lo0;
-        e[4] = sq.lo1;
-        e[5] = sq.bad ? 1 : 0;
+        const PfItem I = pf_item(w >= 0 ? w : 0, g, sq);
+        pf_item_put(sy.item[s], w, I);
         ptx::mbar_arrive(A(sy.item_full[s]));
         if (w < 0) break;
         if (sq.bad) report(status, sq.P < 0 || sq.N < 0 ? GQA_DEV_BAD_LEN : GQA_DEV_CAPACITY);
-        const PfItem I = pf_item(w, g, sq);
         if (I.n_kv == 0) continue;
         // The previous item's last S MMA has released the Q tiles.
         ok = ptx::mbar_wait(A(sy.q_empty), (qc & 1) ^ 1);
@@ -400,12 +427,11 @@ __device__ void mma_issuer(PfSync &sy, uint8_t *smem, uint32_t tmem, const PfGri
     int pc0 = 0, pc1 = 0;           // P hand-overs received from each softmax group
     bool ok = true;
     for (int k = 0; ok; ++k) {
-        PfSeq sq;
-        const int w = pf_item_at(sy, k, sq);
+        PfItem I;
+        const int w = pf_item_at(sy, k, I);
         __syncwarp();
         if (w < 0) break;
         if (go) ptx::mbar_arrive(A(sy.item_empty[k & 3]));   // the ring slot has been read
-        const PfItem I = pf_item(w, g, sq);
         if (I.n_kv == 0) continue;
         const int kc0 = kc;           // K ring index of key tile lo0
         ok = ptx::mbar_wait_warp(A(sy.q_full), qc & 1) &&
@@ -494,12 +520,11 @@ __device__ void softmax_tile(const PfMaps &maps, PfSync &sy, uint8_t *smem, uint
     int vc = 0;                     // V tiles of the items before this one
     bool ok = true;
     for (int k = 0; ok; ++k) {
-        PfSeq sq;
-        const int w = pf_item_at(sy, k, sq);
+        PfItem I;
+        const int w = pf_item_at(sy, k, I);
         __syncwarp();
         if (w < 0) break;
         if (lane == 0) ptx::mbar_arrive(A(sy.item_empty[k & 3]));   // the ring slot has been read
-        const PfItem I = pf_item(w, g, sq);
         const int vc0 = vc;
         vc += I.n_kv - I.lo0;
         if (I.n_kv == 0 || (t == 1 && !I.has1)) continue;
