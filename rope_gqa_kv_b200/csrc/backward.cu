@@ -421,9 +421,11 @@ __device__ void kv_elementwise(const BwMaps &maps, BwSync &sy, uint8_t *smem, ui
         kv_item(w, g, b, kvh, j);
         const int key = j * 128 + r;
         const int n_half = 2 * grp * (g.nT - j);
-        for (int x = 0; x < n_half && ok; ++x) {
+        // half x is the (x & 1) half of query tile i, which runs j .. nT - 1 once
+        // per query head of the group (counted, not divided: a division here
+        // waits on the special-function unit behind the exponentials)
+        for (int x = 0, i = j; x < n_half && ok; i = (x & 1) ? (i + 1 == g.nT ? j : i + 1) : i, ++x) {
             const int u = hc + x;
-            const int i = j + (x / 2) % (g.nT - j);
             const int st = (sc + x / 2) % S::kStages;
             ok = __all_sync(0xffffffffu, ptx::mbar_wait(A(sy.h_full[u & 1]), (u >> 1) & 1));
             if (!ok) break;
