@@ -27,6 +27,13 @@ steps together in the order the pages give them:
   the chain rule through softmax written out with numpy matrix products.
 
 Inputs are bfloat16 bit patterns (``numpy.uint16``), widened exactly to float64.
+
+Parity unpinned (conventions no page fixes, declared rather than pinned):
+the interior of YaRN's ramp between alpha and beta (``RopeScaling``: taken
+continuous in r; its limits, temperature and the other methods are pinned),
+the RoPE pairing (halves; the oracle implements both pairings, each pinned to
+the complex-number form), and the contiguous head grouping h -> h // g
+(pinned against torch's SDPA with ``repeat_interleave``).
 """
 from __future__ import annotations
 
